@@ -1,0 +1,400 @@
+"""Benchmark of the quantized-KV decode hot path on B200.
+
+One step = one decode token through every layer of the workload: for each
+layer, quantize-on-append of the new token's K/V rows (kvq_append_quantize),
+split-KV decode over the whole cache (kvq_decode_attention) and the split
+combine (kvq_combine).  Default workload: Llama-3.1-70B-shaped cache, 80
+layers, 64 query / 8 KV heads, head_dim 128, context 32768, batch 4,
+K q8_0 / V q4_0 (~17.4 GB of quantized cache, every layer a distinct 218 MB
+buffer, so nothing stays in the 126 MB L2 between layers).
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+instead, on a bounded sample of the same workload.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-KV decode attention: achieved HBM GB/s (% of peak), µs/layer-step"
+UNIT = "GB/s"
+DEFAULT_WORKLOAD = "llama70b_ctx32k_b4"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (0 = workload's)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def row_bytes(kind, d):
+    from decode_attention_q8_b200 import kvq_row_bytes
+    return kvq_row_bytes(kind, d)
+
+
+def algorithmic_bytes(w, n_layers):
+    """Bytes the step must move at minimum, per the format definitions:
+    decode reads every cached row once (codes + scales) and the queries and
+    writes the fp32 outputs; append reads the new fp16 rows and writes their
+    cache rows."""
+    rk, rv = row_bytes(w.k_type, w.head_dim), row_bytes(w.v_type, w.head_dim)
+    decode = w.batch * w.n_kv * w.ctx * (rk + rv) + w.batch * w.n_q * w.head_dim * (2 + 4)
+    append = w.batch * w.n_kv * (2 * w.head_dim * 2 + rk + rv)
+    return decode, append, n_layers * (decode + append)
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index, enabled=True):
+        self.proc = None
+        self.idx = device_index
+        if enabled:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={device_index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                     "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = max(smax, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, seconds=10.0, max_units=None):
+    """Times the oracle's decode step (append the new row, dequantize the cached
+    rows, fp64 attention) on whole (batch row, KV head) units of one layer, as
+    many as fit in about `seconds`; returns (GB/s, units, seconds, threads)."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+    import synth
+    from oracle import attention, blocks, turbo3
+
+    def quant(kind, x, seed):
+        if kind == "q8_0":
+            return blocks.quantize_q8_0(x)
+        if kind == "q4_0":
+            return blocks.quantize_q4_0(x)
+        if kind == "turbo3":
+            return turbo3.quantize_turbo3(x, seed)
+        return None, x
+
+    def deq(kind, s, c, seed):
+        if kind == "q8_0":
+            return blocks.dequantize_q8_0(s, c)
+        if kind == "q4_0":
+            return blocks.dequantize_q4_0(s, c)
+        if kind == "turbo3":
+            return turbo3.dequantize_turbo3(s, c, seed, w.head_dim)
+        return blocks.dequantize_f16(c)
+
+    G = w.n_q // w.n_kv
+    q, k, v = synth.layer_inputs(w, layer=0, device="cpu", batch=1)
+    q, k, v = q.numpy(), k.numpy(), v.numpy()
+    units = []
+    for g in range(w.n_kv):
+        ks, kc = quant(w.k_type, k[0, :, g, :], w.turbo_seed)
+        vs, vc = quant(w.v_type, v[0, :, g, :], w.turbo_seed)
+        units.append((q[0, g * G:(g + 1) * G], k[0, -1:, g, :], v[0, -1:, g, :], ks, kc, vs, vc))
+    limit = max_units or 4 * len(units)
+    done, t_total = 0, 0.0
+    with threadpool_limits(limits=1):
+        while done < limit and t_total < seconds:
+            qg, kn, vn, ks, kc, vs, vc = units[done % len(units)]
+            t0 = time.perf_counter()
+            quant(w.k_type, kn, w.turbo_seed)
+            quant(w.v_type, vn, w.turbo_seed)
+            kh = deq(w.k_type, ks, kc, w.turbo_seed)
+            vh = deq(w.v_type, vs, vc, w.turbo_seed)
+            attention.decode_attention(qg[None].astype(np.float64), kh[None, None], vh[None, None], w.scale)
+            t_total += time.perf_counter() - t0
+            done += 1
+    rk, rv = row_bytes(w.k_type, w.head_dim), row_bytes(w.v_type, w.head_dim)
+    unit_bytes = w.ctx * (rk + rv) + G * w.head_dim * 6 + 2 * w.head_dim * 2 + rk + rv
+    return done * unit_bytes / t_total / 1e9, done, t_total, 1
+
+
+def run_reference(args):
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    gbs, units, secs, cores = oracle_sample(w, seconds=max(3.0, 2.0 * (args.steps + args.warmup)))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 6), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(w, args, None),
+        "cpu_baseline": {"value": round(gbs, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{units} (batch row, KV head) units of layer 0, ctx {w.ctx}, "
+                                   f"{secs:.1f} s, 1 BLAS thread"},
+        "e2e": {"value": round(gbs, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _config(w, args, n_layers):
+    return {"workload": w.name, "layers": n_layers or w.layers, "batch": w.batch, "n_q_heads": w.n_q,
+            "n_kv_heads": w.n_kv, "head_dim": w.head_dim, "ctx": w.ctx, "k_type": w.k_type,
+            "v_type": w.v_type, "step": "per layer: append 1 row + split decode + combine",
+            "l2": "inputs larger than L2: every layer a distinct cache buffer larger than the 126 MB L2"}
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def run_kvq(args):
+    import torch
+    import torch.distributed as dist
+
+    import decode_attention_q8_b200 as kvq
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = synth.WORKLOADS[args.workload]
+    L = args.layers or w.layers
+    desc = kvq.make_desc(w.n_q, w.n_kv, w.head_dim, w.k_type, w.v_type, w.ctx, turbo_seed=w.turbo_seed)
+    B, ctx = w.batch, w.ctx
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- caches: prefill every layer with its own seeded rows (timed: bulk append)
+    kcs, vcs, qs, kn, vn = [], [], [], [], []
+    pre_ev = []
+    for layer in range(L):
+        q, k, v = synth.layer_inputs(w, layer=layer + 1000 * rank, device=dev)
+        kc = torch.empty(kvq.kvq_cache_bytes(desc, B, 0), dtype=torch.uint8, device=dev)
+        vc = torch.empty(kvq.kvq_cache_bytes(desc, B, 1), dtype=torch.uint8, device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kvq.kvq_append_quantize(desc, kc, vc, k, v, B, 0, ctx, stream)
+        e1.record(stream)
+        pre_ev.append((e0, e1))
+        kcs.append(kc)
+        vcs.append(vc)
+        qs.append(q)
+        kn.append(k[:, ctx - 1:ctx].contiguous())
+        vn.append(v[:, ctx - 1:ctx].contiguous())
+        del k, v
+    torch.cuda.synchronize()
+    prefill_ms = [a.elapsed_time(b) for a, b in pre_ev[1:]] or [pre_ev[0][0].elapsed_time(pre_ev[0][1])]
+    torch.cuda.empty_cache()
+
+    S = kvq.kvq_auto_splits(desc, B, ctx)
+    ws = torch.empty(kvq.kvq_workspace_bytes(desc, B, 0), dtype=torch.uint8, device=dev)
+    outs = [torch.empty((B, w.n_q, w.head_dim), dtype=torch.float32, device=dev) for _ in range(L)]
+    scale = w.scale
+
+    dec_events = []
+
+    def step(record=False):
+        for layer in range(L):
+            kvq.kvq_append_quantize(desc, kcs[layer], vcs[layer], kn[layer], vn[layer], B, ctx - 1, 1, stream)
+            if record:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+            kvq.kvq_decode_attention(desc, kcs[layer], vcs[layer], qs[layer], B, ctx, scale, 0, ws, stream=stream)
+            if record:
+                b.record(stream)
+                dec_events.append((a, b))
+            kvq.kvq_combine(desc, ws, B, ctx, 0, outs[layer], stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    clocks = ClockSampler(local, enabled=not args.no_clocks)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(record=True)
+    t_end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    dec_ms = [a.elapsed_time(b) for a, b in dec_events]
+
+    # ---- end to end through the public API with host buffers
+    q_h = [torch.empty_like(x, device="cpu").pin_memory() for x in qs]
+    kn_h = [x.cpu().pin_memory() for x in kn]
+    vn_h = [x.cpu().pin_memory() for x in vn]
+    for i, x in enumerate(qs):
+        q_h[i].copy_(x)
+    out_h = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
+    qd = [torch.empty_like(x) for x in qs]
+    knd = [torch.empty_like(x) for x in kn]
+    vnd = [torch.empty_like(x) for x in vn]
+
+    def e2e_step():
+        for layer in range(L):
+            qd[layer].copy_(q_h[layer], non_blocking=True)
+            knd[layer].copy_(kn_h[layer], non_blocking=True)
+            vnd[layer].copy_(vn_h[layer], non_blocking=True)
+            kvq.kvq_append_quantize(desc, kcs[layer], vcs[layer], knd[layer], vnd[layer], B, ctx - 1, 1, stream)
+            kvq.kvq_decode_attention(desc, kcs[layer], vcs[layer], qd[layer], B, ctx, scale, 0, ws, stream=stream)
+            kvq.kvq_combine(desc, ws, B, ctx, 0, outs[layer], stream=stream)
+            out_h[layer].copy_(outs[layer], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    # ---- max over ranks
+    vals = torch.tensor([ms, e2e_ms, statistics.mean(dec_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms, e2e_ms, dec_avg = vals.tolist()
+
+    dec_bytes, app_bytes, step_bytes = algorithmic_bytes(w, L)
+    value = world * step_bytes * args.steps / (ms * 1e-3) / 1e9
+    e2e_value = world * step_bytes * args.steps / (e2e_ms * 1e-3) / 1e9
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except OSError:
+        pass
+    peak = peaks.get("hbm_gbs")
+    peak_src = "measured" if peak else "fallback"
+    peak = peak or 6650.0
+    achieved = dec_bytes / (dec_avg * 1e-3) / 1e9
+    ms_step = ms / args.steps
+    traffic = _profiled_traffic(w.name)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": _config(w, args, L),
+            "us_per_layer_step": round(1e3 * ms_step / L, 3),
+            "tokens_per_s": round(world * B * 1e3 / ms_step, 2),
+            "frac_of_8tbs": round(value / 8000.0, 4),
+            "splits": S,
+            "roofline": {"bound": "hbm", "kernel": "decode split kernel", "achieved": round(achieved, 2),
+                         "peak": peak, "peak_source": f"{peak_src} copy bandwidth", "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "algorithmic_bytes_per_launch": dec_bytes,
+                         "avg_launch_us": round(dec_avg * 1e3, 3)},
+            "e2e": {"value": round(e2e_value, 3), "unit": UNIT,
+                    "h2d_bytes_per_step": L * (qs[0].numel() * 2 + kn[0].numel() * 2 + vn[0].numel() * 2),
+                    "d2h_bytes_per_step": L * outs[0].numel() * 4},
+            "gpu_launches": args.steps * L * (2 + 1 + 1),
+            "append_bulk": {"rows_per_layer": B * ctx * w.n_kv, "us_per_layer": round(1e3 * statistics.median(prefill_ms), 2),
+                            "GB_per_s": round((B * w.n_kv * ctx * (2 * w.head_dim * 2 + row_bytes(w.k_type, w.head_dim)
+                                                                     + row_bytes(w.v_type, w.head_dim)))
+                                              / (statistics.median(prefill_ms) * 1e-3) / 1e9, 2)},
+        }
+        if clk:
+            line["clocks"] = clk
+        if not args.no_cpu_baseline and world == 1:
+            gbs, units, secs, cores = oracle_sample(w, seconds=10.0)
+            line["cpu_baseline"] = {"value": round(gbs, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                                    "sample": f"{units} (batch row, KV head) units of one layer (ctx {w.ctx}), "
+                                              f"{secs:.1f} s, 1 BLAS thread"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+
+
+def _decode_source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "decode_attention_q8_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.startswith("decode"):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic(name):
+    """DRAM bytes per decode launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from the committed ncu summary, scaled to this workload, or None when no
+    summary was taken of the decode kernel as it is now (source hash differs)."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.txt")
+    try:
+        lines = open(p).read().splitlines()
+    except OSError:
+        return None
+    sha = _decode_source_sha()
+    for line in lines:
+        f = line.split()
+        if len(f) == 3 and f[0] == name and f[2] == sha:
+            return int(f[1])
+    return None
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_kvq(args)
+
+
+if __name__ == "__main__":
+    main()

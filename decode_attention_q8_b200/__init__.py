@@ -1,0 +1,204 @@
+"""Python binding of libkvq (quantized-KV decode attention for B200).
+
+Argument marshalling only: every entry point forwards to the C ABI declared in
+``include/kvq.h`` under the same name, passing raw device pointers and a CUDA
+stream handle.  All work runs in the library's CUDA kernels; there is no
+Python or CPU implementation behind these functions.  Importing fails loudly
+when the compiled library is missing.
+
+Pointers may be given as ``torch.Tensor`` (its ``data_ptr()``), as ``None``
+(NULL) or as a plain integer address; streams as ``torch.cuda.Stream``, an
+integer handle, or ``None`` for the current torch stream.
+"""
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libkvq.so not found at {LIB_PATH}; build it with "
+        "`python -m decode_attention_q8_b200.build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+KVQ_F16, KVQ_Q8_0, KVQ_Q4_0, KVQ_TURBO3 = 0, 1, 2, 3
+TYPES = {"f16": KVQ_F16, "q8_0": KVQ_Q8_0, "q4_0": KVQ_Q4_0, "turbo3": KVQ_TURBO3}
+
+KVQ_OK, KVQ_ERR_INVALID, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA = 0, 1, 2, 3, 4
+
+EXPORTED = (
+    "kvq_status_string", "kvq_last_cuda_error", "kvq_row_bytes", "kvq_check_desc",
+    "kvq_cache_layout", "kvq_cache_bytes", "kvq_auto_splits", "kvq_workspace_bytes",
+    "kvq_turbo3_codebook", "kvq_turbo3_signs", "kvq_append_quantize",
+    "kvq_decode_attention", "kvq_combine",
+)
+
+
+class kvq_cache_desc(ctypes.Structure):
+    _fields_ = [
+        ("n_q_heads", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("k_type", ctypes.c_int32),
+        ("v_type", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("max_ctx", ctypes.c_int64),
+        ("turbo_seed", ctypes.c_uint64),
+    ]
+
+
+class kvq_plane_layout(ctypes.Structure):
+    _fields_ = [
+        ("rows_per_plane", ctypes.c_int64),
+        ("code_bytes", ctypes.c_int64),
+        ("n_scales", ctypes.c_int64),
+        ("scale_offset", ctypes.c_int64),
+        ("total_bytes", ctypes.c_int64),
+    ]
+
+
+_P = ctypes.c_void_p
+_D = ctypes.POINTER(kvq_cache_desc)
+_sigs = {
+    "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "kvq_last_cuda_error": (ctypes.c_char_p, []),
+    "kvq_row_bytes": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int32]),
+    "kvq_check_desc": (ctypes.c_int, [_D]),
+    "kvq_cache_layout": (ctypes.c_int, [_D, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(kvq_plane_layout)]),
+    "kvq_cache_bytes": (ctypes.c_size_t, [_D, ctypes.c_int32, ctypes.c_int32]),
+    "kvq_auto_splits": (ctypes.c_int32, [_D, ctypes.c_int32, ctypes.c_int64]),
+    "kvq_workspace_bytes": (ctypes.c_size_t, [_D, ctypes.c_int32, ctypes.c_int32]),
+    "kvq_turbo3_codebook": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
+    "kvq_turbo3_signs": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]),
+    "kvq_append_quantize": (ctypes.c_int, [_D, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int64,
+                                           ctypes.c_int32, _P]),
+    "kvq_decode_attention": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                                            ctypes.c_int32, _P, ctypes.c_size_t, _P]),
+    "kvq_combine": (ctypes.c_int, [_D, _P, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                                   _P, _P]),
+}
+for _name, (_res, _args) in _sigs.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class KvqError(RuntimeError):
+    def __init__(self, status, where):
+        msg = _lib.kvq_status_string(status).decode()
+        if status == KVQ_ERR_CUDA:
+            msg += ": " + _lib.kvq_last_cuda_error().decode()
+        super().__init__(f"{where}: {msg}")
+        self.status = status
+
+
+def _check(status, where):
+    if status != KVQ_OK:
+        raise KvqError(status, where)
+    return status
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _type(t):
+    return TYPES[t] if isinstance(t, str) else int(t)
+
+
+def make_desc(n_q_heads, n_kv_heads, head_dim, k_type, v_type, max_ctx, turbo_seed=0):
+    return kvq_cache_desc(n_q_heads, n_kv_heads, head_dim, _type(k_type), _type(v_type), 0,
+                          max_ctx, turbo_seed)
+
+
+# ----------------------------------------------------------------- queries
+
+def kvq_status_string(status):
+    return _lib.kvq_status_string(status).decode()
+
+
+def kvq_row_bytes(type_, head_dim):
+    return _lib.kvq_row_bytes(_type(type_), head_dim)
+
+
+def kvq_check_desc(desc):
+    return _lib.kvq_check_desc(ctypes.byref(desc))
+
+
+def kvq_cache_layout(desc, batch, which):
+    out = kvq_plane_layout()
+    _check(_lib.kvq_cache_layout(ctypes.byref(desc), batch, which, ctypes.byref(out)), "kvq_cache_layout")
+    return out
+
+
+def kvq_cache_bytes(desc, batch, which):
+    return _lib.kvq_cache_bytes(ctypes.byref(desc), batch, which)
+
+
+def kvq_auto_splits(desc, batch, ctx_len):
+    return _lib.kvq_auto_splits(ctypes.byref(desc), batch, ctx_len)
+
+
+def kvq_workspace_bytes(desc, batch, n_splits=0):
+    return _lib.kvq_workspace_bytes(ctypes.byref(desc), batch, n_splits)
+
+
+def kvq_turbo3_codebook():
+    lv = (ctypes.c_float * 8)()
+    th = (ctypes.c_float * 7)()
+    _check(_lib.kvq_turbo3_codebook(lv, th), "kvq_turbo3_codebook")
+    return list(lv), list(th)
+
+
+def kvq_turbo3_signs(seed, head_dim):
+    out = (ctypes.c_float * head_dim)()
+    _check(_lib.kvq_turbo3_signs(seed, head_dim, out), "kvq_turbo3_signs")
+    return list(out)
+
+
+# ----------------------------------------------------------------- kernels
+
+def kvq_append_quantize(desc, k_cache, v_cache, k_new, v_new, batch, pos, n_tok, stream=None):
+    return _check(_lib.kvq_append_quantize(ctypes.byref(desc), _ptr(k_cache), _ptr(v_cache), _ptr(k_new),
+                                           _ptr(v_new), batch, pos, n_tok, _stream(stream)),
+                  "kvq_append_quantize")
+
+
+def kvq_decode_attention(desc, k_cache, v_cache, q, batch, ctx_len, softmax_scale, n_splits, workspace,
+                         workspace_bytes=None, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return _check(_lib.kvq_decode_attention(ctypes.byref(desc), _ptr(k_cache), _ptr(v_cache), _ptr(q), batch,
+                                            ctx_len, softmax_scale, n_splits, _ptr(workspace), workspace_bytes,
+                                            _stream(stream)),
+                  "kvq_decode_attention")
+
+
+def kvq_combine(desc, workspace, batch, ctx_len, n_splits, out, workspace_bytes=None, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return _check(_lib.kvq_combine(ctypes.byref(desc), _ptr(workspace), workspace_bytes, batch, ctx_len,
+                                   n_splits, _ptr(out), _stream(stream)),
+                  "kvq_combine")
+
+
+def raw_status(name, *args):
+    """Calls a C entry point with already-marshalled arguments and returns its
+    raw status (for tests of the error paths)."""
+    return getattr(_lib, name)(*args)

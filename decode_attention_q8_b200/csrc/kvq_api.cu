@@ -1,0 +1,400 @@
+// libkvq C ABI: argument checks, cache layout, split selection, the turbo3
+// constants (sign vector, codebook) and kernel launches.  Declarations and the
+// format definitions are in include/kvq.h.
+//
+// Error convention ("Eval bug: Metal fails mixed quantized KV on Apple Silicon
+// when Flash Attention is unavailable, ...", section "Expected behavior"): an
+// unsupported combination is rejected early and cleanly -- every check runs on
+// the host before any launch, and an error status means nothing was launched.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+
+int64_t rows_per_plane(int64_t max_ctx) { return (max_ctx + kRowAlign - 1) / kRowAlign * kRowAlign; }
+
+int32_t code_bytes_of(int32_t type, int32_t d) {
+  switch (type) {
+    case KVQ_F16: return 2 * d;
+    case KVQ_Q8_0: return d;
+    case KVQ_Q4_0: return d / 2;
+    case KVQ_TURBO3: return 3 * d / 8;
+  }
+  return 0;
+}
+
+int32_t n_scales_of(int32_t type, int32_t d) {
+  switch (type) {
+    case KVQ_F16: return 0;
+    case KVQ_Q8_0:
+    case KVQ_Q4_0: return d / kBlock;
+    case KVQ_TURBO3: return 1;
+  }
+  return 0;
+}
+
+namespace {
+
+thread_local std::string g_last_cuda_error;
+
+constexpr int64_t kMaxCtx = (int64_t)1 << 31;
+constexpr int64_t kMinChunk = 256;  // fewest rows per split the heuristic plans
+
+bool known_type(int32_t t) { return t >= KVQ_F16 && t <= KVQ_TURBO3; }
+bool pow2(int32_t v) { return v > 0 && (v & (v - 1)) == 0; }
+bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
+int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+kvq_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = cudaGetErrorString(e);
+  return KVQ_ERR_CUDA;
+}
+
+// ---- turbo3 constants ------------------------------------------------------
+
+// splitmix64 (Steele, Lea & Flood 2014): advance the state by the golden-ratio
+// increment, then two xor-shift-multiply rounds and a final xor-shift.
+uint64_t splitmix64_next(uint64_t& state) {
+  state += 0x9E3779B97F4A7C15ull;
+  uint64_t z = state;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+void sign_bits(uint64_t seed, int32_t d, uint32_t out[kMaxHeadDim / 32]) {
+  std::memset(out, 0, sizeof(uint32_t) * (kMaxHeadDim / 32));
+  uint64_t st = seed;
+  for (int i = 0; i < d; ++i)
+    if (splitmix64_next(st) >> 63) out[i >> 5] |= 1u << (i & 31);
+}
+
+// 8-level Lloyd-Max quantizer of N(0,1) by Lloyd's iteration in double:
+// thresholds are midpoints of neighbouring levels, each level is the mean of
+// N(0,1) on its cell, (phi(a) - phi(b)) / (Q(a) - Q(b)) with Q the upper tail.
+// Symmetric: the positive half is iterated with the middle threshold at 0.
+struct Codebook {
+  float levels[8];
+  float tau[7];
+};
+
+double npdf(double x) { return std::exp(-0.5 * x * x) * 0.39894228040143267794; }
+double upper_tail(double x) { return 0.5 * std::erfc(x * 0.70710678118654752440); }
+
+Codebook compute_codebook() {
+  double c[4] = {0.3, 0.8, 1.4, 2.2};
+  for (int it = 0; it < 100000; ++it) {
+    double t[5] = {0.0, 0.5 * (c[0] + c[1]), 0.5 * (c[1] + c[2]), 0.5 * (c[2] + c[3]), INFINITY};
+    double next[4];
+    double change = 0.0;
+    for (int k = 0; k < 4; ++k) {
+      const double pa = npdf(t[k]), qa = upper_tail(t[k]);
+      const double pb = std::isinf(t[k + 1]) ? 0.0 : npdf(t[k + 1]);
+      const double qb = std::isinf(t[k + 1]) ? 0.0 : upper_tail(t[k + 1]);
+      next[k] = (pa - pb) / (qa - qb);
+      change = std::fmax(change, std::fabs(next[k] - c[k]));
+    }
+    std::memcpy(c, next, sizeof(c));
+    if (change < 1e-15) break;
+  }
+  double lv[8];
+  for (int k = 0; k < 4; ++k) {
+    lv[4 + k] = c[k];
+    lv[3 - k] = -c[k];
+  }
+  Codebook cb;
+  for (int k = 0; k < 8; ++k) cb.levels[k] = (float)lv[k];
+  for (int k = 0; k < 7; ++k) cb.tau[k] = (float)(0.5 * (lv[k] + lv[k + 1]));
+  return cb;
+}
+
+const Codebook& codebook() {
+  static std::once_flag once;
+  static Codebook cb;
+  std::call_once(once, [] { cb = compute_codebook(); });
+  return cb;
+}
+
+Turbo3Consts turbo3_consts(const kvq_cache_desc* d) {
+  Turbo3Consts t{};
+  const Codebook& cb = codebook();
+  std::memcpy(t.levels, cb.levels, sizeof(t.levels));
+  std::memcpy(t.tau, cb.tau, sizeof(t.tau));
+  sign_bits(d->turbo_seed, d->head_dim, t.sign_bits);
+  return t;
+}
+
+// ---- splits -----------------------------------------------------------------
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    return 148;  // B200
+  }
+  return n;
+}
+
+// Splits for `units` independent (batch, KV head) rows of work over ctx rows:
+// as many as the context allows (>= kMinChunk rows each) up to S*, where S*
+// maximises the fraction of CTA slots busy over the waves it takes, less 2%
+// per extra wave.  Non-decreasing in ctx.
+int32_t choose_splits(int64_t units, int64_t ctx, int sms, int per_sm) {
+  const int64_t slots = (int64_t)sms * per_sm;
+  const int64_t cap = std::max<int64_t>(1, std::min<int64_t>(kMaxSplits, (ctx + kMinChunk - 1) / kMinChunk));
+  const int64_t s_min = std::max<int64_t>(1, (slots + units - 1) / units);
+  const int64_t s_hi = std::min<int64_t>(kMaxSplits, 4 * s_min);
+  int64_t best = 1;
+  double best_score = -1e30;
+  for (int64_t s = 1; s <= s_hi; ++s) {
+    const int64_t ctas = units * s;
+    const int64_t waves = (ctas + slots - 1) / slots;
+    const double score = (double)ctas / (double)(waves * slots) - 0.02 * (double)(waves - 1);
+    if (score > best_score + 1e-12) {
+      best_score = score;
+      best = s;
+    }
+  }
+  return (int32_t)std::min(best, cap);
+}
+
+int64_t chunk_rows(int64_t ctx, int32_t S) { return round_up((ctx + S - 1) / S, kSplitAlign); }
+
+// Upper bound of the automatic split count over ctx_len <= ctx (sizes the
+// workspace for n_splits = 0).
+int32_t auto_splits_bound(const kvq_cache_desc* d, int32_t batch, int64_t ctx) {
+  return choose_splits((int64_t)batch * d->n_kv_heads, ctx, sm_count(), decode_ctas_per_sm());
+}
+
+// Explicit counts are used as given (trailing splits may be empty); the
+// automatic count drops the splits that rounding the chunk to 16 rows leaves
+// empty, so it never exceeds auto_splits_bound(max_ctx).
+int32_t resolve_splits(const kvq_cache_desc* d, int32_t batch, int64_t ctx, int32_t n_splits) {
+  if (n_splits > 0) return n_splits;
+  const int32_t S = auto_splits_bound(d, batch, ctx);
+  return (int32_t)((ctx + chunk_rows(ctx, S) - 1) / chunk_rows(ctx, S));
+}
+
+struct WsLayout {
+  int64_t m_off, l_off, acc_off, total;
+};
+
+WsLayout ws_layout(const kvq_cache_desc* d, int32_t batch, int32_t S) {
+  WsLayout w;
+  const int64_t rows = (int64_t)batch * d->n_q_heads * S;
+  w.m_off = 0;
+  w.l_off = round_up(rows * 4, 256);
+  w.acc_off = w.l_off + round_up(rows * 4, 256);
+  w.total = w.acc_off + rows * d->head_dim * 4;
+  return w;
+}
+
+Plane plane_of(const kvq_cache_desc* d, int32_t batch, int which, void* base) {
+  kvq_plane_layout L;
+  kvq_cache_layout(d, batch, which, &L);
+  Plane p;
+  p.codes = static_cast<uint8_t*>(base);
+  p.scales = reinterpret_cast<__half*>(static_cast<uint8_t*>(base) + L.scale_offset);
+  p.T = L.rows_per_plane;
+  p.code_bytes = (int32_t)L.code_bytes;
+  p.n_scales = (int32_t)L.n_scales;
+  return p;
+}
+
+}  // namespace
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" {
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_WORKSPACE: return "workspace too small";
+    case KVQ_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* kvq_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+
+size_t kvq_row_bytes(int32_t type, int32_t head_dim) {
+  if (!known_type(type) || head_dim <= 0 || head_dim % kBlock || head_dim > kMaxHeadDim) return 0;
+  if (type == KVQ_TURBO3 && !pow2(head_dim)) return 0;
+  return (size_t)code_bytes_of(type, head_dim) + 2 * (size_t)n_scales_of(type, head_dim);
+}
+
+kvq_status kvq_check_desc(const kvq_cache_desc* d) {
+  if (!d) return KVQ_ERR_INVALID;
+  if (d->n_q_heads < 1 || d->n_kv_heads < 1 || d->n_q_heads % d->n_kv_heads) return KVQ_ERR_INVALID;
+  if (d->head_dim < 1 || d->reserved != 0) return KVQ_ERR_INVALID;
+  if (d->max_ctx < 1 || d->max_ctx > kMaxCtx) return KVQ_ERR_INVALID;
+  if (!known_type(d->k_type) || !known_type(d->v_type)) return KVQ_ERR_INVALID;
+  if (d->head_dim % kBlock || d->head_dim > kMaxHeadDim) return KVQ_ERR_UNSUPPORTED;
+  if (d->k_type == KVQ_TURBO3) return KVQ_ERR_UNSUPPORTED;  // turbo3 is a value format
+  if (d->v_type == KVQ_TURBO3 && !pow2(d->head_dim)) return KVQ_ERR_UNSUPPORTED;
+  if (d->n_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_layout(const kvq_cache_desc* d, int32_t batch, int32_t which, kvq_plane_layout* out) {
+  const kvq_status st = kvq_check_desc(d);
+  if (st != KVQ_OK) return st;
+  if (!out || batch < 1 || batch > 65535 || (which != 0 && which != 1)) return KVQ_ERR_INVALID;
+  const int32_t type = which ? d->v_type : d->k_type;
+  const int64_t T = rows_per_plane(d->max_ctx);
+  const int64_t planes = (int64_t)batch * d->n_kv_heads;
+  const int64_t cb = code_bytes_of(type, d->head_dim);
+  const int64_t ns = n_scales_of(type, d->head_dim);
+  const double approx = (double)planes * (double)T * (double)(cb + 2 * ns);
+  if (approx > 9.0e18) return KVQ_ERR_INVALID;
+  out->rows_per_plane = T;
+  out->code_bytes = cb;
+  out->n_scales = ns;
+  out->scale_offset = round_up(planes * T * cb, 256);
+  out->total_bytes = out->scale_offset + planes * T * ns * 2;
+  return KVQ_OK;
+}
+
+size_t kvq_cache_bytes(const kvq_cache_desc* d, int32_t batch, int32_t which) {
+  kvq_plane_layout L;
+  if (kvq_cache_layout(d, batch, which, &L) != KVQ_OK) return 0;
+  return (size_t)L.total_bytes;
+}
+
+int32_t kvq_auto_splits(const kvq_cache_desc* d, int32_t batch, int64_t ctx_len) {
+  if (kvq_check_desc(d) != KVQ_OK || batch < 1 || ctx_len < 1 || ctx_len > d->max_ctx) return 0;
+  return resolve_splits(d, batch, ctx_len, 0);
+}
+
+size_t kvq_workspace_bytes(const kvq_cache_desc* d, int32_t batch, int32_t n_splits) {
+  if (kvq_check_desc(d) != KVQ_OK || batch < 1 || batch > 65535 || n_splits < 0 || n_splits > kMaxSplits) return 0;
+  const int32_t S = n_splits > 0 ? n_splits : auto_splits_bound(d, batch, d->max_ctx);
+  return (size_t)ws_layout(d, batch, S).total;
+}
+
+kvq_status kvq_turbo3_codebook(float levels[8], float thresholds[7]) {
+  if (!levels || !thresholds) return KVQ_ERR_INVALID;
+  const Codebook& cb = codebook();
+  std::memcpy(levels, cb.levels, sizeof(cb.levels));
+  std::memcpy(thresholds, cb.tau, sizeof(cb.tau));
+  return KVQ_OK;
+}
+
+kvq_status kvq_turbo3_signs(uint64_t seed, int32_t head_dim, float* signs) {
+  if (!signs || head_dim < 1 || head_dim > kMaxHeadDim) return KVQ_ERR_INVALID;
+  uint32_t bits[kMaxHeadDim / 32];
+  sign_bits(seed, head_dim, bits);
+  for (int i = 0; i < head_dim; ++i) signs[i] = ((bits[i >> 5] >> (i & 31)) & 1u) ? -1.f : 1.f;
+  return KVQ_OK;
+}
+
+kvq_status kvq_append_quantize(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* k_new,
+                               const void* v_new, int32_t batch, int64_t pos, int32_t n_tok, void* stream) {
+  kvq_status st = kvq_check_desc(d);
+  if (st != KVQ_OK) return st;
+  if (batch < 1 || batch > 65535 || n_tok < 1 || pos < 0 || pos + n_tok > d->max_ctx) return KVQ_ERR_INVALID;
+  const bool do_k = k_cache != nullptr, do_v = v_cache != nullptr;
+  if (do_k != (k_new != nullptr) || do_v != (v_new != nullptr) || (!do_k && !do_v)) return KVQ_ERR_INVALID;
+  if ((do_k && (!aligned(k_cache, 256) || !aligned(k_new, 16))) ||
+      (do_v && (!aligned(v_cache, 256) || !aligned(v_new, 16))))
+    return KVQ_ERR_INVALID;
+  const int64_t rows = (int64_t)batch * n_tok * d->n_kv_heads;
+  if (rows * (d->head_dim / 4) > ((int64_t)1 << 40)) return KVQ_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int which = 0; which < 2; ++which) {
+    void* cache = which ? v_cache : k_cache;
+    if (!cache) continue;
+    AppendParams p{};
+    p.src = static_cast<const __half*>(which ? v_new : k_new);
+    p.dst = plane_of(d, batch, which, cache);
+    p.B = batch;
+    p.H = d->n_kv_heads;
+    p.D = d->head_dim;
+    p.n_tok = n_tok;
+    p.pos = pos;
+    const int32_t type = which ? d->v_type : d->k_type;
+    if (type == KVQ_TURBO3) p.t3 = turbo3_consts(d);
+    const cudaError_t e = launch_append(type, p, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* k_cache, const void* v_cache, const void* q,
+                                int32_t batch, int64_t ctx_len, float softmax_scale, int32_t n_splits,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  kvq_status st = kvq_check_desc(d);
+  if (st != KVQ_OK) return st;
+  if (!k_cache || !v_cache || !q || !workspace) return KVQ_ERR_INVALID;
+  if (batch < 1 || batch > 65535 || ctx_len < 1 || ctx_len > d->max_ctx) return KVQ_ERR_INVALID;
+  if (n_splits < 0 || n_splits > kMaxSplits || !std::isfinite(softmax_scale)) return KVQ_ERR_INVALID;
+  if (!aligned(k_cache, 256) || !aligned(v_cache, 256) || !aligned(q, 16) || !aligned(workspace, 256))
+    return KVQ_ERR_INVALID;
+  const int32_t G = d->n_q_heads / d->n_kv_heads;
+  if (!decode_supported(d->k_type, d->v_type, G, d->head_dim)) return KVQ_ERR_UNSUPPORTED;
+  const int32_t S = resolve_splits(d, batch, ctx_len, n_splits);
+  const WsLayout w = ws_layout(d, batch, S);
+  if (workspace_bytes < (size_t)w.total) return KVQ_ERR_WORKSPACE;
+
+  DecodeParams p{};
+  p.k = plane_of(d, batch, 0, const_cast<void*>(k_cache));
+  p.v = plane_of(d, batch, 1, const_cast<void*>(v_cache));
+  p.q = static_cast<const __half*>(q);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.ws_m = reinterpret_cast<float*>(ws + w.m_off);
+  p.ws_l = reinterpret_cast<float*>(ws + w.l_off);
+  p.ws_acc = reinterpret_cast<float*>(ws + w.acc_off);
+  p.B = batch;
+  p.n_q = d->n_q_heads;
+  p.n_kv = d->n_kv_heads;
+  p.G = G;
+  p.D = d->head_dim;
+  p.S = S;
+  p.ctx = ctx_len;
+  p.chunk = chunk_rows(ctx_len, S);
+  p.qscale = softmax_scale * 1.4426950408889634f;
+  if (d->v_type == KVQ_TURBO3) p.t3 = turbo3_consts(d);
+  const cudaError_t e = launch_decode(d->k_type, d->v_type, p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KVQ_OK;
+}
+
+kvq_status kvq_combine(const kvq_cache_desc* d, const void* workspace, size_t workspace_bytes, int32_t batch,
+                       int64_t ctx_len, int32_t n_splits, float* out, void* stream) {
+  kvq_status st = kvq_check_desc(d);
+  if (st != KVQ_OK) return st;
+  if (!workspace || !out) return KVQ_ERR_INVALID;
+  if (batch < 1 || batch > 65535 || ctx_len < 1 || ctx_len > d->max_ctx) return KVQ_ERR_INVALID;
+  if (n_splits < 0 || n_splits > kMaxSplits) return KVQ_ERR_INVALID;
+  if (!aligned(workspace, 256) || !aligned(out, 16)) return KVQ_ERR_INVALID;
+  const int32_t S = resolve_splits(d, batch, ctx_len, n_splits);
+  const WsLayout w = ws_layout(d, batch, S);
+  if (workspace_bytes < (size_t)w.total) return KVQ_ERR_WORKSPACE;
+  CombineParams p{};
+  const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+  p.ws_m = reinterpret_cast<const float*>(ws + w.m_off);
+  p.ws_l = reinterpret_cast<const float*>(ws + w.l_off);
+  p.ws_acc = reinterpret_cast<const float*>(ws + w.acc_off);
+  p.out = out;
+  p.B = batch;
+  p.n_q = d->n_q_heads;
+  p.D = d->head_dim;
+  p.S = S;
+  p.turbo3 = d->v_type == KVQ_TURBO3;
+  if (p.turbo3) p.t3 = turbo3_consts(d);
+  const cudaError_t e = launch_combine(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KVQ_OK;
+}
+
+}  // extern "C"

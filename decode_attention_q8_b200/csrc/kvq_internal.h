@@ -1,0 +1,75 @@
+// Internal declarations shared by the libkvq translation units (host + device).
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kBlock = 32;          // elements per q8_0 / q4_0 block
+constexpr int kMaxHeadDim = 256;
+constexpr int kRowAlign = 16;       // rows per plane are a multiple of this
+constexpr int kMaxSplits = 4096;
+constexpr int kSplitAlign = 16;     // split chunks are a multiple of this many rows
+
+// Device view of one cache tensor (K or V) of one layer.
+struct Plane {
+  uint8_t* codes;      // [B][H][T][code_bytes]
+  __half* scales;      // [B][H][T][n_scales]
+  int64_t T;           // rows per (batch, head) plane
+  int32_t code_bytes;
+  int32_t n_scales;
+};
+
+struct Turbo3Consts {
+  float levels[8];
+  float tau[7];
+  uint32_t sign_bits[kMaxHeadDim / 32];  // bit i set -> s_i = -1
+};
+
+struct AppendParams {
+  const __half* src;   // [B][n_tok][H][D]
+  Plane dst;
+  int32_t B, H, D, n_tok;
+  int64_t pos;
+  Turbo3Consts t3;
+};
+
+struct DecodeParams {
+  Plane k, v;
+  const __half* q;     // [B][n_q][D]
+  float* ws_m;         // [B][n_q][S]
+  float* ws_l;
+  float* ws_acc;       // [B][n_q][S][D]
+  int32_t B, n_q, n_kv, G, D, S;
+  int64_t ctx, chunk;
+  float qscale;        // softmax_scale * log2(e)
+  Turbo3Consts t3;
+};
+
+struct CombineParams {
+  const float* ws_m;
+  const float* ws_l;
+  const float* ws_acc;
+  float* out;          // [B][n_q][D]
+  int32_t B, n_q, D, S;
+  int32_t turbo3;      // apply s * H_un * (.) / D
+  Turbo3Consts t3;
+};
+
+// Host-side helpers (kvq_api.cu).
+int64_t rows_per_plane(int64_t max_ctx);
+int32_t code_bytes_of(int32_t type, int32_t d);
+int32_t n_scales_of(int32_t type, int32_t d);
+
+// Launchers; each returns cudaGetLastError() after its launch.
+cudaError_t launch_append(int32_t type, const AppendParams& p, cudaStream_t st);
+cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p, cudaStream_t st);
+bool decode_supported(int32_t k_type, int32_t v_type, int32_t G, int32_t D);
+int decode_ctas_per_sm();  // resident decode CTAs per SM the split heuristic plans for
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
+
+}  // namespace kvq

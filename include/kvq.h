@@ -1,0 +1,214 @@
+/*
+ * kvq.h -- C ABI of libkvq: quantized-KV decode attention on NVIDIA B200 (sm_100a).
+ *
+ * What it computes
+ * ----------------
+ * Attention decoding over a KV cache whose keys and values are stored at
+ * independently chosen precisions.  The pages this library follows:
+ *   - "KVSplit - 2- bis 3-mal längerer Kontext auf Apple Silicon", sections
+ *     "Zentrale Benchmark-Ergebnisse" and "Anwendungsbeispiele und
+ *     Konfigurationsempfehlungen": keys and values quantized at different
+ *     precisions (K8V4, K8V8, K4V4, K4V8 demo), chosen per tensor;
+ *   - "llama.cpp für Geschwindigkeit und Speicher optimieren", section
+ *     "KV-Cache-Präzision": cache types f16 / q8_0 / q4_0, set independently for
+ *     K and V; section "Flash Attention": tiled attention that is exactly
+ *     standard attention, not an approximation;
+ *   - "Benchmark TurboQuant en Apple Silicon", section "¿Qué es TurboQuant?":
+ *     a 3-bit value cache ("turbo3") after a random Walsh-Hadamard rotation and
+ *     an optimal scalar quantizer; section "Explicación de la configuración":
+ *     q8_0 keys with turbo3 values;
+ *   - "Eval bug: Metal fails mixed quantized KV on Apple Silicon when Flash
+ *     Attention is unavailable, ...", section "Expected behavior": an
+ *     unsupported combination must be rejected early and cleanly, without
+ *     partial initialization or a crash.
+ *
+ * Cache types (per 32-element block unless stated):
+ *   KVQ_F16    the fp16 input, unchanged (2 bytes / element).
+ *   KVQ_Q8_0   fp16 scale d = amax/127 and 32 int8 q_j = round-half-away(x_j/d),
+ *              computed in binary32 with an IEEE divide per element; the fp32 d
+ *              (not its fp16 image) quantizes; d == 0 gives q_j = 0.  34 bytes.
+ *   KVQ_Q4_0   m = signed value of the largest |x_j| (lowest j on ties),
+ *              d = m / -8, q_j = min(15, trunc(fl(fl(x_j * fl(1/d)) + 8.5))),
+ *              element j in the low nibble of byte j, element j+16 in the high
+ *              nibble; d == 0 gives nibble 8.  18 bytes.
+ *   KVQ_TURBO3 (values only; head_dim a power of two) one row of head_dim
+ *              elements: signs s_i = -1 when output i of splitmix64(turbo_seed)
+ *              has its top bit set; v = s*x; norm = sqrtf(tree sum of v_i^2,
+ *              pairs at stride d/2, d/4, ..., 1); w = unnormalised fast
+ *              Walsh-Hadamard transform of v (stages h = 1, 2, ..., d/2);
+ *              g_i = w_i * fl(1/norm); code_i = #{k : g_i > tau_k} against the
+ *              seven binary32 midpoints of the 8-level Lloyd-Max quantizer of
+ *              N(0,1) (so g/sqrt(d) is coded with the N(0,1/d) codebook);
+ *              codes packed 3 bits each, little-endian (code i in bits
+ *              3i..3i+2); stored norm fp16(min(norm, 65504)).  3d/8 + 2 bytes.
+ *              Decoded value: x_hat = (norm/d) * s * H_un * c[code].
+ *
+ * Memory layout of one cache tensor (K or V) of one layer, in device memory
+ * owned by the caller:
+ *   rows_per_plane T = max_ctx rounded up to a multiple of 16;
+ *   code plane  at byte 0:           [batch][n_kv_heads][T][code_bytes]
+ *   scale plane at byte scale_offset: [batch][n_kv_heads][T][n_scales] fp16
+ *   with code_bytes = 2d (f16), d (q8_0), d/2 (q4_0), 3d/8 (turbo3);
+ *   n_scales = 0 (f16), d/32 (q8_0, q4_0), 1 (turbo3, the norm);
+ *   scale_offset = code plane bytes rounded up to a multiple of 256.
+ *   Within a row, q8_0 codes and q4_0 bytes are in block order, exactly as the
+ *   block formats above; scale n of a row belongs to block n.
+ *   The base pointer must be 256-byte aligned (cudaMalloc's is).
+ *
+ * Conventions
+ *   Query head h attends with KV head floor(h / G), G = n_q_heads / n_kv_heads.
+ *   A decode query attends to cache rows 0 .. ctx_len-1 (no mask).
+ *   New K/V rows: fp16 [batch][n_tok][n_kv_heads][head_dim], row-major.
+ *   Queries: fp16 [batch][n_q_heads][head_dim].  Output: fp32
+ *   [batch][n_q_heads][head_dim].
+ *   Split-KV: with S splits, chunk = ceil(ctx_len / S) rounded up to a multiple
+ *   of 16; split s covers rows [s*chunk, min((s+1)*chunk, ctx_len)) and may be
+ *   empty.
+ *
+ * Ownership, threading, errors
+ *   The caller owns every buffer.  No entry point allocates device memory,
+ *   synchronizes the device or keeps per-call state; kernel launches go to the
+ *   given CUDA stream (NULL = legacy default stream) and run asynchronously.
+ *   Every argument check happens before any launch; on an error status
+ *   nothing has been written and nothing launched.  KVQ_ERR_CUDA means a
+ *   launch was refused by the CUDA runtime (see kvq_last_cuda_error()).
+ *   Entry points are thread-safe.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_F16 = 0,
+  KVQ_Q8_0 = 1,
+  KVQ_Q4_0 = 2,
+  KVQ_TURBO3 = 3
+} kvq_type;
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID = 1,      /* null pointer, bad count, range outside the cache */
+  KVQ_ERR_UNSUPPORTED = 2,  /* valid arguments this library does not implement */
+  KVQ_ERR_WORKSPACE = 3,    /* workspace smaller than kvq_workspace_bytes() */
+  KVQ_ERR_CUDA = 4          /* the CUDA runtime refused a launch or a query */
+} kvq_status;
+
+/* One layer's cache description (K and V of one layer share it). */
+typedef struct {
+  int32_t n_q_heads;   /* query heads, a multiple of n_kv_heads */
+  int32_t n_kv_heads;  /* KV heads */
+  int32_t head_dim;    /* multiple of 32, at most 256 */
+  int32_t k_type;      /* kvq_type of the key cache: F16, Q8_0 or Q4_0 */
+  int32_t v_type;      /* kvq_type of the value cache: any */
+  int32_t reserved;    /* must be 0 */
+  int64_t max_ctx;     /* rows the cache holds per (batch, KV head), >= 1 */
+  uint64_t turbo_seed; /* seed of the turbo3 sign vector (V only) */
+} kvq_cache_desc;
+
+/* Byte layout of one cache tensor, as described above. */
+typedef struct {
+  int64_t rows_per_plane;  /* T */
+  int64_t code_bytes;      /* bytes of codes per row */
+  int64_t n_scales;        /* fp16 scales per row */
+  int64_t scale_offset;    /* byte offset of the scale plane */
+  int64_t total_bytes;     /* bytes to allocate */
+} kvq_plane_layout;
+
+/* Human-readable name of a status.  Never NULL. */
+KVQ_API const char* kvq_status_string(kvq_status s);
+
+/* Text of the last CUDA error this thread saw (empty if none). */
+KVQ_API const char* kvq_last_cuda_error(void);
+
+/* Bytes of one cached row of head_dim elements of `type` (codes + scales),
+ * the quantity the pages' cache sizes count; 0 if unsupported. */
+KVQ_API size_t kvq_row_bytes(int32_t type, int32_t head_dim);
+
+/* Checks a descriptor: KVQ_OK, KVQ_ERR_INVALID or KVQ_ERR_UNSUPPORTED. */
+KVQ_API kvq_status kvq_check_desc(const kvq_cache_desc* desc);
+
+/* Layout of the K (which = 0) or V (which = 1) cache of one layer. */
+KVQ_API kvq_status kvq_cache_layout(const kvq_cache_desc* desc, int32_t batch, int32_t which,
+                            kvq_plane_layout* out);
+
+/* Bytes to allocate for the K (which = 0) or V (which = 1) cache; 0 on error. */
+KVQ_API size_t kvq_cache_bytes(const kvq_cache_desc* desc, int32_t batch, int32_t which);
+
+/* Split count the library picks for this problem on the current device
+ * (n_splits = 0 in kvq_decode_attention means this value); >= 1, or 0 on error. */
+KVQ_API int32_t kvq_auto_splits(const kvq_cache_desc* desc, int32_t batch, int64_t ctx_len);
+
+/* Workspace bytes kvq_decode_attention / kvq_combine need for n_splits
+ * (0 = automatic, resolved as kvq_auto_splits would for ctx_len = max_ctx);
+ * 0 on error.  Layout: m and l fp32 [batch][n_q][S] each, then acc fp32
+ * [batch][n_q][S][head_dim], each part 256-byte aligned. */
+KVQ_API size_t kvq_workspace_bytes(const kvq_cache_desc* desc, int32_t batch, int32_t n_splits);
+
+/* The turbo3 codebook this library uses: 8 binary32 levels (ascending) and
+ * the 7 binary32 thresholds between them.  Host only; no device needed. */
+KVQ_API kvq_status kvq_turbo3_codebook(float levels[8], float thresholds[7]);
+
+/* The turbo3 sign vector (+1.f / -1.f) for `seed`, head_dim entries.  Host only. */
+KVQ_API kvq_status kvq_turbo3_signs(uint64_t seed, int32_t head_dim, float* signs);
+
+/*
+ * Quantize-on-append: writes n_tok new rows per (batch, KV head) into both
+ * caches at rows pos .. pos+n_tok-1 (the CPY step that precedes attention in
+ * the llama.cpp issue's failing path, "Possibly related": unsupported "CPY").
+ *   k_cache, v_cache  device, layouts from kvq_cache_layout(desc, batch, 0/1)
+ *   k_new, v_new      device fp16 [batch][n_tok][n_kv_heads][head_dim]
+ *   pos >= 0, n_tok >= 1, pos + n_tok <= max_ctx.
+ * Either cache/row pair may be NULL to skip that tensor (not both).
+ * Quantized bytes are deterministic and bit-exact to the formats above.
+ */
+KVQ_API kvq_status kvq_append_quantize(const kvq_cache_desc* desc, void* k_cache, void* v_cache,
+                               const void* k_new, const void* v_new, int32_t batch,
+                               int64_t pos, int32_t n_tok, void* cuda_stream);
+
+/*
+ * Split-KV decode: for every (batch b, query head h, split s) writes the
+ * partial softmax state of rows in split s to the workspace:
+ *   m  = max_t s_t * log2(e)       (scores in base-2 units; -inf if empty)
+ *   l  = sum_t 2^(s_t*log2(e) - m)
+ *   acc= sum_t 2^(s_t*log2(e) - m) * v_hat_t   (turbo3: in the rotated domain,
+ *        acc = sum_t p_t * norm_t * c[code_t], before the inverse transform)
+ * with s_t = softmax_scale * <q_h, k_hat_t>.
+ *   q              device fp16 [batch][n_q_heads][head_dim]
+ *   ctx_len        1 <= ctx_len <= max_ctx rows attended
+ *   n_splits       0 = kvq_auto_splits, else 1 .. 4096
+ *   workspace      device, >= kvq_workspace_bytes(desc, batch, n_splits)
+ */
+KVQ_API kvq_status kvq_decode_attention(const kvq_cache_desc* desc, const void* k_cache,
+                                const void* v_cache, const void* q, int32_t batch,
+                                int64_t ctx_len, float softmax_scale, int32_t n_splits,
+                                void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * Combine: merges the n_splits partials of kvq_decode_attention into
+ *   out[b][h] = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s,
+ * and for a turbo3 value cache applies the inverse rotation s * H_un * (.) / d.
+ *   n_splits must equal the value kvq_decode_attention used (after resolving 0,
+ *   pass the same 0 and the same ctx_len).
+ *   out            device fp32 [batch][n_q_heads][head_dim]
+ */
+KVQ_API kvq_status kvq_combine(const kvq_cache_desc* desc, const void* workspace,
+                       size_t workspace_bytes, int32_t batch, int64_t ctx_len,
+                       int32_t n_splits, float* out, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,188 @@
+"""Host-side tests of the C ABI: the library loads, exports what include/kvq.h
+declares, and its size / layout / turbo3 constants / argument checks behave.
+No GPU: nothing here launches a kernel (every call below is rejected or answered
+on the host)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import decode_attention_q8_b200 as kvq
+from oracle import cache_model, turbo3
+from conftest import ROOT, read_golden
+
+HEADER = os.path.join(ROOT, "include", "kvq.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"KVQ_API\s+[\w\s\*]+?\b(kvq_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) == len(kvq.EXPORTED) and set(names) == set(kvq.EXPORTED)
+    dyn = subprocess.run(["nm", "-D", "--defined-only", kvq.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (kvq_\w+)", dyn))
+    for n in names:
+        assert n in exported, n
+        assert getattr(kvq._lib, n) is not None
+    # nothing else leaks out under the kvq_ prefix
+    assert exported == set(names)
+
+
+def test_status_strings():
+    for s in range(5):
+        assert kvq.kvq_status_string(s)
+    assert kvq.kvq_status_string(99) == "unknown status"
+
+
+def test_row_bytes_match_oracle_model():
+    for t in ("f16", "q8_0", "q4_0"):
+        for d in (32, 64, 128, 256):
+            assert kvq.kvq_row_bytes(t, d) == cache_model.row_bytes(t, d)
+    for d in (32, 64, 128, 256):
+        assert kvq.kvq_row_bytes("turbo3", d) == cache_model.row_bytes("turbo3", d)
+    assert kvq.kvq_row_bytes("q8_0", 48) == 0
+    assert kvq.kvq_row_bytes("turbo3", 96) == 0
+    assert kvq.kvq_row_bytes(7, 128) == 0
+
+
+def test_cache_bytes_reproduce_pages():
+    """Layer caches allocated by the library sum to the sizes the pages print."""
+    mib = 1024.0 * 1024.0
+    for row in read_golden("kv_cache_bytes.txt"):
+        L, H, D, T, kt, vt, exp, which = row.split()
+        L, H, D, T, exp = int(L), int(H), int(D), int(T), float(exp)
+        desc = kvq.make_desc(H, H, D, kt, vt, T)
+        k = L * kvq.kvq_cache_bytes(desc, 1, 0)
+        v = L * kvq.kvq_cache_bytes(desc, 1, 1)
+        got = {"K": k, "V": v, "KV": k + v}[which] / mib
+        assert got == exp, row
+
+
+def test_layout_formula():
+    desc = kvq.make_desc(32, 8, 128, "q8_0", "turbo3", 1000, turbo_seed=5)
+    L = kvq.kvq_cache_layout(desc, 3, 0)
+    assert L.rows_per_plane == 1008 and L.code_bytes == 128 and L.n_scales == 4
+    assert L.scale_offset == 3 * 8 * 1008 * 128
+    assert L.total_bytes == L.scale_offset + 3 * 8 * 1008 * 4 * 2
+    V = kvq.kvq_cache_layout(desc, 3, 1)
+    assert V.code_bytes == 48 and V.n_scales == 1
+    assert V.scale_offset % 256 == 0 and V.scale_offset >= 3 * 8 * 1008 * 48
+    assert V.total_bytes == V.scale_offset + 3 * 8 * 1008 * 2
+
+
+def test_turbo3_codebook_equals_oracle():
+    lv, th = kvq.kvq_turbo3_codebook()
+    olv, oth = turbo3.codebook_f32()
+    np.testing.assert_array_equal(np.array(lv, np.float32), olv)
+    np.testing.assert_array_equal(np.array(th, np.float32), oth)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 1234567, 0x7475726233, 2**64 - 1])
+def test_turbo3_signs_equal_oracle(seed):
+    for d in (32, 128, 256):
+        np.testing.assert_array_equal(np.array(kvq.kvq_turbo3_signs(seed, d), np.float32),
+                                      turbo3.signs(seed, d))
+
+
+def test_check_desc():
+    ok = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 32768)
+    assert kvq.kvq_check_desc(ok) == kvq.KVQ_OK
+    bad = [
+        (kvq.make_desc(63, 8, 128, "q8_0", "q4_0", 32768), kvq.KVQ_ERR_INVALID),   # n_q % n_kv
+        (kvq.make_desc(64, 0, 128, "q8_0", "q4_0", 32768), kvq.KVQ_ERR_INVALID),
+        (kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 0), kvq.KVQ_ERR_INVALID),
+        (kvq.make_desc(64, 8, 128, 9, "q4_0", 16), kvq.KVQ_ERR_INVALID),           # unknown type
+        (kvq.make_desc(64, 8, 80, "q8_0", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),   # head_dim % 32
+        (kvq.make_desc(64, 8, 512, "q8_0", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),  # head_dim > 256
+        (kvq.make_desc(64, 8, 128, "turbo3", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),  # turbo3 K
+        (kvq.make_desc(64, 8, 96, "q8_0", "turbo3", 16), kvq.KVQ_ERR_UNSUPPORTED),   # WHT needs 2^k
+    ]
+    for desc, st in bad:
+        assert kvq.kvq_check_desc(desc) == st
+    d = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 16)
+    d.reserved = 1
+    assert kvq.kvq_check_desc(d) == kvq.KVQ_ERR_INVALID
+    assert kvq.raw_status("kvq_check_desc", None) == kvq.KVQ_ERR_INVALID
+
+
+FAKE = 0x7f0000000000  # 256-byte aligned address that is never dereferenced
+
+
+def _append(desc, k_cache=FAKE, v_cache=FAKE, k_new=FAKE, v_new=FAKE, batch=1, pos=0, n_tok=1):
+    return kvq.raw_status("kvq_append_quantize", ctypes.byref(desc), k_cache, v_cache, k_new, v_new,
+                          batch, pos, n_tok, None)
+
+
+def _decode(desc, k=FAKE, v=FAKE, q=FAKE, batch=1, ctx=16, scale=0.1, S=0, ws=FAKE, ws_bytes=1 << 40):
+    return kvq.raw_status("kvq_decode_attention", ctypes.byref(desc), k, v, q, batch, ctx, scale, S, ws,
+                          ws_bytes, None)
+
+
+def _combine(desc, ws=FAKE, ws_bytes=1 << 40, batch=1, ctx=16, S=0, out=FAKE):
+    return kvq.raw_status("kvq_combine", ctypes.byref(desc), ws, ws_bytes, batch, ctx, S, out, None)
+
+
+def test_append_rejects_before_launch():
+    d = kvq.make_desc(8, 2, 64, "q8_0", "q4_0", 256)
+    assert _append(d, pos=250, n_tok=7) == kvq.KVQ_ERR_INVALID     # past max_ctx
+    assert _append(d, pos=-1) == kvq.KVQ_ERR_INVALID
+    assert _append(d, n_tok=0) == kvq.KVQ_ERR_INVALID
+    assert _append(d, batch=0) == kvq.KVQ_ERR_INVALID
+    assert _append(d, k_new=None) == kvq.KVQ_ERR_INVALID            # cache without rows
+    assert _append(d, k_cache=None, k_new=None, v_cache=None, v_new=None) == kvq.KVQ_ERR_INVALID
+    assert _append(d, k_cache=FAKE + 16) == kvq.KVQ_ERR_INVALID     # cache not 256-aligned
+    assert _append(d, v_new=FAKE + 2) == kvq.KVQ_ERR_INVALID        # rows not 16-aligned
+    assert _append(kvq.make_desc(8, 2, 64, "turbo3", "q4_0", 256)) == kvq.KVQ_ERR_UNSUPPORTED
+
+
+def test_decode_and_combine_reject_before_launch():
+    d = kvq.make_desc(32, 8, 128, "q8_0", "q4_0", 8192)
+    assert _decode(d, ctx=0) == kvq.KVQ_ERR_INVALID
+    assert _decode(d, ctx=8193) == kvq.KVQ_ERR_INVALID
+    assert _decode(d, q=None) == kvq.KVQ_ERR_INVALID
+    assert _decode(d, S=-1) == kvq.KVQ_ERR_INVALID
+    assert _decode(d, S=5000) == kvq.KVQ_ERR_INVALID
+    assert _decode(d, scale=float("nan")) == kvq.KVQ_ERR_INVALID
+    assert _decode(d, ws=FAKE + 8) == kvq.KVQ_ERR_INVALID
+    need = kvq.kvq_workspace_bytes(d, 1, 4)
+    assert need > 0
+    assert _decode(d, S=4, ws_bytes=need - 1) == kvq.KVQ_ERR_WORKSPACE
+    assert _combine(d, S=4, ws_bytes=need - 1) == kvq.KVQ_ERR_WORKSPACE
+    assert _combine(d, out=None) == kvq.KVQ_ERR_INVALID
+    assert _combine(d, ctx=0) == kvq.KVQ_ERR_INVALID
+    assert _decode(kvq.make_desc(32, 8, 128, "turbo3", "q4_0", 64)) == kvq.KVQ_ERR_UNSUPPORTED
+
+
+def test_workspace_bytes_formula():
+    d = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 32768)
+    B, S = 4, 9
+    rows = B * 64 * S
+    r256 = lambda v: (v + 255) // 256 * 256
+    assert kvq.kvq_workspace_bytes(d, B, S) == 2 * r256(rows * 4) + rows * 128 * 4
+    assert kvq.kvq_workspace_bytes(d, 0, S) == 0
+    # the automatic split count never needs more workspace than n_splits = 0 reserves
+    auto_ws = kvq.kvq_workspace_bytes(d, B, 0)
+    for ctx in (1, 100, 4096, 32768):
+        s = kvq.kvq_auto_splits(d, B, ctx)
+        assert 1 <= s and kvq.kvq_workspace_bytes(d, B, s) <= auto_ws
+
+
+def test_auto_splits_bounded_and_nonempty():
+    for batch in (1, 4, 16):
+        d = kvq.make_desc(32, 8, 128, "q4_0", "q4_0", 131072)
+        bound = kvq.kvq_workspace_bytes(d, batch, 0)
+        for ctx in (1, 15, 16, 17, 255, 256, 257, 1000, 4096, 8192, 65536, 100003, 131072):
+            s = kvq.kvq_auto_splits(d, batch, ctx)
+            assert 1 <= s <= 4096
+            assert kvq.kvq_workspace_bytes(d, batch, s) <= bound
+            # chunks are whole 16-row groups and no automatic split is empty
+            chunk = -(-(-(-ctx // s)) // 16) * 16
+            assert (s - 1) * chunk < ctx
+    assert kvq.kvq_auto_splits(d, 1, 0) == 0

@@ -1,0 +1,160 @@
+"""Decode attention (split-KV decode + combine) on the GPU against the fp64 oracle.
+
+Tolerance: max abs error 2e-3 and relative L2 error 1e-3 of the fp32 output
+against the oracle's fp64 attention over the oracle's own dequantization of the
+same fp16 inputs (the stored bytes are checked bit-exact in test_gpu_append)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_q8_b200 as kvq
+import synth
+from kvq_testlib import (alloc_cache, assert_attention_close, decode, oracle_attention_rows, oracle_dequant,
+                         oracle_rows, rows_of)
+
+pytestmark = pytest.mark.gpu
+
+
+def _setup(k_type, v_type, B, n_q, n_kv, D, ctx, seed, max_ctx=None, outliers=(3, 17), oscale=10.0,
+           turbo_seed=None):
+    max_ctx = max_ctx or ctx
+    desc = kvq.make_desc(n_q, n_kv, D, k_type, v_type, max_ctx,
+                         turbo_seed=(seed * 31 + 7) if turbo_seed is None else turbo_seed)
+    w = synth.Workload("case", B, 1, n_q, n_kv, D, ctx, k_type, v_type, outliers, oscale, seed)
+    q, k, v = synth.layer_inputs(w, device="cuda")
+    kc, vc = alloc_cache(desc, B, 0), alloc_cache(desc, B, 1)
+    kvq.kvq_append_quantize(desc, kc, vc, k, v, B, 0, ctx)
+    return desc, q, k, v, kc, vc
+
+
+def _oracle_out(desc, q, k, v, b, g, ctx, scale):
+    """Oracle outputs [G, D] of the query heads of KV head g in batch row b."""
+    G = desc.n_q_heads // desc.n_kv_heads
+    names = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3"}
+    kt, vt = names[desc.k_type], names[desc.v_type]
+    kx = k[b, :ctx, g, :].cpu().numpy()
+    vx = v[b, :ctx, g, :].cpu().numpy()
+    kh = oracle_dequant(kt, *oracle_rows(kt, kx), desc.head_dim)
+    vh = oracle_dequant(vt, *oracle_rows(vt, vx, desc.turbo_seed), desc.head_dim, desc.turbo_seed)
+    return oracle_attention_rows(q[b, g * G:(g + 1) * G].cpu().numpy(), kh, vh, scale)
+
+
+def _check_all(desc, q, k, v, out, ctx, scale, what):
+    G = desc.n_q_heads // desc.n_kv_heads
+    o = out.cpu().numpy()
+    for b in range(q.shape[0]):
+        for g in range(desc.n_kv_heads):
+            exp = _oracle_out(desc, q, k, v, b, g, ctx, scale)
+            assert_attention_close(o[b, g * G:(g + 1) * G], exp, f"{what} b{b} g{g}")
+
+
+def test_tiny_workload():
+    """Batch 1, 4 query / 2 KV heads, head_dim 64, context 256, K q8_0 / V q4_0,
+    K channels 3 and 17 x10, scale 1/sqrt(64); all 256 rows appended."""
+    w = synth.WORKLOADS["tiny"]
+    desc = kvq.make_desc(w.n_q, w.n_kv, w.head_dim, w.k_type, w.v_type, w.ctx)
+    q, k, v = synth.layer_inputs(w, device="cuda")
+    kc, vc = alloc_cache(desc, 1, 0), alloc_cache(desc, 1, 1)
+    kvq.kvq_append_quantize(desc, kc, vc, k, v, 1, 0, w.ctx)
+    out = decode(desc, kc, vc, q, 1, w.ctx, w.scale)
+    _check_all(desc, q, k, v, out, w.ctx, w.scale, "tiny")
+
+
+@pytest.mark.parametrize("k_type", ["f16", "q8_0", "q4_0"])
+@pytest.mark.parametrize("v_type", ["f16", "q8_0", "q4_0", "turbo3"])
+def test_type_matrix(k_type, v_type):
+    B, n_q, n_kv, D, ctx = 2, 16, 4, 128, 1000
+    desc, q, k, v, kc, vc = _setup(k_type, v_type, B, n_q, n_kv, D, ctx, seed=41, max_ctx=1100)
+    scale = 1 / math.sqrt(D)
+    for S in (0, 3):
+        out = decode(desc, kc, vc, q, B, ctx, scale, S)
+        _check_all(desc, q, k, v, out, ctx, scale, f"{k_type}/{v_type} S={S}")
+
+
+@pytest.mark.parametrize("ctx", [1, 2, 15, 16, 17, 33, 129, 777])
+def test_ragged_context_lengths(ctx):
+    desc, q, k, v, kc, vc = _setup("q8_0", "q4_0", 1, 8, 2, 128, ctx, seed=ctx, max_ctx=800)
+    for S in (0, 1, 5):
+        out = decode(desc, kc, vc, q, 1, ctx, 0.09, S)
+        _check_all(desc, q, k, v, out, ctx, 0.09, f"ctx={ctx} S={S}")
+
+
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("D", [64, 128])
+def test_group_sizes_and_head_dims(G, D):
+    n_kv = 2
+    desc, q, k, v, kc, vc = _setup("q8_0", "turbo3", 2, n_kv * G, n_kv, D, 300, seed=G * 10 + D)
+    out = decode(desc, kc, vc, q, 2, 300, 1 / math.sqrt(D))
+    _check_all(desc, q, k, v, out, 300, 1 / math.sqrt(D), f"G={G} D={D}")
+
+
+def test_split_invariance_and_empty_splits():
+    """S = 1, 2, 7, auto and S larger than ctx/16 (trailing splits empty) agree."""
+    ctx = 520
+    desc, q, k, v, kc, vc = _setup("q4_0", "q4_0", 1, 8, 2, 128, ctx, seed=5)
+    outs = [decode(desc, kc, vc, q, 1, ctx, 0.1, S).cpu().numpy() for S in (1, 2, 7, 0, 40)]
+    for o in outs[1:]:
+        assert np.abs(o - outs[0]).max() < 1e-5
+    _check_all(desc, q, k, v, torch.from_numpy(outs[-1]), ctx, 0.1, "S=40")
+
+
+def test_prefix_of_a_longer_cache():
+    """ctx_len < max_ctx: rows past ctx_len (here filled with other data) are ignored."""
+    desc, q, k, v, kc, vc = _setup("q8_0", "q4_0", 1, 8, 2, 128, 600, seed=9, max_ctx=600)
+    out = decode(desc, kc, vc, q, 1, 333, 0.1)
+    _check_all(desc, q, k, v, out, 333, 0.1, "prefix")
+
+
+def test_decode_leaves_cache_untouched():
+    desc, q, k, v, kc, vc = _setup("q8_0", "turbo3", 1, 8, 2, 128, 200, seed=2)
+    k0, v0 = kc.clone(), vc.clone()
+    decode(desc, kc, vc, q, 1, 200, 0.1)
+    torch.cuda.synchronize()
+    assert torch.equal(k0, kc) and torch.equal(v0, vc)
+
+
+def test_llama8b_layer_with_controls():
+    """Llama-3.1-8B-shaped layer (32/8 heads, head_dim 128, ctx 8192): K8V4 and the
+    f16/f16 and q8_0/q8_0 controls on the same fp16 inputs, every output checked."""
+    w = synth.WORKLOADS["llama8b_ctx8k"]
+    q, k, v = synth.layer_inputs(w, device="cuda")
+    for kt, vt in ((w.k_type, w.v_type),) + w.controls:
+        desc = kvq.make_desc(w.n_q, w.n_kv, w.head_dim, kt, vt, w.ctx)
+        kc, vc = alloc_cache(desc, 1, 0), alloc_cache(desc, 1, 1)
+        kvq.kvq_append_quantize(desc, kc, vc, k, v, 1, 0, w.ctx)
+        out = decode(desc, kc, vc, q, 1, w.ctx, w.scale)
+        _check_all(desc, q, k, v, out, w.ctx, w.scale, f"8B {kt}/{vt}")
+
+
+@pytest.mark.parametrize("name", ["llama70b_ctx32k_b4", "turbo3_ctx32k", "k4v4_ctx128k_b1",
+                                  "k4v4_ctx128k_b4", "k4v4_ctx128k_b16"])
+def test_full_size_sampled(name):
+    """One layer at full size in the benchmark's launch configuration (automatic
+    splits); every output of sampled (batch row, KV head) groups is checked, plus
+    the stored bytes of sampled rows."""
+    w = synth.WORKLOADS[name]
+    desc = kvq.make_desc(w.n_q, w.n_kv, w.head_dim, w.k_type, w.v_type, w.ctx, turbo_seed=w.turbo_seed)
+    q, k, v = synth.layer_inputs(w, layer=0, device="cuda")
+    kc, vc = alloc_cache(desc, w.batch, 0), alloc_cache(desc, w.batch, 1)
+    kvq.kvq_append_quantize(desc, kc, vc, k, v, w.batch, 0, w.ctx)
+    out = decode(desc, kc, vc, q, w.batch, w.ctx, w.scale).cpu().numpy()
+    G = w.n_q // w.n_kv
+    samples = {(0, 0), (w.batch - 1, w.n_kv - 1), (w.batch // 2, w.n_kv // 2)}
+    for b, g in sorted(samples):
+        exp = _oracle_out(desc, q, k, v, b, g, w.ctx, w.scale)
+        assert_attention_close(out[b, g * G:(g + 1) * G], exp, f"{name} b{b} g{g}")
+    # stored bytes of a few rows per sampled plane
+    for which, cache, new, kind in ((0, kc, k, w.k_type), (1, vc, v, w.v_type)):
+        lay = kvq.kvq_cache_layout(desc, w.batch, which)
+        host = cache.cpu().numpy()
+        for b, g in sorted(samples):
+            for t0 in (0, w.ctx // 2 + 3, w.ctx - 5):
+                codes, scales = rows_of(host, lay, b, g, w.n_kv, t0, t0 + 5)
+                ec, es = oracle_rows(kind, new[b, t0:t0 + 5, g, :].cpu().numpy(), w.turbo_seed)
+                np.testing.assert_array_equal(codes, ec)
+                np.testing.assert_array_equal(scales.view(np.uint16), es.view(np.uint16))
+    del kc, vc, k, v
+    torch.cuda.empty_cache()
