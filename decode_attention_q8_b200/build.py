@@ -1,7 +1,7 @@
 """Builds libkvq.so in-tree with nvcc for sm_100a (B200).
 
-    python -m decode_attention_q8_b200.build            # incremental
-    python -m decode_attention_q8_b200.build --force    # rebuild
+    python decode_attention_q8_b200/build.py            # incremental
+    python decode_attention_q8_b200/build.py --force    # rebuild
 
 The library links the CUDA runtime statically, so it loads on a machine
 without a GPU (entry points that only compute sizes work there; launches
@@ -19,7 +19,6 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libkvq.so")
 OBJDIR = os.path.join(HERE, "_build")
 
-SOURCES = ["kvq_api.cu", "append.cu", "decode_cudacore.cu", "combine.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
          "-Xptxas", "-v", "--expt-relaxed-constexpr"]
@@ -50,7 +49,7 @@ def build(force=False, verbose=False):
     os.makedirs(OBJDIR, exist_ok=True)
     objs = []
     nvcc = _nvcc()
-    for src in SOURCES:
+    for src in sorted(f for f in os.listdir(CSRC) if f.endswith(".cu")):
         obj = os.path.join(OBJDIR, src.replace(".cu", ".o"))
         objs.append(obj)
         if force or _stale(obj, deps):
