@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libkvq.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"libkvq.so not found at {LIB_PATH}; build it with "
-        "`python -m decode_attention_q8_b200.build` (nvcc, sm_100a)")
+        "`python decode_attention_q8_b200/build.py` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -33,7 +33,7 @@ EXPORTED = (
     "kvq_status_string", "kvq_last_cuda_error", "kvq_row_bytes", "kvq_check_desc",
     "kvq_cache_layout", "kvq_cache_bytes", "kvq_auto_splits", "kvq_workspace_bytes",
     "kvq_turbo3_codebook", "kvq_turbo3_signs", "kvq_append_quantize",
-    "kvq_decode_attention", "kvq_combine",
+    "kvq_decode_attention", "kvq_combine", "kvq_decode_attention_noalloc",
 )
 
 
@@ -79,6 +79,8 @@ _sigs = {
                                             ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "kvq_combine": (ctypes.c_int, [_D, _P, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
                                    _P, _P]),
+    "kvq_decode_attention_noalloc": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                                                    ctypes.c_int32, _P, _P]),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -196,6 +198,16 @@ def kvq_combine(desc, workspace, batch, ctx_len, n_splits, out, workspace_bytes=
     return _check(_lib.kvq_combine(ctypes.byref(desc), _ptr(workspace), workspace_bytes, batch, ctx_len,
                                    n_splits, _ptr(out), _stream(stream)),
                   "kvq_combine")
+
+
+def kvq_decode_attention_noalloc(desc, k_cache, v_cache, q, batch, ctx_len, softmax_scale, n_splits, out,
+                                 stream=None):
+    """Decode + combine into ``out`` using the library's own 8 MiB per-GPU
+    scratch array instead of a caller workspace (see include/kvq.h)."""
+    return _check(_lib.kvq_decode_attention_noalloc(ctypes.byref(desc), _ptr(k_cache), _ptr(v_cache), _ptr(q),
+                                                    batch, ctx_len, softmax_scale, n_splits, _ptr(out),
+                                                    _stream(stream)),
+                  "kvq_decode_attention_noalloc")
 
 
 def raw_status(name, *args):

@@ -208,6 +208,9 @@ Plane plane_of(const kvq_cache_desc* d, int32_t batch, int which, void* base) {
 }
 
 }  // namespace
+
+void set_last_cuda_error(cudaError_t e) { g_last_cuda_error = cudaGetErrorString(e); }
+
 }  // namespace kvq
 
 using namespace kvq;

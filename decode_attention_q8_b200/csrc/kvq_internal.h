@@ -64,6 +64,7 @@ struct CombineParams {
 int64_t rows_per_plane(int64_t max_ctx);
 int32_t code_bytes_of(int32_t type, int32_t d);
 int32_t n_scales_of(int32_t type, int32_t d);
+void set_last_cuda_error(cudaError_t e);  // text returned by kvq_last_cuda_error()
 
 // Launchers; each returns cudaGetLastError() after its launch.
 cudaError_t launch_append(int32_t type, const AppendParams& p, cudaStream_t st);

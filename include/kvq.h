@@ -207,6 +207,34 @@ KVQ_API kvq_status kvq_combine(const kvq_cache_desc* desc, const void* workspace
                        size_t workspace_bytes, int32_t batch, int64_t ctx_len,
                        int32_t n_splits, float* out, void* cuda_stream);
 
+/*
+ * Allocation-free decode: kvq_decode_attention followed by kvq_combine, with the
+ * split partials kept in scratch memory that the library itself owns, so the
+ * caller passes only inputs and the output.  The pages have no counterpart; it
+ * exists for callers that cannot allocate device memory when they decode (a
+ * fixed memory arena handed out up front, a process that must not call the
+ * allocator during another stream's graph capture, a foreign-language host that
+ * only passes pointers it was given).
+ *   Scratch: one 8 MiB array in each GPU's memory (a file-scope __device__
+ *   variable), held from the library's first use on that GPU until the process
+ *   exits.  Problems whose workspace (kvq_workspace_bytes for the split count
+ *   used) exceeds 8 MiB return KVQ_ERR_WORKSPACE without launching anything.
+ *   Set-up: the first call on a GPU looks up the array's device address there
+ *   (cudaGetSymbolAddress, with that GPU current); make that first call before
+ *   any stream capture.
+ *   Sharing: every call on a GPU uses the same array, which keeps the previous
+ *   call's contents (each call writes every entry before reading it back).
+ *   Calls that overlap on the GPU (unordered streams) race and give wrong
+ *   results; order them on one stream or use kvq_decode_attention with a
+ *   workspace of your own.
+ *   Arguments are those of kvq_decode_attention and kvq_combine;
+ *   out is device fp32 [batch][n_q_heads][head_dim], 16-byte aligned.
+ */
+KVQ_API kvq_status kvq_decode_attention_noalloc(const kvq_cache_desc* desc, const void* k_cache,
+                                                const void* v_cache, const void* q, int32_t batch,
+                                                int64_t ctx_len, float softmax_scale, int32_t n_splits,
+                                                float* out, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif
