@@ -49,16 +49,25 @@ def build(force=False, verbose=False):
     os.makedirs(OBJDIR, exist_ok=True)
     objs = []
     nvcc = _nvcc()
+    procs = []
     for src in sorted(f for f in os.listdir(CSRC) if f.endswith(".cu")):
         obj = os.path.join(OBJDIR, src.replace(".cu", ".o"))
         objs.append(obj)
         if force or _stale(obj, deps):
             cmd = [nvcc, *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", os.path.join(CSRC, src), "-o", obj]
-            r = subprocess.run(cmd, capture_output=True, text=True)
-            if r.returncode != 0:
-                raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
-            if verbose:
-                sys.stderr.write(r.stderr)
+            procs.append((src, obj, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.PIPE,
+                                                     text=True)))
+    failed = []
+    for src, obj, pr in procs:  # translation units compile in parallel
+        out, err = pr.communicate()
+        if pr.returncode != 0:
+            failed.append(f"nvcc failed for {src}:\n{out}\n{err}")
+            if os.path.exists(obj):
+                os.remove(obj)
+        elif verbose:
+            sys.stderr.write(err)
+    if failed:
+        raise RuntimeError("\n".join(failed))
     if force or _stale(LIB, objs):
         cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-Xcompiler", "-fPIC", "-o", LIB, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)

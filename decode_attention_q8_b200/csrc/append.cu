@@ -41,10 +41,10 @@ __device__ __forceinline__ int64_t dst_row(const AppendParams& p, int64_t row) {
 }
 
 // q8_0: d = amax/127; q = roundf(x / d) (IEEE divide per element); d == 0 -> 0.
-__global__ void append_q8_0_kernel(AppendParams p) {
+__device__ __forceinline__ void append_q8_0(const AppendParams& p, int64_t cta) {
   const int nb = p.D / kBlock;
   const int64_t total = (int64_t)p.B * p.n_tok * p.H * nb;
-  const int64_t gblk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
+  const int64_t gblk = (cta * blockDim.x + threadIdx.x) >> 3;
   const int sub = threadIdx.x & 7;
   const bool active = gblk < total;
   float x[4] = {0.f, 0.f, 0.f, 0.f};
@@ -70,10 +70,10 @@ __global__ void append_q8_0_kernel(AppendParams p) {
 
 // q4_0: m = signed max-magnitude element (lowest index on ties); d = m / -8;
 // q = min(15, trunc(fl(fl(x * fl(1/d)) + 8.5))); byte j = q_j | q_{j+16} << 4.
-__global__ void append_q4_0_kernel(AppendParams p) {
+__device__ __forceinline__ void append_q4_0(const AppendParams& p, int64_t cta) {
   const int nb = p.D / kBlock;
   const int64_t total = (int64_t)p.B * p.n_tok * p.H * nb;
-  const int64_t gblk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
+  const int64_t gblk = (cta * blockDim.x + threadIdx.x) >> 3;
   const int sub = threadIdx.x & 7;
   const bool active = gblk < total;
   float x[4] = {0.f, 0.f, 0.f, 0.f};
@@ -112,10 +112,10 @@ __global__ void append_q4_0_kernel(AppendParams p) {
 }
 
 // f16: copy rows, 16 bytes per thread.
-__global__ void append_f16_kernel(AppendParams p) {
+__device__ __forceinline__ void append_f16(const AppendParams& p, int64_t cta) {
   const int per_row = p.D / 8;  // 16-byte chunks per row
   const int64_t total = (int64_t)p.B * p.n_tok * p.H * per_row;
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t i = cta * blockDim.x + threadIdx.x;
   if (i >= total) return;
   const int64_t row = i / per_row;
   const int c = (int)(i % per_row);
@@ -126,10 +126,10 @@ __global__ void append_f16_kernel(AppendParams p) {
 
 // turbo3: one warp per row, E = D/32 contiguous elements per lane.
 template <int E>
-__global__ void append_turbo3_kernel(AppendParams p) {
+__device__ __forceinline__ void append_turbo3(const AppendParams& p, int64_t cta) {
   constexpr int D = 32 * E;
   const int64_t total = (int64_t)p.B * p.n_tok * p.H;
-  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t row = (cta * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= total) return;  // whole warps exit together
   const __half* src = p.src + row * D + lane * E;
@@ -215,41 +215,71 @@ __global__ void append_turbo3_kernel(AppendParams p) {
   if (lane == 0) p.dst.scales[r_dst] = __float2half_rn(fminf(norm, 65504.0f));
 }
 
-}  // namespace
+constexpr int kAppendThreads = 256;
 
-cudaError_t launch_append(int32_t type, const AppendParams& p, cudaStream_t st) {
-  const int threads = 256;
+// CTAs a tensor of `type` needs (each CTA: 256 threads).
+int64_t append_ctas(int32_t type, const AppendParams& p) {
   const int64_t rows = (int64_t)p.B * p.n_tok * p.H;
+  int64_t threads = 0;
   switch (type) {
-    case KVQ_F16: {
-      const int64_t n = rows * (p.D / 8);
-      append_f16_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, st>>>(p);
-      break;
-    }
+    case KVQ_F16: threads = rows * (p.D / 8); break;             // one 16-byte chunk each
     case KVQ_Q8_0:
-    case KVQ_Q4_0: {
-      const int64_t n = rows * (p.D / kBlock) * 8;  // 8 lanes per block
-      const unsigned grid = (unsigned)((n + threads - 1) / threads);
-      if (type == KVQ_Q8_0)
-        append_q8_0_kernel<<<grid, threads, 0, st>>>(p);
-      else
-        append_q4_0_kernel<<<grid, threads, 0, st>>>(p);
-      break;
-    }
-    case KVQ_TURBO3: {
-      const unsigned grid = (unsigned)((rows * 32 + threads - 1) / threads);
+    case KVQ_Q4_0: threads = rows * (p.D / kBlock) * 8; break;   // 8 lanes per block
+    case KVQ_TURBO3: threads = rows * 32; break;                 // a warp per row
+  }
+  return (threads + kAppendThreads - 1) / kAppendThreads;
+}
+
+// K and V rows of one append call in one launch: CTAs [0, ctas0) quantize the
+// first tensor, the rest the second; the branch on the type is uniform per CTA.
+struct AppendPair {
+  AppendParams p[2];
+  int32_t type[2];
+  int64_t ctas0;
+};
+
+__global__ void __launch_bounds__(kAppendThreads) append_pair_kernel(const AppendPair pp) {
+  const int which = (int64_t)blockIdx.x < pp.ctas0 ? 0 : 1;
+  const int64_t cta = which ? (int64_t)blockIdx.x - pp.ctas0 : (int64_t)blockIdx.x;
+  const AppendParams& p = pp.p[which];
+  switch (pp.type[which]) {
+    case KVQ_F16: append_f16(p, cta); break;
+    case KVQ_Q8_0: append_q8_0(p, cta); break;
+    case KVQ_Q4_0: append_q4_0(p, cta); break;
+    case KVQ_TURBO3:
       switch (p.D) {
-        case 32: append_turbo3_kernel<1><<<grid, threads, 0, st>>>(p); break;
-        case 64: append_turbo3_kernel<2><<<grid, threads, 0, st>>>(p); break;
-        case 128: append_turbo3_kernel<4><<<grid, threads, 0, st>>>(p); break;
-        case 256: append_turbo3_kernel<8><<<grid, threads, 0, st>>>(p); break;
-        default: return cudaErrorInvalidValue;
+        case 32: append_turbo3<1>(p, cta); break;
+        case 64: append_turbo3<2>(p, cta); break;
+        case 128: append_turbo3<4>(p, cta); break;
+        case 256: append_turbo3<8>(p, cta); break;
       }
       break;
-    }
-    default:
-      return cudaErrorInvalidValue;
   }
+}
+
+}  // namespace
+
+cudaError_t launch_append(const AppendParams* k, int32_t k_type, const AppendParams* v, int32_t v_type,
+                          cudaStream_t st) {
+  AppendPair pp{};
+  int n = 0;
+  int64_t ctas[2] = {0, 0};
+  if (k) {
+    pp.p[n] = *k;
+    pp.type[n] = k_type;
+    ctas[n++] = append_ctas(k_type, *k);
+  }
+  if (v) {
+    pp.p[n] = *v;
+    pp.type[n] = v_type;
+    ctas[n++] = append_ctas(v_type, *v);
+  }
+  if (n == 0) return cudaSuccess;
+  if (n == 1) ctas[1] = 0;
+  pp.ctas0 = ctas[0];
+  const int64_t total = ctas[0] + ctas[1];
+  if (total <= 0 || total > 0x7fffffff) return cudaErrorInvalidValue;
+  append_pair_kernel<<<(unsigned)total, kAppendThreads, 0, st>>>(pp);
   return cudaGetLastError();
 }
 

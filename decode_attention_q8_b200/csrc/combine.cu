@@ -16,34 +16,66 @@
 namespace kvq {
 namespace {
 
-__global__ void combine_kernel(CombineParams p) {
-  extern __shared__ float x_s[];
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const float x = __shfl_xor_sync(0xffffffffu, v, o);
+    v = is_max ? fmaxf(v, x) : v + x;
+  }
+  __syncthreads();  // red[] may still be read from a previous reduction
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  v = red[0];
+  for (int w = 1; w < nw; ++w) v = is_max ? fmaxf(v, red[w]) : v + red[w];
+  return v;
+}
+
+// One CTA per (query head, batch row), one thread per output dim.  The split
+// partials are read in parallel: the maxima and sums with one load per thread,
+// then every thread's accumulator column with independent loads (the workspace
+// is L2-resident behind the decode kernel).
+__global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
+  extern __shared__ float sm[];
+  float* red = sm;              // 8 floats
+  float* wts = sm + 8;          // S weights
+  float* xs = wts + p.S;        // D values (turbo3 inverse transform)
   const int h = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
   const int64_t base = ((int64_t)b * p.n_q + h) * p.S;
   float M = -INFINITY;
-  for (int s = 0; s < p.S; ++s) M = fmaxf(M, p.ws_m[base + s]);
-  float num = 0.f, den = 0.f;
-  for (int s = 0; s < p.S; ++s) {
+  for (int s = j; s < p.S; s += blockDim.x) M = fmaxf(M, p.ws_m[base + s]);
+  M = block_reduce(M, true, red);
+  float den = 0.f;
+  for (int s = j; s < p.S; s += blockDim.x) {
     const float ms = p.ws_m[base + s];
-    if (ms == -INFINITY) continue;  // empty split
-    const float w = exp2f(ms - M);
-    num += w * p.ws_acc[(base + s) * p.D + j];
+    const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);  // empty split: weight 0
+    wts[s] = w;
     den += w * p.ws_l[base + s];
   }
+  den = block_reduce(den, false, red);  // its barriers also publish wts[]
+  const float* acc = p.ws_acc + base * p.D + j;
+  float num = 0.f;
+  int s = 0;
+  for (; s + 4 <= p.S; s += 4) {
+    const float a0 = acc[(int64_t)(s + 0) * p.D], a1 = acc[(int64_t)(s + 1) * p.D];
+    const float a2 = acc[(int64_t)(s + 2) * p.D], a3 = acc[(int64_t)(s + 3) * p.D];
+    num += wts[s] * a0 + wts[s + 1] * a1 + wts[s + 2] * a2 + wts[s + 3] * a3;
+  }
+  for (; s < p.S; ++s) num += wts[s] * acc[(int64_t)s * p.D];
   float o = num / den;
   if (p.turbo3) {
-    x_s[j] = o;
+    xs[j] = o;
     for (int hs = 1; hs < p.D; hs <<= 1) {
       __syncthreads();
       if ((j & hs) == 0) {
-        const float a = x_s[j], c = x_s[j + hs];
-        x_s[j] = a + c;
-        x_s[j + hs] = a - c;
+        const float a = xs[j], c = xs[j + hs];
+        xs[j] = a + c;
+        xs[j + hs] = a - c;
       }
     }
     __syncthreads();
     const float sgn = ((p.t3.sign_bits[j >> 5] >> (j & 31)) & 1u) ? -1.f : 1.f;
-    o = x_s[j] * sgn / (float)p.D;
+    o = xs[j] * sgn / (float)p.D;
   }
   p.out[((int64_t)b * p.n_q + h) * p.D + j] = o;
 }
@@ -52,7 +84,9 @@ __global__ void combine_kernel(CombineParams p) {
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st) {
   const dim3 grid(p.n_q, p.B);
-  combine_kernel<<<grid, p.D, p.turbo3 ? p.D * sizeof(float) : 0, st>>>(p);
+  const size_t smem = (8 + (size_t)p.S + (size_t)p.D) * sizeof(float);
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;
+  combine_kernel<<<grid, p.D, smem, st>>>(p);
   return cudaGetLastError();
 }
 

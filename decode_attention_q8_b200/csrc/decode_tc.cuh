@@ -1,0 +1,924 @@
+// Split-KV decode attention over a quantized KV cache -- tensor-core version
+// for sm_100a.
+//
+// What it computes is the decode form of flash attention ("llama.cpp für
+// Geschwindigkeit und Speicher optimieren", section "Flash Attention": tiled,
+// exactly standard attention): each CTA owns one (split, KV head, batch row),
+// streams its contiguous slice of cache rows once for the whole GQA group of
+// that KV head, keeps an online softmax and writes (m, l, acc) partials that
+// kvq_combine merges.  Keys and values are decoded from their own cache types
+// ("KV-Cache-Präzision": set independently for K and V; turbo3 values per
+// "Benchmark TurboQuant en Apple Silicon", "¿Qué es TurboQuant?").
+//
+// Why the tensor cores: at the HBM rate a K8V4 row (208 bytes) reaches each SM
+// about every 0.1 cycles, and the G query heads of a group need 2*G*d
+// multiply-adds per row (2048 at G = 8, d = 128) -- far more than the FMA pipes
+// issue in that time.  The QK and PV products of one 16-row tile are
+// m16n8k16 tensor-core MMAs (fp16 operands, fp32 accumulation); the kernel stays
+// bound by HBM bytes.
+//
+// Data movement: every warp runs its own ring of kStages shared-memory stages.
+// Lane 0 fills a stage with cp.async.bulk.tensor copies (TMA) of one 16-row
+// tile -- K codes, K scales, V codes, V scales -- completing on the stage's
+// mbarrier; the code planes are copied with the hardware 32/64/128-byte swizzle
+// so the fragment loads below are free of bank conflicts.  Rows past ctx_len
+// read as zeros (tensor-map bounds).  No warp waits on another warp; every wait
+// is bounded by a wall-clock limit (2 s), after which the warp stops, drains its
+// own copies (bounded again) and the CTA writes NaN partials, so the affected
+// outputs read NaN.
+//
+// Fragment mapping (lane = 4*g + c; MMA row m is tile row m):
+//   QK   S[row][head] = sum_dim K[row][dim] * Q[head][dim]: A = K tile (16
+//        rows) read by ldmatrix from the swizzled stage (8 rows x 16 bytes per
+//        matrix; the swizzle puts the 8 rows in distinct bank groups), B = Q^T
+//        (8 heads), fp32 C.  What ldmatrix hands a lane (4 bytes of a 16-byte
+//        segment) fixes the dim order inside each 32-dim block; Q is loaded in
+//        the same order.  int8 codes enter as fp16 1024 + (k + 128) (an xor and
+//        two byte permutes per four codes), q4_0 nibbles as 1024 + n (one LOP3
+//        per two); the MMA's C input carries -1152 * sum_block(q) (-1032 for
+//        q4_0), so D = sum k*q per block exactly; block scale and
+//        softmax_scale * log2 e are applied in fp32.
+//   P    ex2 of the scores in fp32, rounded to fp16; movmatrix.trans turns the
+//        (row x head) accumulator layout into the (row x head) B operand of PV.
+//   PV   O^T[dim][head] += V^T[dim][row] * P[row][head]: A = V^T (16 dims) by
+//        ldmatrix.trans, which hands a lane the same two bytes of rows 2c and
+//        2c+1 in one register -- exactly the pair an A fragment holds -- so the
+//        codes only need masking into fp16 (q4_0: 1024 + n, minus 1032) or an
+//        xor and a permute (q8_0).  Each row's block scale (turbo3: its norm)
+//        multiplies P in fp16; the codes stay exact small integers (turbo3: the
+//        codebook level, from a per-lane replicated 64-entry pair table).
+//   turbo3 values accumulate in the rotated domain; kvq_combine rotates back.
+#pragma once
+
+#include <cuda.h>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace tc {
+
+constexpr int kNWMax = 8;    // warps per CTA (4 for the widest f16 stages)
+constexpr int kSub = 32;     // cache rows per warp tile (one TMA box per plane)
+constexpr int kHalf = 16;    // rows per MMA row block (two per tile)
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+
+__host__ __device__ constexpr int code_bytes(int t, int d) {
+  return t == KVQ_F16 ? 2 * d : t == KVQ_Q8_0 ? d : t == KVQ_Q4_0 ? d / 2 : 3 * d / 8;
+}
+__host__ __device__ constexpr int n_scales(int t, int d) {
+  return t == KVQ_F16 ? 0 : t == KVQ_TURBO3 ? 1 : d / 32;
+}
+// swizzle of a code plane: 16-byte chunk index XOR ((offset >> 7) & mask)
+__host__ __device__ constexpr int swz_mask(int t, int d) {
+  return t == KVQ_TURBO3 ? 0 : (code_bytes(t, d) >= 128 ? 8 : code_bytes(t, d) / 16) - 1;
+}
+__host__ __device__ constexpr int round_up_c(int v, int a) { return (v + a - 1) / a * a; }
+__host__ __device__ constexpr int stage_bytes(int kt, int vt, int d) {
+  return round_up_c(kSub * code_bytes(kt, d), 1024) +
+         round_up_c(kSub * code_bytes(vt, d), vt == KVQ_TURBO3 ? 128 : 1024) +
+         round_up_c(kSub * n_scales(kt, d) * 2, 128) + round_up_c(kSub * n_scales(vt, d) * 2, 128);
+}
+// Warps per CTA: 8 while two 2-stage rings per warp fit in ~110 KB (two CTAs per
+// SM), else 4 (one CTA per SM).  Stages per warp ring: up to 4, as many as fit.
+__host__ __device__ constexpr int warps_for(int kt, int vt, int d) {
+  return kNWMax * 2 * stage_bytes(kt, vt, d) <= 112640 ? kNWMax : kNWMax / 2;
+}
+__host__ __device__ constexpr int stages_for(int kt, int vt, int d) {
+  return (112640 / (warps_for(kt, vt, d) * stage_bytes(kt, vt, d))) >= 4 ? 4
+         : (112640 / (warps_for(kt, vt, d) * stage_bytes(kt, vt, d))) >= 3 ? 3 : 2;
+}
+
+template <int KT, int VT, int D>
+struct Layout {
+  static constexpr int NW = warps_for(KT, VT, D);
+  static constexpr int kStages = stages_for(KT, VT, D);
+  static constexpr int RBK = code_bytes(KT, D), RBV = code_bytes(VT, D);
+  static constexpr int NSK = n_scales(KT, D), NSV = n_scales(VT, D);
+  static constexpr int KC = round_up_c(kSub * RBK, 1024);
+  static constexpr int VC = round_up_c(kSub * RBV, VT == KVQ_TURBO3 ? 128 : 1024);
+  static constexpr int KS = round_up_c(kSub * NSK * 2, 128);
+  static constexpr int VS = round_up_c(kSub * NSV * 2, 128);
+  static constexpr int STAGE = KC + VC + KS + VS;
+  static constexpr int WARP = round_up_c(kStages * STAGE, 1024);
+  static constexpr int TABLE = VT == KVQ_TURBO3 ? 64 * 32 * 4 : 0;
+  static constexpr int BARS = NW * kStages * 8;
+  static constexpr int TX = kSub * (RBK + 2 * NSK + RBV + 2 * NSV);  // bytes landing per tile
+  // CTA-level merge scratch (reuses the stage memory after the main loop)
+  static constexpr int MERGE_HEADS = 8;
+  static constexpr int MERGE = NW * MERGE_HEADS * (D + 2) * 4;
+  static constexpr int TOTAL = 1024 + NW * WARP + TABLE + BARS + 16;
+  static_assert(MERGE <= NW * WARP, "merge area must fit in the stage memory");
+  static_assert(TOTAL <= 227 * 1024, "shared memory per CTA");
+};
+
+// ------------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits for phase `parity` of `bar`; false after kWaitLimitNs of wall time.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+      "%5}], [%6];" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mma16816(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1, const float c[4]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%11,%12,%13};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t r[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t r[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+
+// 2^x by the SFU's ex2 (about 2 ulp; subnormal results flush to 0, which only
+// drops weights below 2^-126)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
+  return (a & mask) | orv;  // one LOP3
+}
+
+__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
+  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
+  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b),
+                      *reinterpret_cast<__half2*>(&c));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int MASK>
+__device__ __forceinline__ int swz(int off) {
+  return off ^ (((off >> 7) & MASK) << 4);
+}
+
+constexpr uint32_t kMagic = 0x64006400u;   // fp16 1024 in both halves
+constexpr uint32_t kBias1032 = 0x64086408u;  // fp16 1032 (1024 + 8)
+constexpr uint32_t kBias1152 = 0x64806480u;  // fp16 1152 (1024 + 128)
+
+// ------------------------------------------------------------------ kernel
+
+struct TcArgs {
+  DecodeParams p;
+};
+
+template <int KT, int VT, int NB, int NTH>
+__global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
+                                  (NB >= 8 || NTH == 2 || warps_for(KT, VT, NB * 32) < kNWMax) ? 1 : 2)
+    decode_tc_kernel(const TcArgs args, const __grid_constant__ CUtensorMap tm_kc,
+                     const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vc,
+                     const __grid_constant__ CUtensorMap tm_vs) {
+  constexpr int D = NB * 32;
+  using L = Layout<KT, VT, D>;
+  constexpr int S = L::kStages;
+  constexpr int KMASK = swz_mask(KT, D), VMASK = swz_mask(VT, D);
+  constexpr int NMT = D / 16;  // PV m-tiles
+  const DecodeParams& p = args.p;
+
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  unsigned char* wbase = smem + warp * L::WARP;
+  __shared__ int cta_failed;
+  uint32_t* table = reinterpret_cast<uint32_t*>(smem + L::NW * L::WARP);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::NW * L::WARP + L::TABLE) + warp * S;
+
+  const int s_idx = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int64_t t0 = (int64_t)s_idx * p.chunk;
+  const int64_t t1 = min(p.ctx, t0 + p.chunk);
+  const int n_sub = t0 < t1 ? (int)((t1 - t0 + kSub - 1) / kSub) : 0;
+  const int plane = b * p.n_kv + kvh;
+
+  if (threadIdx.x == 0) cta_failed = 0;
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+  if (VT == KVQ_TURBO3) {
+    // table[idx6 * 32 + lane] = half2(c[idx6 & 7], c[idx6 >> 3]); one copy per bank
+    for (int e = threadIdx.x; e < 64 * 32; e += L::NW * 32) {
+      const int idx = e >> 5;
+      table[e] = pack_half2(p.t3.levels[idx & 7], p.t3.levels[idx >> 3]);
+    }
+  }
+  __syncthreads();
+
+  auto kc_of = [&](int st) { return wbase + st * L::KC; };
+  auto vc_of = [&](int st) { return wbase + S * L::KC + st * L::VC; };
+  auto ks_of = [&](int st) { return wbase + S * (L::KC + L::VC) + st * L::KS; };
+  auto vs_of = [&](int st) { return wbase + S * (L::KC + L::VC + L::KS) + st * L::VS; };
+
+  // tile j of this warp covers rows t0 + 32*(warp + NW*j) ...
+  const int my_tiles = n_sub > warp ? (n_sub - warp + L::NW - 1) / L::NW : 0;
+  auto issue = [&](int j) {
+    const int st = j % S;
+    const int r0 = (int)(t0 + (int64_t)kSub * (warp + L::NW * j));
+    mbar_expect_tx(&bars[st], L::TX);
+    if (L::RBK > 128)
+      tma_load_4d(kc_of(st), &tm_kc, 0, 0, r0, plane, &bars[st]);
+    else
+      tma_load_3d(kc_of(st), &tm_kc, 0, r0, plane, &bars[st]);
+    if (L::NSK) tma_load_2d(ks_of(st), &tm_ks, r0 * L::NSK / 2, plane, &bars[st]);
+    if (VT == KVQ_TURBO3) {
+      if (kSub * L::RBV / 4 <= 256)
+        tma_load_2d(vc_of(st), &tm_vc, r0 * L::RBV / 4, plane, &bars[st]);
+      else
+        tma_load_3d(vc_of(st), &tm_vc, 0, r0, plane, &bars[st]);
+    } else if (L::RBV > 128) {
+      tma_load_4d(vc_of(st), &tm_vc, 0, 0, r0, plane, &bars[st]);
+    } else {
+      tma_load_3d(vc_of(st), &tm_vc, 0, r0, plane, &bars[st]);
+    }
+    if (L::NSV) tma_load_2d(vs_of(st), &tm_vs, r0 * L::NSV / 2, plane, &bars[st]);
+  };
+  if (lane == 0) {
+    for (int j = 0; j < S && j < my_tiles; ++j) issue(j);
+  }
+
+  // ---- queries: B fragments of Q^T per (block, k-step) and the per-block
+  //      correction -bias * sum(q) for heads 2c, 2c+1 of each n-tile.  The dim
+  //      order inside a block follows the A-operand loads below (lane = 4g + c):
+  //        q8_0  k-step s = 16-byte segment 2*blk+s; lane c holds bytes 4c..4c+3:
+  //              cols 2c,2c+1 <- bytes 4c,4c+1 and cols 2c+8,2c+9 <- 4c+2,4c+3
+  //        q4_0  lane c holds bytes 4c..4c+3 of the block; low nibbles (dims
+  //              4c..4c+3) feed k-step 0, high nibbles (4c+16..4c+19) k-step 1;
+  //              cols 2c,2c+1 <- dims (4c, 4c+2), cols 2c+8,2c+9 <- (4c+1, 4c+3)
+  //        f16   natural: k-step s covers dims 32*blk + 16*s .. +15
+  uint32_t qb[NTH][NB][2][2];
+  float corr[NTH][NB][2];
+  const float bias = KT == KVQ_Q8_0 ? 1152.f : KT == KVQ_Q4_0 ? 1032.f : 0.f;
+#pragma unroll
+  for (int nt = 0; nt < NTH; ++nt) {
+    const int head = nt * 8 + g;
+    const bool hv = head < p.G;
+    const __half* qrow = p.q + ((int64_t)b * p.n_q + (int64_t)kvh * p.G + (hv ? head : 0)) * D;
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
+      uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
+      if (hv) {
+        if (KT == KVQ_Q4_0) {
+          const uint2 lo = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 4 * c);       // dims 4c..4c+3
+          const uint2 hi = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 16 + 4 * c);  // 4c+16..
+          w0 = prmt(lo.x, lo.y, 0x5410);  // (4c, 4c+2)
+          w1 = prmt(lo.x, lo.y, 0x7632);  // (4c+1, 4c+3)
+          w2 = prmt(hi.x, hi.y, 0x5410);
+          w3 = prmt(hi.x, hi.y, 0x7632);
+        } else if (KT == KVQ_Q8_0) {
+          const uint2 s0 = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 4 * c);       // segment 0
+          const uint2 s1 = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 16 + 4 * c);  // segment 1
+          w0 = s0.x;
+          w1 = s0.y;
+          w2 = s1.x;
+          w3 = s1.y;
+        } else {
+          w0 = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 2 * c);
+          w1 = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 8 + 2 * c);
+          w2 = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 16 + 2 * c);
+          w3 = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 24 + 2 * c);
+        }
+      }
+      qb[nt][blk][0][0] = w0;
+      qb[nt][blk][0][1] = w1;
+      qb[nt][blk][1][0] = w2;
+      qb[nt][blk][1][1] = w3;
+      // partial sum of this lane's 8 dims of head g, then over the 4 lanes of the group
+      float part = 0.f;
+      const uint32_t ws[4] = {w0, w1, w2, w3};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[i]));
+        part += f.x + f.y;
+      }
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      part += __shfl_xor_sync(0xffffffffu, part, 2);
+      // lane (g', c') needs the sums of heads 2c', 2c'+1 (held by groups 2c', 2c'+1)
+      const float s0 = __shfl_sync(0xffffffffu, part, (2 * c) * 4);
+      const float s1 = __shfl_sync(0xffffffffu, part, (2 * c + 1) * 4);
+      corr[nt][blk][0] = -bias * s0;
+      corr[nt][blk][1] = -bias * s1;
+    }
+  }
+
+  // ---- running state
+  float m_run[NTH][2], l_run[NTH][2];
+  float acc[NTH][NMT][4];
+#pragma unroll
+  for (int nt = 0; nt < NTH; ++nt) {
+    m_run[nt][0] = m_run[nt][1] = -INFINITY;
+    l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+    for (int i = 0; i < NMT; ++i) acc[nt][i][0] = acc[nt][i][1] = acc[nt][i][2] = acc[nt][i][3] = 0.f;
+  }
+
+  // ldmatrix addressing: this lane supplies the address of tile row lm_row in
+  // matrix lane >> 3; lm_hi selects the second segment / block of an x4 load
+  const int lm_row = (lane & 7) + 8 * ((lane >> 3) & 1);
+  const int lm_hi = lane >> 4;
+  int failed_at = -1;  // tile whose wait timed out (warp-uniform), -1 if none
+
+  // QK of one 16-row tile: scaled scores S[row][head] of rows g, g+8 (heads 2c, 2c+1)
+  auto qk_tile = [&](const unsigned char* kc, const __half* ksc, float (&sc)[NTH][4]) {
+    // ---------------- QK: S[row][head] for rows g, g+8
+#pragma unroll
+    for (int nt = 0; nt < NTH; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    float dA[NB], dB[NB];  // block scales of rows g and g+8
+    if (L::NSK) {
+      uint32_t sa[NB / 2], sb[NB / 2];
+      if (NB == 2) {
+        sa[0] = *reinterpret_cast<const uint32_t*>(ksc + g * L::NSK);
+        sb[0] = *reinterpret_cast<const uint32_t*>(ksc + (g + 8) * L::NSK);
+      } else {
+#pragma unroll
+        for (int i = 0; i < NB / 4; ++i) {
+          const uint2 xa = *reinterpret_cast<const uint2*>(ksc + g * L::NSK + 4 * i);
+          const uint2 xb = *reinterpret_cast<const uint2*>(ksc + (g + 8) * L::NSK + 4 * i);
+          sa[2 * i] = xa.x;
+          sa[2 * i + 1] = xa.y;
+          sb[2 * i] = xb.x;
+          sb[2 * i + 1] = xb.y;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < NB / 2; ++i) {
+        const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&sa[i]));
+        const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&sb[i]));
+        dA[2 * i] = fa.x;
+        dA[2 * i + 1] = fa.y;
+        dB[2 * i] = fb.x;
+        dB[2 * i + 1] = fb.y;
+      }
+    }
+    uint32_t kr[4];  // q4_0 keys: one x4 load per two blocks
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
+      uint32_t a[2][4];  // [k-step][a0..a3]
+      if constexpr (KT == KVQ_Q8_0) {
+        uint32_t r[4];
+        ldmatrix_x4(r, kc + swz<KMASK>(lm_row * L::RBK + 16 * (2 * blk + lm_hi)));
+        const uint32_t u0 = r[0] ^ 0x80808080u, u1 = r[1] ^ 0x80808080u;
+        const uint32_t u2 = r[2] ^ 0x80808080u, u3 = r[3] ^ 0x80808080u;
+        a[0][0] = prmt(u0, 0x64646464u, 0x4140);
+        a[0][2] = prmt(u0, 0x64646464u, 0x4342);
+        a[0][1] = prmt(u1, 0x64646464u, 0x4140);
+        a[0][3] = prmt(u1, 0x64646464u, 0x4342);
+        a[1][0] = prmt(u2, 0x64646464u, 0x4140);
+        a[1][2] = prmt(u2, 0x64646464u, 0x4342);
+        a[1][1] = prmt(u3, 0x64646464u, 0x4140);
+        a[1][3] = prmt(u3, 0x64646464u, 0x4342);
+      } else if constexpr (KT == KVQ_Q4_0) {
+        // one x4 load covers blocks blk (regs 0, 1) and blk + 1 (regs 2, 3):
+        // reg = bytes 4c..4c+3 of the block in row g (even regs) or g+8 (odd)
+        if ((blk & 1) == 0) ldmatrix_x4(kr, kc + swz<KMASK>(lm_row * L::RBK + 16 * (blk + lm_hi)));
+        const uint32_t wa = kr[(blk & 1) * 2], wb = kr[(blk & 1) * 2 + 1];
+        a[0][0] = lop_and_or(wa, 0x000F000Fu, kMagic);        // dims (4c, 4c+2)
+        a[0][2] = lop_and_or(wa >> 8, 0x000F000Fu, kMagic);   // dims (4c+1, 4c+3)
+        a[1][0] = lop_and_or(wa >> 4, 0x000F000Fu, kMagic);   // dims (4c+16, 4c+18)
+        a[1][2] = lop_and_or(wa >> 12, 0x000F000Fu, kMagic);  // dims (4c+17, 4c+19)
+        a[0][1] = lop_and_or(wb, 0x000F000Fu, kMagic);
+        a[0][3] = lop_and_or(wb >> 8, 0x000F000Fu, kMagic);
+        a[1][1] = lop_and_or(wb >> 4, 0x000F000Fu, kMagic);
+        a[1][3] = lop_and_or(wb >> 12, 0x000F000Fu, kMagic);
+      } else {  // f16
+#pragma unroll
+        for (int s2 = 0; s2 < 2; ++s2) {
+          uint32_t r[4];
+          ldmatrix_x4(r, kc + swz<KMASK>(lm_row * L::RBK + 64 * blk + 32 * s2 + 16 * lm_hi));
+          a[s2][0] = r[0];
+          a[s2][1] = r[1];
+          a[s2][2] = r[2];
+          a[s2][3] = r[3];
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < NTH; ++nt) {
+        float dblk[4];
+        const float cin[4] = {corr[nt][blk][0], corr[nt][blk][1], corr[nt][blk][0], corr[nt][blk][1]};
+        mma16816(dblk, a[0][0], a[0][1], a[0][2], a[0][3], qb[nt][blk][0][0], qb[nt][blk][0][1], cin);
+        mma16816(dblk, a[1][0], a[1][1], a[1][2], a[1][3], qb[nt][blk][1][0], qb[nt][blk][1][1], dblk);
+        if (L::NSK) {
+          sc[nt][0] = fmaf(dA[blk], dblk[0], sc[nt][0]);
+          sc[nt][1] = fmaf(dA[blk], dblk[1], sc[nt][1]);
+          sc[nt][2] = fmaf(dB[blk], dblk[2], sc[nt][2]);
+          sc[nt][3] = fmaf(dB[blk], dblk[3], sc[nt][3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sc[nt][i] += dblk[i];
+        }
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NTH; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sc[nt][i] *= p.qscale;
+  };
+
+  // PV of one 16-row tile with its P fragments (rows 2c, 2c+1 | 2c+8, 2c+9)
+  auto pv_tile = [&](const unsigned char* vc, const __half* vsc, const uint32_t (&pb)[NTH][2], bool tail,
+                     uint32_t pmask_lo, uint32_t pmask_hi) {
+    // ---------------- PV
+    if constexpr (VT == KVQ_F16) {
+#pragma unroll
+      for (int mt = 0; mt < NMT; ++mt) {
+        const int jm = lane >> 3;
+        const int krow = (lane & 7) + 8 * (jm >> 1);
+        uint32_t a[4];
+        ldmatrix_x4_trans(a, vc + swz<VMASK>(krow * L::RBV + 2 * (16 * mt + 8 * (jm & 1))));
+#pragma unroll
+        for (int nt = 0; nt < NTH; ++nt) {
+          uint32_t b0 = pb[nt][0], b1 = pb[nt][1];
+          if (tail) {
+            b0 &= pmask_lo;
+            b1 &= pmask_hi;
+          }
+          mma16816(acc[nt][mt], a[0], a[1], a[2], a[3], b0, b1, acc[nt][mt]);
+        }
+      }
+    } else if constexpr (VT == KVQ_TURBO3) {
+      // lane g owns dims [g*D/8, (g+1)*D/8): 3*D/8 bits of each row's codes
+      constexpr int BITS = 3 * D / 8;
+      constexpr int BYTE0_STEP = BITS / 8;  // bytes per lane group
+      auto field = [&](int row) -> unsigned long long {
+        const int byte0 = g * BYTE0_STEP;
+        const int w0 = byte0 >> 2;
+        const unsigned char* rp = vc + row * L::RBV;
+        unsigned long long v = *reinterpret_cast<const uint32_t*>(rp + 4 * w0);
+        if (BITS + 8 * (byte0 & 3) > 32)
+          v |= (unsigned long long)(*reinterpret_cast<const uint32_t*>(rp + 4 * w0 + 4)) << 32;
+        return v >> (8 * (byte0 & 3));
+      };
+      // norms of rows (2c, 2c+1) and (2c+8, 2c+9) are adjacent fp16 pairs
+      const uint32_t nAB = *reinterpret_cast<const uint32_t*>(vsc + 2 * c);
+      const uint32_t nCD = *reinterpret_cast<const uint32_t*>(vsc + 2 * c + 8);
+      uint32_t pbw[NTH][2];
+#pragma unroll
+      for (int nt = 0; nt < NTH; ++nt) {
+        pbw[nt][0] = hmul2_u32(pb[nt][0], nAB);
+        pbw[nt][1] = hmul2_u32(pb[nt][1], nCD);
+        if (tail) {
+          pbw[nt][0] &= pmask_lo;
+          pbw[nt][1] &= pmask_hi;
+        }
+      }
+      if (D <= 128) {
+        const unsigned long long fA = field(2 * c), fB = field(2 * c + 1);
+        const unsigned long long fC = field(2 * c + 8), fD = field(2 * c + 9);
+#pragma unroll
+        for (int mt = 0; mt < NMT; ++mt) {
+          const uint32_t xA = (uint32_t)(fA >> (6 * mt)) & 63u, xB = (uint32_t)(fB >> (6 * mt)) & 63u;
+          const uint32_t xC = (uint32_t)(fC >> (6 * mt)) & 63u, xD = (uint32_t)(fD >> (6 * mt)) & 63u;
+          uint32_t a[4];
+          a[0] = table[(((xA & 7u) | ((xB & 7u) << 3)) << 5) + lane];
+          a[1] = table[(((xA >> 3) | (xB & 0x38u)) << 5) + lane];
+          a[2] = table[(((xC & 7u) | ((xD & 7u) << 3)) << 5) + lane];
+          a[3] = table[(((xC >> 3) | (xD & 0x38u)) << 5) + lane];
+#pragma unroll
+          for (int nt = 0; nt < NTH; ++nt)
+            mma16816(acc[nt][mt], a[0], a[1], a[2], a[3], pbw[nt][0], pbw[nt][1], acc[nt][mt]);
+        }
+      } else {
+        // D = 256: 96 bits per lane group, read as two 48-bit halves
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          auto field48 = [&](int row) -> unsigned long long {
+            const unsigned char* rp = vc + row * L::RBV + g * 12 + half * 6;
+            const unsigned long long lo = *reinterpret_cast<const uint16_t*>(rp);
+            const unsigned long long mid = *reinterpret_cast<const uint16_t*>(rp + 2);
+            const unsigned long long hi = *reinterpret_cast<const uint16_t*>(rp + 4);
+            return lo | (mid << 16) | (hi << 32);
+          };
+          const unsigned long long fA = field48(2 * c), fB = field48(2 * c + 1);
+          const unsigned long long fC = field48(2 * c + 8), fD = field48(2 * c + 9);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int mt = half * 8 + k;
+            const uint32_t xA = (uint32_t)(fA >> (6 * k)) & 63u, xB = (uint32_t)(fB >> (6 * k)) & 63u;
+            const uint32_t xC = (uint32_t)(fC >> (6 * k)) & 63u, xD = (uint32_t)(fD >> (6 * k)) & 63u;
+            uint32_t a[4];
+            a[0] = table[(((xA & 7u) | ((xB & 7u) << 3)) << 5) + lane];
+            a[1] = table[(((xA >> 3) | (xB & 0x38u)) << 5) + lane];
+            a[2] = table[(((xC & 7u) | ((xD & 7u) << 3)) << 5) + lane];
+            a[3] = table[(((xC >> 3) | (xD & 0x38u)) << 5) + lane];
+#pragma unroll
+            for (int nt = 0; nt < NTH; ++nt)
+              mma16816(acc[nt][mt], a[0], a[1], a[2], a[3], pbw[nt][0], pbw[nt][1], acc[nt][mt]);
+          }
+        }
+      }
+    } else {
+      // q8_0 / q4_0 values: per 32-dim block two m-tiles; each row's block scale
+      // multiplies P.  Scales of rows (2c, 2c+1) and (2c+8, 2c+9) are adjacent.
+      uint32_t sAB[L::NSV > 0 ? L::NSV : 1], sCD[L::NSV > 0 ? L::NSV : 1];  // words: row 2c blocks | row 2c+1 blocks
+      if (L::NSV == 2) {
+        const uint2 x = *reinterpret_cast<const uint2*>(vsc + 2 * c * L::NSV);
+        const uint2 y = *reinterpret_cast<const uint2*>(vsc + (2 * c + 8) * L::NSV);
+        sAB[0] = x.x; sAB[1] = x.y; sCD[0] = y.x; sCD[1] = y.y;
+      } else {
+#pragma unroll
+        for (int i = 0; i < L::NSV / 4; ++i) {
+          const uint4 x = *reinterpret_cast<const uint4*>(vsc + 2 * c * L::NSV + 8 * i);
+          const uint4 y = *reinterpret_cast<const uint4*>(vsc + (2 * c + 8) * L::NSV + 8 * i);
+          sAB[4 * i] = x.x; sAB[4 * i + 1] = x.y; sAB[4 * i + 2] = x.z; sAB[4 * i + 3] = x.w;
+          sCD[4 * i] = y.x; sCD[4 * i + 1] = y.y; sCD[4 * i + 2] = y.z; sCD[4 * i + 3] = y.w;
+        }
+      }
+      uint32_t vr[4];  // q4_0: one x4 load per two blocks
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk) {
+        // row 2c's scales are words 0 .. NSV/2-1, row 2c+1's are NSV/2 ..
+        const uint32_t sel = (blk & 1) ? 0x7632u : 0x5410u;
+        const uint32_t dAB = prmt(sAB[blk >> 1], sAB[L::NSV / 2 + (blk >> 1)], sel);
+        const uint32_t dCD = prmt(sCD[blk >> 1], sCD[L::NSV / 2 + (blk >> 1)], sel);
+        uint32_t pbw[NTH][2];
+#pragma unroll
+        for (int nt = 0; nt < NTH; ++nt) {
+          pbw[nt][0] = hmul2_u32(pb[nt][0], dAB);
+          pbw[nt][1] = hmul2_u32(pb[nt][1], dCD);
+          if (tail) {
+            pbw[nt][0] &= pmask_lo;
+            pbw[nt][1] &= pmask_hi;
+          }
+        }
+        uint32_t a0[4], a1[4];  // m-tiles (blk, 0) and (blk, 1)
+        if (VT == KVQ_Q4_0) {
+          // trans load: reg = [row 2c: bytes 2g, 2g+1 | row 2c+1: bytes 2g, 2g+1]
+          // of the block -> dims 2g, 2g+1 (low nibbles), 2g+16, 2g+17 (high)
+          if ((blk & 1) == 0) ldmatrix_x4_trans(vr, vc + swz<VMASK>(lm_row * L::RBV + 16 * (blk + lm_hi)));
+          const uint32_t w1 = vr[(blk & 1) * 2], w2 = vr[(blk & 1) * 2 + 1];
+          const uint32_t w1s = w1 >> 8, w2s = w2 >> 8;
+          a0[0] = hsub2_u32(lop_and_or(w1, 0x000F000Fu, kMagic), kBias1032);   // dim 2g, rows 2c,2c+1
+          a0[1] = hsub2_u32(lop_and_or(w1s, 0x000F000Fu, kMagic), kBias1032);  // dim 2g+1
+          a0[2] = hsub2_u32(lop_and_or(w2, 0x000F000Fu, kMagic), kBias1032);   // dim 2g, rows 2c+8,2c+9
+          a0[3] = hsub2_u32(lop_and_or(w2s, 0x000F000Fu, kMagic), kBias1032);
+          // high nibbles: 1024 + 16 n -> (x / 16) - 72 = n - 8
+          const uint32_t sc16 = 0x2C002C00u;   // fp16 1/16
+          const uint32_t m72 = 0xD480D480u;    // fp16 -72
+          a1[0] = hfma2_u32(lop_and_or(w1, 0x00F000F0u, kMagic), sc16, m72);
+          a1[1] = hfma2_u32(lop_and_or(w1s, 0x00F000F0u, kMagic), sc16, m72);
+          a1[2] = hfma2_u32(lop_and_or(w2, 0x00F000F0u, kMagic), sc16, m72);
+          a1[3] = hfma2_u32(lop_and_or(w2s, 0x00F000F0u, kMagic), sc16, m72);
+        } else {
+          // q8_0 trans load of segments 2blk (regs 0, 1) and 2blk+1 (regs 2, 3):
+          // reg = [row 2c: bytes 2g, 2g+1 | row 2c+1: bytes 2g, 2g+1]
+          ldmatrix_x4_trans(vr, vc + swz<VMASK>(lm_row * L::RBV + 16 * (2 * blk + lm_hi)));
+          const uint32_t x0 = vr[0] ^ 0x80808080u, x1 = vr[1] ^ 0x80808080u;
+          const uint32_t y0 = vr[2] ^ 0x80808080u, y1 = vr[3] ^ 0x80808080u;
+          a0[0] = hsub2_u32(prmt(x0, 0x64646464u, 0x4240), kBias1152);  // dim 2g
+          a0[1] = hsub2_u32(prmt(x0, 0x64646464u, 0x4341), kBias1152);  // dim 2g+1
+          a0[2] = hsub2_u32(prmt(x1, 0x64646464u, 0x4240), kBias1152);
+          a0[3] = hsub2_u32(prmt(x1, 0x64646464u, 0x4341), kBias1152);
+          a1[0] = hsub2_u32(prmt(y0, 0x64646464u, 0x4240), kBias1152);  // dim 16+2g
+          a1[1] = hsub2_u32(prmt(y0, 0x64646464u, 0x4341), kBias1152);  // dim 16+2g+1
+          a1[2] = hsub2_u32(prmt(y1, 0x64646464u, 0x4240), kBias1152);
+          a1[3] = hsub2_u32(prmt(y1, 0x64646464u, 0x4341), kBias1152);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NTH; ++nt) {
+          mma16816(acc[nt][2 * blk], a0[0], a0[1], a0[2], a0[3], pbw[nt][0], pbw[nt][1], acc[nt][2 * blk]);
+          mma16816(acc[nt][2 * blk + 1], a1[0], a1[1], a1[2], a1[3], pbw[nt][0], pbw[nt][1],
+                   acc[nt][2 * blk + 1]);
+        }
+      }
+    }
+
+  };
+
+#pragma unroll 1
+  for (int j = 0; j < my_tiles; ++j) {
+    // one 32-row tile per iteration, as two 16-row MMA halves (the second may
+    // lie past the split end): one wait and one refill per 32 rows
+    const int st = j % S;
+    const bool ok = mbar_wait(&bars[st], (uint32_t)((j / S) & 1));
+    if (!__all_sync(0xffffffffu, ok)) {
+      failed_at = j;
+      break;
+    }
+    const int64_t r0 = t0 + (int64_t)kSub * (warp + L::NW * j);
+    const int nv0 = (int)(t1 - r0 < kHalf ? t1 - r0 : kHalf);
+    const int64_t rem1 = t1 - r0 - kHalf;
+    const int nv1 = rem1 <= 0 ? 0 : (int)(rem1 < kHalf ? rem1 : kHalf);
+    const bool two = nv1 > 0;
+    const bool tail0 = nv0 < kHalf, tail1 = two && nv1 < kHalf;
+    const unsigned char* kc0 = kc_of(st);
+    const __half* ks0 = reinterpret_cast<const __half*>(ks_of(st));
+    const unsigned char* vc0 = vc_of(st);
+    const __half* vs0 = reinterpret_cast<const __half*>(vs_of(st));
+
+    float sc0[NTH][4], sc1[NTH][4];
+    qk_tile(kc0, ks0, sc0);
+    if (two) {
+      qk_tile(kc0 + kHalf * L::RBK, ks0 + kHalf * L::NSK, sc1);
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < NTH; ++nt) sc1[nt][0] = sc1[nt][1] = sc1[nt][2] = sc1[nt][3] = -INFINITY;
+    }
+    if (tail0 || tail1 || !two) {
+#pragma unroll
+      for (int nt = 0; nt < NTH; ++nt) {
+        if (g >= nv0) sc0[nt][0] = sc0[nt][1] = -INFINITY;
+        if (g + 8 >= nv0) sc0[nt][2] = sc0[nt][3] = -INFINITY;
+        if (g >= nv1) sc1[nt][0] = sc1[nt][1] = -INFINITY;
+        if (g + 8 >= nv1) sc1[nt][2] = sc1[nt][3] = -INFINITY;
+      }
+    }
+
+    // ---------------- online softmax over the 32 rows (heads 2c, 2c+1)
+    uint32_t pb0[NTH][2], pb1[NTH][2];
+#pragma unroll
+    for (int nt = 0; nt < NTH; ++nt) {
+      float mx0 = fmaxf(fmaxf(sc0[nt][0], sc0[nt][2]), fmaxf(sc1[nt][0], sc1[nt][2]));
+      float mx1 = fmaxf(fmaxf(sc0[nt][1], sc0[nt][3]), fmaxf(sc1[nt][1], sc1[nt][3]));
+#pragma unroll
+      for (int o = 4; o <= 16; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+      const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
+      m_run[nt][0] = mn0;
+      m_run[nt][1] = mn1;
+      const float p0 = fast_exp2(sc0[nt][0] - mn0), p1 = fast_exp2(sc0[nt][1] - mn1);
+      const float p2 = fast_exp2(sc0[nt][2] - mn0), p3 = fast_exp2(sc0[nt][3] - mn1);
+      const float q0 = fast_exp2(sc1[nt][0] - mn0), q1 = fast_exp2(sc1[nt][1] - mn1);
+      const float q2 = fast_exp2(sc1[nt][2] - mn0), q3 = fast_exp2(sc1[nt][3] - mn1);
+      l_run[nt][0] = fmaf(l_run[nt][0], al0, (p0 + p2) + (q0 + q2));
+      l_run[nt][1] = fmaf(l_run[nt][1], al1, (p1 + p3) + (q1 + q3));
+      if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+        for (int i = 0; i < NMT; ++i) {
+          acc[nt][i][0] *= al0;
+          acc[nt][i][1] *= al1;
+          acc[nt][i][2] *= al0;
+          acc[nt][i][3] *= al1;
+        }
+      }
+      pb0[nt][0] = movmatrix_trans(pack_half2(p0, p1));
+      pb0[nt][1] = movmatrix_trans(pack_half2(p2, p3));
+      pb1[nt][0] = movmatrix_trans(pack_half2(q0, q1));
+      pb1[nt][1] = movmatrix_trans(pack_half2(q2, q3));
+    }
+    // In a tail tile, P rows past the split end contribute exactly 0 whatever
+    // the row's scale holds (b operand halves: rows 2c, 2c+1 | 2c+8, 2c+9).
+    auto pmask = [&](int nv, uint32_t& lo, uint32_t& hi) {
+      lo = (2 * c < nv ? 0x0000FFFFu : 0u) | (2 * c + 1 < nv ? 0xFFFF0000u : 0u);
+      hi = (2 * c + 8 < nv ? 0x0000FFFFu : 0u) | (2 * c + 9 < nv ? 0xFFFF0000u : 0u);
+    };
+    uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
+    if (tail0) pmask(nv0, mlo, mhi);
+    pv_tile(vc0, vs0, pb0, tail0, mlo, mhi);
+    if (two) {
+      if (tail1) pmask(nv1, mlo, mhi);
+      pv_tile(vc0 + kHalf * L::RBV, vs0 + kHalf * L::NSV, pb1, tail1, mlo, mhi);
+    }
+
+    // release the stage and refill it with this warp's tile j + S
+    __syncwarp();
+    if (lane == 0 && j + S < my_tiles) {
+      fence_proxy_async();
+      issue(j + S);
+    }
+  }
+
+  if (failed_at >= 0) {
+    // A copy did not land within the limit.  Wait (bounded again) for every
+    // copy this warp still has in flight -- tiles failed_at .. failed_at+S-1 --
+    // so none writes into shared memory after the CTA exits, and make this
+    // CTA's partials NaN so the outputs show the failure.
+    const int last = min(my_tiles, failed_at + S);
+    for (int jj = failed_at; jj < last; ++jj) (void)mbar_wait(&bars[jj % S], (uint32_t)((jj / S) & 1));
+    if (lane == 0) atomicExch(&cta_failed, 1);
+  }
+  __syncwarp();
+
+  // ---- reduce l over the 8 row groups; each lane keeps heads 2c, 2c+1
+#pragma unroll
+  for (int nt = 0; nt < NTH; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+      for (int o = 4; o <= 16; o <<= 1) l_run[nt][e] += __shfl_xor_sync(0xffffffffu, l_run[nt][e], o);
+
+  __syncthreads();  // every warp is done with its stages: reuse them for the merge
+
+  // merge area: per warp [8 heads][D] acc, then m[8], l[8]
+  float* mrg = reinterpret_cast<float*>(smem);
+  auto dim_of = [&](int mt, int row) -> int {  // PV m-tile row -> head dim
+    if (VT == KVQ_F16) return 16 * mt + row;                       // row in 0..15
+    if (VT == KVQ_TURBO3) return (row & 7) * (D / 8) + 2 * mt + (row >> 3);
+    return 32 * (mt >> 1) + 16 * (mt & 1) + 2 * (row & 7) + (row >> 3);  // q8_0, q4_0
+  };
+#pragma unroll
+  for (int nt = 0; nt < NTH; ++nt) {
+    float* wacc = mrg + warp * (8 * D + 16);
+    float* wm = wacc + 8 * D;
+    float* wl = wm + 8;
+#pragma unroll
+    for (int mt = 0; mt < NMT; ++mt) {
+      wacc[(2 * c) * D + dim_of(mt, g)] = acc[nt][mt][0];
+      wacc[(2 * c + 1) * D + dim_of(mt, g)] = acc[nt][mt][1];
+      wacc[(2 * c) * D + dim_of(mt, g + 8)] = acc[nt][mt][2];
+      wacc[(2 * c + 1) * D + dim_of(mt, g + 8)] = acc[nt][mt][3];
+    }
+    if (g == 0) {
+      wm[2 * c] = m_run[nt][0];
+      wm[2 * c + 1] = m_run[nt][1];
+      wl[2 * c] = l_run[nt][0];
+      wl[2 * c + 1] = l_run[nt][1];
+    }
+    __syncthreads();
+    const int heads_here = min(8, p.G - nt * 8);
+    for (int i = threadIdx.x; i < heads_here * D; i += L::NW * 32) {
+      const int h = i / D, dd = i % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < L::NW; ++w) M = fmaxf(M, mrg[w * (8 * D + 16) + 8 * D + h]);
+      float a = 0.f, l = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < L::NW; ++w) {
+          const float* base = mrg + w * (8 * D + 16);
+          const float mw = base[8 * D + h];
+          if (mw == -INFINITY) continue;
+          const float f = exp2f(mw - M);
+          a = fmaf(f, base[h * D + dd], a);
+          l = fmaf(f, base[8 * D + 8 + h], l);
+        }
+      }
+      if (cta_failed) a = l = M = __int_as_float(0x7fc00000);  // NaN
+      const int64_t row = ((int64_t)b * p.n_q + (int64_t)kvh * p.G + nt * 8 + h) * p.S + s_idx;
+      p.ws_acc[row * D + dd] = a;
+      if (dd == 0) {
+        p.ws_m[row] = M;
+        p.ws_l[row] = l;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+struct TcMaps {
+  CUtensorMap kc, ks, vc, vs;
+};
+
+template <int KT, int VT, int NB, int NTH>
+cudaError_t launch_one(const TcArgs& a, const TcMaps& m, cudaStream_t st) {
+  using L = Layout<KT, VT, NB * 32>;
+  auto kern = decode_tc_kernel<KT, VT, NB, NTH>;
+  static bool attr_set = false;  // idempotent; a race only repeats the call
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const dim3 grid(a.p.S, a.p.n_kv, a.p.B);
+  kern<<<grid, L::NW * 32, L::TOTAL, st>>>(a, m.kc, m.ks, m.vc, m.vs);
+  return cudaGetLastError();
+}
+
+template <int KT, int VT, int NB>
+cudaError_t launch_nb(int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st) {
+  return nth == 1 ? launch_one<KT, VT, NB, 1>(a, m, st) : launch_one<KT, VT, NB, 2>(a, m, st);
+}
+
+template <int KT, int VT>
+cudaError_t launch_v(int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st) {
+  switch (nb) {
+    case 2: return launch_nb<KT, VT, 2>(nth, a, m, st);
+    case 4: return launch_nb<KT, VT, 4>(nth, a, m, st);
+    case 8:
+      if constexpr (KT == KVQ_F16 && VT == KVQ_F16) return cudaErrorInvalidValue;
+      else return launch_nb<KT, VT, 8>(nth, a, m, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int KT>
+cudaError_t launch_k(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st) {
+  switch (vt) {
+    case KVQ_F16: return launch_v<KT, KVQ_F16>(nb, nth, a, m, st);
+    case KVQ_Q8_0: return launch_v<KT, KVQ_Q8_0>(nb, nth, a, m, st);
+    case KVQ_Q4_0: return launch_v<KT, KVQ_Q4_0>(nb, nth, a, m, st);
+    case KVQ_TURBO3: return launch_v<KT, KVQ_TURBO3>(nb, nth, a, m, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// one per key type, each in its own translation unit
+cudaError_t launch_kf16(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kq8(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kq4(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+
+}  // namespace tc
+}  // namespace kvq

@@ -314,10 +314,12 @@ kvq_status kvq_append_quantize(const kvq_cache_desc* d, void* k_cache, void* v_c
   const int64_t rows = (int64_t)batch * n_tok * d->n_kv_heads;
   if (rows * (d->head_dim / 4) > ((int64_t)1 << 40)) return KVQ_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  AppendParams ap[2];
   for (int which = 0; which < 2; ++which) {
     void* cache = which ? v_cache : k_cache;
     if (!cache) continue;
-    AppendParams p{};
+    AppendParams& p = ap[which];
+    p = AppendParams{};
     p.src = static_cast<const __half*>(which ? v_new : k_new);
     p.dst = plane_of(d, batch, which, cache);
     p.B = batch;
@@ -325,11 +327,10 @@ kvq_status kvq_append_quantize(const kvq_cache_desc* d, void* k_cache, void* v_c
     p.D = d->head_dim;
     p.n_tok = n_tok;
     p.pos = pos;
-    const int32_t type = which ? d->v_type : d->k_type;
-    if (type == KVQ_TURBO3) p.t3 = turbo3_consts(d);
-    const cudaError_t e = launch_append(type, p, s);
-    if (e != cudaSuccess) return cuda_fail(e);
+    if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) p.t3 = turbo3_consts(d);
   }
+  const cudaError_t e = launch_append(do_k ? &ap[0] : nullptr, d->k_type, do_v ? &ap[1] : nullptr, d->v_type, s);
+  if (e != cudaSuccess) return cuda_fail(e);
   return KVQ_OK;
 }
 

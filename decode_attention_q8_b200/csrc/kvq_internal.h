@@ -67,7 +67,9 @@ int32_t n_scales_of(int32_t type, int32_t d);
 void set_last_cuda_error(cudaError_t e);  // text returned by kvq_last_cuda_error()
 
 // Launchers; each returns cudaGetLastError() after its launch.
-cudaError_t launch_append(int32_t type, const AppendParams& p, cudaStream_t st);
+// Quantize-on-append of K and/or V rows (either may be null) in one launch.
+cudaError_t launch_append(const AppendParams* k, int32_t k_type, const AppendParams* v, int32_t v_type,
+                          cudaStream_t st);
 cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p, cudaStream_t st);
 bool decode_supported(int32_t k_type, int32_t v_type, int32_t G, int32_t D);
 int decode_ctas_per_sm();  // resident decode CTAs per SM the split heuristic plans for
