@@ -60,48 +60,118 @@ def algorithmic_bytes(w, n_layers):
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event (throttle) reasons of one GPU, sampled every few
+    ms by a thread through NVML (read-only queries), keeping the samples taken
+    between begin() and end(), i.e. during the timed region.  Falls back to an
+    `nvidia-smi -lms` process when the NVML binding is missing."""
 
-    def __init__(self, device_index, enabled=True):
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, device_index, enabled=True, period_s=0.004, query=None):
+        import threading
+        self.samples = []            # (host time, sm MHz, set of reason names)
+        self.window = [None, None]
+        self.max_mhz = None
         self.proc = None
-        self.idx = device_index
-        if enabled:
+        self._stop = threading.Event()
+        self._thread = None
+        if not enabled:
+            return
+        if query is None:
+            query = self._nvml_query(device_index)
+        if query is None:
+            self._start_smi(device_index)
+            return
+        self._query = query
+        self._period = period_s
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+
+    def _nvml_query(self, device_index):
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
             try:
-                self.proc = subprocess.Popen(
-                    ["nvidia-smi", f"--id={device_index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                     "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            except OSError:
-                self.proc = None
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            masks = [(name, getattr(pynvml, sym)) for name, sym in self.REASONS if hasattr(pynvml, sym)]
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def query():
+                sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                bits = get_reasons(h)
+                return sm, {name for name, m in masks if bits & m}
+            query()
+            return query
+        except Exception:
+            return None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                sm, reasons = self._query()
+            except Exception:
+                break
+            self.samples.append((time.perf_counter(), sm, reasons))
+            self._stop.wait(self._period)
+
+    def _start_smi(self, device_index):
+        q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={device_index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def begin(self):
+        self.window[0] = time.perf_counter()
+
+    def end(self):
+        self.window[1] = time.perf_counter()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, smax, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
+        """Summary of the samples inside the window: median SM MHz, max MHz and
+        every reason seen active, or None without samples."""
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+        if self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(f[1]))
-                smax = max(smax, float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for line in out.strip().splitlines():
+                f = [x.strip() for x in line.split(",")]
+                try:
+                    sm, mx = float(f[0]), float(f[1])
+                except (ValueError, IndexError):
+                    continue
+                self.max_mhz = max(self.max_mhz or 0.0, mx)
+                self.samples.append((None, sm, {n for n, v in zip(names, f[2:6]) if v.lower() == "active"}))
+        t0, t1 = self.window
+        inside = [s for s in self.samples
+                  if s[0] is None or ((t0 is None or s[0] >= t0) and (t1 is None or s[0] <= t1))]
+        if not inside:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for s in inside:
+            reasons |= s[2]
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(inside)}
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -161,9 +231,8 @@ def oracle_sample(w, seconds=10.0, max_units=None):
 
 def run_reference(args):
     import synth
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
-        return
+    if rank_env()[1] != 0:
+        return   # the oracle baseline runs on rank 0 only
     w = synth.WORKLOADS[args.workload]
     gbs, units, secs, cores = oracle_sample(w, seconds=max(3.0, 2.0 * (args.steps + args.warmup)))
     line = {
@@ -186,6 +255,31 @@ def _config(w, args, n_layers):
             "l2": "inputs larger than L2: every layer a distinct cache buffer larger than the 126 MB L2"}
 
 
+# ----------------------------------------------------------------- ranks
+
+def rank_env():
+    """(world size, rank, local rank) from the launcher's environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise maximum over all ranks of this rank's timings; every rank
+    takes part and gets the result."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_gbs(world, bytes_per_rank_step, steps, ms):
+    """Weak scaling: each rank runs its own replica of the workload, so the job
+    moves world x the per-rank bytes in the slowest rank's time (ms)."""
+    return world * bytes_per_rank_step * steps / (ms * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------- GPU arm
 
 def run_kvq(args):
@@ -195,9 +289,7 @@ def run_kvq(args):
     import decode_attention_q8_b200 as kvq
     import synth
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -271,11 +363,13 @@ def run_kvq(args):
     clocks = ClockSampler(local, enabled=not args.no_clocks)
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
+    clocks.begin()
     t_start.record()
     for _ in range(args.steps):
         graph.replay()
     t_end.record()
     barrier()
+    clocks.end()
     clk = clocks.stop()
     ms = t_start.elapsed_time(t_end)
     if dec_ev is not None:
@@ -333,14 +427,11 @@ def run_kvq(args):
     del e2e_graph
 
     # ---- max over ranks
-    vals = torch.tensor([ms, e2e_ms, statistics.mean(dec_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms, e2e_ms, dec_avg = vals.tolist()
+    ms, e2e_ms, dec_avg = max_over_ranks([ms, e2e_ms, statistics.mean(dec_ms)], world, dev)
 
     dec_bytes, app_bytes, step_bytes = algorithmic_bytes(w, L)
-    value = world * step_bytes * args.steps / (ms * 1e-3) / 1e9
-    e2e_value = world * step_bytes * args.steps / (e2e_ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_bytes, args.steps, ms)
+    e2e_value = whole_job_gbs(world, step_bytes, args.steps, e2e_ms)
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))

@@ -204,16 +204,16 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t r[4], const void* p) {
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t r[4], uint32_t saddr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_addr(p)));
+               : "r"(saddr));
 }
 
-__device__ __forceinline__ void ldmatrix_x4(uint32_t r[4], const void* p) {
+__device__ __forceinline__ void ldmatrix_x4(uint32_t r[4], uint32_t saddr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_addr(p)));
+               : "r"(saddr));
 }
 
 // 2^x by the SFU's ex2 (about 2 ulp; subnormal results flush to 0, which only
@@ -224,11 +224,8 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
+// byte permute (PRMT) through the intrinsic, so constant operands stay immediates
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) { return __byte_perm(a, b, sel); }
 
 __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
   return (a & mask) | orv;  // one LOP3
@@ -284,11 +281,13 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   const DecodeParams& p = args.p;
 
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                         ~uintptr_t(1023));
+  // 1024-byte alignment (the swizzle atom) by offsetting inside the shared
+  // array, so every derived pointer stays in the shared address space
+  unsigned char* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   unsigned char* wbase = smem + warp * L::WARP;
+  const uint32_t wbase32 = smem_addr(wbase);
   __shared__ int cta_failed;
   uint32_t* table = reinterpret_cast<uint32_t*>(smem + L::NW * L::WARP);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::NW * L::WARP + L::TABLE) + warp * S;
@@ -425,10 +424,20 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   // matrix lane >> 3; lm_hi selects the second segment / block of an x4 load
   const int lm_row = (lane & 7) + 8 * ((lane >> 3) & 1);
   const int lm_hi = lane >> 4;
+  // this lane's swizzled ldmatrix offsets inside a 16-row half (the swizzle
+  // period divides 16 rows, so both halves of a tile use the same offsets)
+  uint32_t koff[NB], voff[NB];
+#pragma unroll
+  for (int blk = 0; blk < NB; ++blk) {
+    koff[blk] = KT == KVQ_Q8_0 ? swz<KMASK>(lm_row * L::RBK + 16 * (2 * blk + lm_hi))
+                               : swz<KMASK>(lm_row * L::RBK + 16 * ((blk & ~1) + lm_hi));
+    voff[blk] = VT == KVQ_Q8_0 ? swz<VMASK>(lm_row * L::RBV + 16 * (2 * blk + lm_hi))
+                               : swz<VMASK>(lm_row * L::RBV + 16 * ((blk & ~1) + lm_hi));
+  }
   int failed_at = -1;  // tile whose wait timed out (warp-uniform), -1 if none
 
   // QK of one 16-row tile: scaled scores S[row][head] of rows g, g+8 (heads 2c, 2c+1)
-  auto qk_tile = [&](const unsigned char* kc, const __half* ksc, float (&sc)[NTH][4]) {
+  auto qk_tile = [&](uint32_t kc, const __half* ksc, float (&sc)[NTH][4]) {
     // ---------------- QK: S[row][head] for rows g, g+8
 #pragma unroll
     for (int nt = 0; nt < NTH; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
@@ -465,7 +474,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       uint32_t a[2][4];  // [k-step][a0..a3]
       if constexpr (KT == KVQ_Q8_0) {
         uint32_t r[4];
-        ldmatrix_x4(r, kc + swz<KMASK>(lm_row * L::RBK + 16 * (2 * blk + lm_hi)));
+        ldmatrix_x4(r, kc + koff[blk]);
         const uint32_t u0 = r[0] ^ 0x80808080u, u1 = r[1] ^ 0x80808080u;
         const uint32_t u2 = r[2] ^ 0x80808080u, u3 = r[3] ^ 0x80808080u;
         a[0][0] = prmt(u0, 0x64646464u, 0x4140);
@@ -479,7 +488,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       } else if constexpr (KT == KVQ_Q4_0) {
         // one x4 load covers blocks blk (regs 0, 1) and blk + 1 (regs 2, 3):
         // reg = bytes 4c..4c+3 of the block in row g (even regs) or g+8 (odd)
-        if ((blk & 1) == 0) ldmatrix_x4(kr, kc + swz<KMASK>(lm_row * L::RBK + 16 * (blk + lm_hi)));
+        if ((blk & 1) == 0) ldmatrix_x4(kr, kc + koff[blk]);
         const uint32_t wa = kr[(blk & 1) * 2], wb = kr[(blk & 1) * 2 + 1];
         a[0][0] = lop_and_or(wa, 0x000F000Fu, kMagic);        // dims (4c, 4c+2)
         a[0][2] = lop_and_or(wa >> 8, 0x000F000Fu, kMagic);   // dims (4c+1, 4c+3)
@@ -493,7 +502,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 #pragma unroll
         for (int s2 = 0; s2 < 2; ++s2) {
           uint32_t r[4];
-          ldmatrix_x4(r, kc + swz<KMASK>(lm_row * L::RBK + 64 * blk + 32 * s2 + 16 * lm_hi));
+          ldmatrix_x4(r, kc + (uint32_t)swz<KMASK>(lm_row * L::RBK + 64 * blk + 32 * s2 + 16 * lm_hi));
           a[s2][0] = r[0];
           a[s2][1] = r[1];
           a[s2][2] = r[2];
@@ -502,18 +511,22 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       }
 #pragma unroll
       for (int nt = 0; nt < NTH; ++nt) {
-        float dblk[4];
-        const float cin[4] = {corr[nt][blk][0], corr[nt][blk][1], corr[nt][blk][0], corr[nt][blk][1]};
-        mma16816(dblk, a[0][0], a[0][1], a[0][2], a[0][3], qb[nt][blk][0][0], qb[nt][blk][0][1], cin);
-        mma16816(dblk, a[1][0], a[1][1], a[1][2], a[1][3], qb[nt][blk][1][0], qb[nt][blk][1][1], dblk);
-        if (L::NSK) {
-          sc[nt][0] = fmaf(dA[blk], dblk[0], sc[nt][0]);
-          sc[nt][1] = fmaf(dA[blk], dblk[1], sc[nt][1]);
-          sc[nt][2] = fmaf(dB[blk], dblk[2], sc[nt][2]);
-          sc[nt][3] = fmaf(dB[blk], dblk[3], sc[nt][3]);
+        if constexpr (L::NSK > 0) {
+          // per-block dot products from a zero accumulator; the offset
+          // correction and the block scale are applied in fp32
+          float dblk[4];
+          const float z4[4] = {0.f, 0.f, 0.f, 0.f};
+          mma16816(dblk, a[0][0], a[0][1], a[0][2], a[0][3], qb[nt][blk][0][0], qb[nt][blk][0][1], z4);
+          mma16816(dblk, a[1][0], a[1][1], a[1][2], a[1][3], qb[nt][blk][1][0], qb[nt][blk][1][1], dblk);
+          const float c0 = corr[nt][blk][0], c1 = corr[nt][blk][1];
+          sc[nt][0] = fmaf(dA[blk], dblk[0] + c0, sc[nt][0]);
+          sc[nt][1] = fmaf(dA[blk], dblk[1] + c1, sc[nt][1]);
+          sc[nt][2] = fmaf(dB[blk], dblk[2] + c0, sc[nt][2]);
+          sc[nt][3] = fmaf(dB[blk], dblk[3] + c1, sc[nt][3]);
         } else {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) sc[nt][i] += dblk[i];
+          // f16 keys: no scale, no correction; accumulate in place
+          mma16816(sc[nt], a[0][0], a[0][1], a[0][2], a[0][3], qb[nt][blk][0][0], qb[nt][blk][0][1], sc[nt]);
+          mma16816(sc[nt], a[1][0], a[1][1], a[1][2], a[1][3], qb[nt][blk][1][0], qb[nt][blk][1][1], sc[nt]);
         }
       }
     }
@@ -524,7 +537,8 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   };
 
   // PV of one 16-row tile with its P fragments (rows 2c, 2c+1 | 2c+8, 2c+9)
-  auto pv_tile = [&](const unsigned char* vc, const __half* vsc, const uint32_t (&pb)[NTH][2], bool tail,
+  auto pv_tile = [&](const unsigned char* vc, uint32_t vc32, const __half* vsc, const uint32_t (&pb)[NTH][2],
+                     bool tail,
                      uint32_t pmask_lo, uint32_t pmask_hi) {
     // ---------------- PV
     if constexpr (VT == KVQ_F16) {
@@ -533,7 +547,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         const int jm = lane >> 3;
         const int krow = (lane & 7) + 8 * (jm >> 1);
         uint32_t a[4];
-        ldmatrix_x4_trans(a, vc + swz<VMASK>(krow * L::RBV + 2 * (16 * mt + 8 * (jm & 1))));
+        ldmatrix_x4_trans(a, vc32 + (uint32_t)swz<VMASK>(krow * L::RBV + 2 * (16 * mt + 8 * (jm & 1))));
 #pragma unroll
         for (int nt = 0; nt < NTH; ++nt) {
           uint32_t b0 = pb[nt][0], b1 = pb[nt][1];
@@ -653,7 +667,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         if (VT == KVQ_Q4_0) {
           // trans load: reg = [row 2c: bytes 2g, 2g+1 | row 2c+1: bytes 2g, 2g+1]
           // of the block -> dims 2g, 2g+1 (low nibbles), 2g+16, 2g+17 (high)
-          if ((blk & 1) == 0) ldmatrix_x4_trans(vr, vc + swz<VMASK>(lm_row * L::RBV + 16 * (blk + lm_hi)));
+          if ((blk & 1) == 0) ldmatrix_x4_trans(vr, vc32 + voff[blk]);
           const uint32_t w1 = vr[(blk & 1) * 2], w2 = vr[(blk & 1) * 2 + 1];
           const uint32_t w1s = w1 >> 8, w2s = w2 >> 8;
           a0[0] = hsub2_u32(lop_and_or(w1, 0x000F000Fu, kMagic), kBias1032);   // dim 2g, rows 2c,2c+1
@@ -670,7 +684,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         } else {
           // q8_0 trans load of segments 2blk (regs 0, 1) and 2blk+1 (regs 2, 3):
           // reg = [row 2c: bytes 2g, 2g+1 | row 2c+1: bytes 2g, 2g+1]
-          ldmatrix_x4_trans(vr, vc + swz<VMASK>(lm_row * L::RBV + 16 * (2 * blk + lm_hi)));
+          ldmatrix_x4_trans(vr, vc32 + voff[blk]);
           const uint32_t x0 = vr[0] ^ 0x80808080u, x1 = vr[1] ^ 0x80808080u;
           const uint32_t y0 = vr[2] ^ 0x80808080u, y1 = vr[3] ^ 0x80808080u;
           a0[0] = hsub2_u32(prmt(x0, 0x64646464u, 0x4240), kBias1152);  // dim 2g
@@ -709,7 +723,8 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     const int nv1 = rem1 <= 0 ? 0 : (int)(rem1 < kHalf ? rem1 : kHalf);
     const bool two = nv1 > 0;
     const bool tail0 = nv0 < kHalf, tail1 = two && nv1 < kHalf;
-    const unsigned char* kc0 = kc_of(st);
+    const uint32_t kc0 = wbase32 + st * L::KC;
+    const uint32_t vc32 = wbase32 + S * L::KC + st * L::VC;
     const __half* ks0 = reinterpret_cast<const __half*>(ks_of(st));
     const unsigned char* vc0 = vc_of(st);
     const __half* vs0 = reinterpret_cast<const __half*>(vs_of(st));
@@ -775,10 +790,10 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     };
     uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
     if (tail0) pmask(nv0, mlo, mhi);
-    pv_tile(vc0, vs0, pb0, tail0, mlo, mhi);
+    pv_tile(vc0, vc32, vs0, pb0, tail0, mlo, mhi);
     if (two) {
       if (tail1) pmask(nv1, mlo, mhi);
-      pv_tile(vc0 + kHalf * L::RBV, vs0 + kHalf * L::NSV, pb1, tail1, mlo, mhi);
+      pv_tile(vc0 + kHalf * L::RBV, vc32 + kHalf * L::RBV, vs0 + kHalf * L::NSV, pb1, tail1, mlo, mhi);
     }
 
     // release the stage and refill it with this warp's tile j + S
