@@ -33,20 +33,26 @@
 //        matrix; the swizzle puts the 8 rows in distinct bank groups), B = Q^T
 //        (8 heads), fp32 C.  What ldmatrix hands a lane (4 bytes of a 16-byte
 //        segment) fixes the dim order inside each 32-dim block; Q is loaded in
-//        the same order.  int8 codes enter as fp16 1024 + (k + 128) (an xor and
-//        two byte permutes per four codes), q4_0 nibbles as 1024 + n (one LOP3
-//        per two); the MMA's C input carries -1152 * sum_block(q) (-1032 for
-//        q4_0), so D = sum k*q per block exactly; block scale and
-//        softmax_scale * log2 e are applied in fp32.
+//        the same order.  Integer codes enter the MMA as fp16 subnormals, which
+//        are exact: q8_0 k as (k + 128) * 2^-24 (an xor and two byte permutes
+//        per four codes), q4_0 n as n * 2^-24 (one AND per two).  The first
+//        MMA of a block starts from C = -128 * sum_block(q) * 2^-24 (-8 for
+//        q4_0), so the block result is 2^-24 * sum k*q exactly up to fp32
+//        rounding; the row's block scale is applied in fp32 and the 2^24 is
+//        folded into softmax_scale * log2 e.
 //   P    ex2 of the scores in fp32, rounded to fp16; movmatrix.trans turns the
 //        (row x head) accumulator layout into the (row x head) B operand of PV.
 //   PV   O^T[dim][head] += V^T[dim][row] * P[row][head]: A = V^T (16 dims) by
 //        ldmatrix.trans, which hands a lane the same two bytes of rows 2c and
 //        2c+1 in one register -- exactly the pair an A fragment holds -- so the
-//        codes only need masking into fp16 (q4_0: 1024 + n, minus 1032) or an
-//        xor and a permute (q8_0).  Each row's block scale (turbo3: its norm)
-//        multiplies P in fp16; the codes stay exact small integers (turbo3: the
-//        codebook level, from a per-lane replicated 64-entry pair table).
+//        codes only need masking into subnormals (q4_0: n * 2^-24 and, for the
+//        high nibble, 16 n * 2^-24) or an xor and a permute (q8_0: (k + 128) *
+//        2^-24).  Each row's block scale (turbo3: its norm) multiplies P in
+//        fp16.  The code offset (8 or 128) times sum_t d[t][blk] p[t] comes from
+//        one more MMA per 16 rows whose A operand is the block-scale matrix
+//        (m = block, k = row); it and the 2^24 are taken out once at the end.
+//        turbo3 codes become codebook levels through a per-lane replicated
+//        64-entry pair table.
 //   turbo3 values accumulate in the rotated domain; kvq_combine rotates back.
 #pragma once
 
@@ -227,21 +233,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // byte permute (PRMT) through the intrinsic, so constant operands stay immediates
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) { return __byte_perm(a, b, sel); }
 
-__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
-  return (a & mask) | orv;  // one LOP3
-}
-
-__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
-  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
-}
-
-__device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
-  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b),
-                      *reinterpret_cast<__half2*>(&c));
-  return *reinterpret_cast<uint32_t*>(&r);
-}
-
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
@@ -257,9 +248,23 @@ __device__ __forceinline__ int swz(int off) {
   return off ^ (((off >> 7) & MASK) << 4);
 }
 
-constexpr uint32_t kMagic = 0x64006400u;   // fp16 1024 in both halves
-constexpr uint32_t kBias1032 = 0x64086408u;  // fp16 1032 (1024 + 8)
-constexpr uint32_t kBias1152 = 0x64806480u;  // fp16 1152 (1024 + 128)
+// Integer codes enter the MMA as fp16 subnormals: a code n in 0..1023 in the
+// low bits of an fp16 word is exactly n * 2^-24, the MMA multiplies such values
+// exactly and accumulates in fp32, and the factor 2^24 is taken out in fp32.
+constexpr float kTwo24 = 16777216.f;
+constexpr float kTwo20 = 1048576.f;
+constexpr float kTwoM24 = 5.9604644775390625e-08f;
+constexpr uint32_t kHalfSixteenth = 0x2C002C00u;  // fp16 1/16 in both halves
+
+// XOR that moves a lane's swizzled ldmatrix offset from block 0 to block blk.
+// The swizzle only permutes 16-byte chunks inside a 128-byte span, so within a
+// code row the offset of block blk is the block-0 offset with the chunk bits of
+// blk flipped; for 256-byte rows the second 128-byte span also flips chunk bit
+// 0 (its swizzle row index is odd).
+__host__ __device__ constexpr uint32_t blk_xor(int t, int rb, int blk) {
+  return t == KVQ_Q8_0 ? (uint32_t)(32 * blk) ^ (rb > 128 && blk >= 4 ? 16u : 0u)
+                       : (uint32_t)(16 * (blk & ~1));
+}
 
 // ------------------------------------------------------------------ kernel
 
@@ -278,6 +283,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   constexpr int S = L::kStages;
   constexpr int KMASK = swz_mask(KT, D), VMASK = swz_mask(VT, D);
   constexpr int NMT = D / 16;  // PV m-tiles
+  constexpr bool kVQ = VT == KVQ_Q8_0 || VT == KVQ_Q4_0;  // block-scaled integer values
   const DecodeParams& p = args.p;
 
   extern __shared__ unsigned char smem_raw[];
@@ -293,9 +299,11 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::NW * L::WARP + L::TABLE) + warp * S;
 
   const int s_idx = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int64_t t0 = (int64_t)s_idx * p.chunk;
-  const int64_t t1 = min(p.ctx, t0 + p.chunk);
-  const int n_sub = t0 < t1 ? (int)((t1 - t0 + kSub - 1) / kSub) : 0;
+  const int64_t t0l = (int64_t)s_idx * p.chunk;
+  const int64_t t1l = min(p.ctx, t0l + p.chunk);
+  const int n_sub = t0l < t1l ? (int)((t1l - t0l + kSub - 1) / kSub) : 0;
+  // row indices fit in 32 bits (the tensor-map coordinates are 32-bit)
+  const int t0 = (int)t0l, t1 = (int)t1l;
   const int plane = b * p.n_kv + kvh;
 
   if (threadIdx.x == 0) cta_failed = 0;
@@ -320,9 +328,8 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 
   // tile j of this warp covers rows t0 + 32*(warp + NW*j) ...
   const int my_tiles = n_sub > warp ? (n_sub - warp + L::NW - 1) / L::NW : 0;
-  auto issue = [&](int j) {
-    const int st = j % S;
-    const int r0 = (int)(t0 + (int64_t)kSub * (warp + L::NW * j));
+  auto issue = [&](int j, int st) {
+    const int r0 = t0 + kSub * (warp + L::NW * j);
     mbar_expect_tx(&bars[st], L::TX);
     if (L::RBK > 128)
       tma_load_4d(kc_of(st), &tm_kc, 0, 0, r0, plane, &bars[st]);
@@ -342,21 +349,26 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     if (L::NSV) tma_load_2d(vs_of(st), &tm_vs, r0 * L::NSV / 2, plane, &bars[st]);
   };
   if (lane == 0) {
-    for (int j = 0; j < S && j < my_tiles; ++j) issue(j);
+    for (int j = 0; j < S && j < my_tiles; ++j) issue(j, j);
   }
 
-  // ---- queries: B fragments of Q^T per (block, k-step) and the per-block
-  //      correction -bias * sum(q) for heads 2c, 2c+1 of each n-tile.  The dim
-  //      order inside a block follows the A-operand loads below (lane = 4g + c):
+  // ---- queries: B fragments of Q^T per (block, k-step) and, for quantized
+  //      keys, the MMA C input -bias * sum(q) * 2^-24 of heads 2c, 2c+1 of each
+  //      n-tile.  The dim order inside a block follows the A-operand loads
+  //      below (lane = 4g + c):
   //        q8_0  k-step s = 16-byte segment 2*blk+s; lane c holds bytes 4c..4c+3:
   //              cols 2c,2c+1 <- bytes 4c,4c+1 and cols 2c+8,2c+9 <- 4c+2,4c+3
   //        q4_0  lane c holds bytes 4c..4c+3 of the block; low nibbles (dims
   //              4c..4c+3) feed k-step 0, high nibbles (4c+16..4c+19) k-step 1;
-  //              cols 2c,2c+1 <- dims (4c, 4c+2), cols 2c+8,2c+9 <- (4c+1, 4c+3)
+  //              cols 2c,2c+1 <- dims (4c, 4c+2), cols 2c+8,2c+9 <- (4c+1, 4c+3).
+  //              The high nibbles enter as 16 n * 2^-24, so k-step 1 takes q / 16.
   //        f16   natural: k-step s covers dims 32*blk + 16*s .. +15
+  //      Key codes enter as (k + 128) * 2^-24 (q8_0, sign bit flipped) or
+  //      n * 2^-24 (q4_0), so the block dot product needs -128 * sum(q) or
+  //      -8 * sum(q), in the same 2^-24 units.
   uint32_t qb[NTH][NB][2][2];
-  float corr[NTH][NB][2];
-  const float bias = KT == KVQ_Q8_0 ? 1152.f : KT == KVQ_Q4_0 ? 1032.f : 0.f;
+  float cq[NTH][NB][4];
+  constexpr float kBiasK = KT == KVQ_Q8_0 ? 128.f : KT == KVQ_Q4_0 ? 8.f : 0.f;
 #pragma unroll
   for (int nt = 0; nt < NTH; ++nt) {
     const int head = nt * 8 + g;
@@ -387,10 +399,6 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           w3 = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 24 + 2 * c);
         }
       }
-      qb[nt][blk][0][0] = w0;
-      qb[nt][blk][0][1] = w1;
-      qb[nt][blk][1][0] = w2;
-      qb[nt][blk][1][1] = w3;
       // partial sum of this lane's 8 dims of head g, then over the 4 lanes of the group
       float part = 0.f;
       const uint32_t ws[4] = {w0, w1, w2, w3};
@@ -404,41 +412,51 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       // lane (g', c') needs the sums of heads 2c', 2c'+1 (held by groups 2c', 2c'+1)
       const float s0 = __shfl_sync(0xffffffffu, part, (2 * c) * 4);
       const float s1 = __shfl_sync(0xffffffffu, part, (2 * c + 1) * 4);
-      corr[nt][blk][0] = -bias * s0;
-      corr[nt][blk][1] = -bias * s1;
+      if (KT == KVQ_Q4_0) {
+        w2 = hmul2_u32(w2, kHalfSixteenth);
+        w3 = hmul2_u32(w3, kHalfSixteenth);
+      }
+      qb[nt][blk][0][0] = w0;
+      qb[nt][blk][0][1] = w1;
+      qb[nt][blk][1][0] = w2;
+      qb[nt][blk][1][1] = w3;
+      const float c0 = -kBiasK * kTwoM24 * s0, c1 = -kBiasK * kTwoM24 * s1;
+      cq[nt][blk][0] = c0;
+      cq[nt][blk][1] = c1;
+      cq[nt][blk][2] = c0;
+      cq[nt][blk][3] = c1;
     }
   }
+  const float qs = KT == KVQ_F16 ? p.qscale : p.qscale * kTwo24;
 
   // ---- running state
   float m_run[NTH][2], l_run[NTH][2];
   float acc[NTH][NMT][4];
+  float off[NTH][4];  // q8_0 / q4_0 values: sum_t d[t][blk] p[t][head], blk = g, heads 2c, 2c+1
 #pragma unroll
   for (int nt = 0; nt < NTH; ++nt) {
     m_run[nt][0] = m_run[nt][1] = -INFINITY;
     l_run[nt][0] = l_run[nt][1] = 0.f;
+    off[nt][0] = off[nt][1] = off[nt][2] = off[nt][3] = 0.f;
 #pragma unroll
     for (int i = 0; i < NMT; ++i) acc[nt][i][0] = acc[nt][i][1] = acc[nt][i][2] = acc[nt][i][3] = 0.f;
   }
 
   // ldmatrix addressing: this lane supplies the address of tile row lm_row in
-  // matrix lane >> 3; lm_hi selects the second segment / block of an x4 load
+  // matrix lane >> 3; lm_hi selects the second segment / block of an x4 load.
+  // koff0 / voff0: the lane's swizzled offset of block 0 inside a 16-row half
+  // (the swizzle period divides 16 rows, so both halves use the same offsets).
   const int lm_row = (lane & 7) + 8 * ((lane >> 3) & 1);
   const int lm_hi = lane >> 4;
-  // this lane's swizzled ldmatrix offsets inside a 16-row half (the swizzle
-  // period divides 16 rows, so both halves of a tile use the same offsets)
-  uint32_t koff[NB], voff[NB];
-#pragma unroll
-  for (int blk = 0; blk < NB; ++blk) {
-    koff[blk] = KT == KVQ_Q8_0 ? swz<KMASK>(lm_row * L::RBK + 16 * (2 * blk + lm_hi))
-                               : swz<KMASK>(lm_row * L::RBK + 16 * ((blk & ~1) + lm_hi));
-    voff[blk] = VT == KVQ_Q8_0 ? swz<VMASK>(lm_row * L::RBV + 16 * (2 * blk + lm_hi))
-                               : swz<VMASK>(lm_row * L::RBV + 16 * ((blk & ~1) + lm_hi));
-  }
+  const uint32_t koff0 = (uint32_t)swz<KMASK>(lm_row * L::RBK + 16 * lm_hi);
+  const uint32_t voff0 = (uint32_t)swz<VMASK>(lm_row * L::RBV + 16 * lm_hi);
+  // offset-MMA operand selection: block g of a scale row (lanes g >= NSV give 0)
+  const uint32_t osel = (g & 1) ? 0x7632u : 0x5410u;
+  const uint32_t omask = g < (L::NSV > 0 ? L::NSV : 1) ? 0xFFFFFFFFu : 0u;
   int failed_at = -1;  // tile whose wait timed out (warp-uniform), -1 if none
 
   // QK of one 16-row tile: scaled scores S[row][head] of rows g, g+8 (heads 2c, 2c+1)
   auto qk_tile = [&](uint32_t kc, const __half* ksc, float (&sc)[NTH][4]) {
-    // ---------------- QK: S[row][head] for rows g, g+8
 #pragma unroll
     for (int nt = 0; nt < NTH; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
     float dA[NB], dB[NB];  // block scales of rows g and g+8
@@ -468,36 +486,38 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         dB[2 * i + 1] = fb.y;
       }
     }
+    const uint32_t kbase = kc + koff0;
     uint32_t kr[4];  // q4_0 keys: one x4 load per two blocks
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk) {
       uint32_t a[2][4];  // [k-step][a0..a3]
       if constexpr (KT == KVQ_Q8_0) {
         uint32_t r[4];
-        ldmatrix_x4(r, kc + koff[blk]);
+        ldmatrix_x4(r, kbase ^ blk_xor(KT, L::RBK, blk));
         const uint32_t u0 = r[0] ^ 0x80808080u, u1 = r[1] ^ 0x80808080u;
         const uint32_t u2 = r[2] ^ 0x80808080u, u3 = r[3] ^ 0x80808080u;
-        a[0][0] = prmt(u0, 0x64646464u, 0x4140);
-        a[0][2] = prmt(u0, 0x64646464u, 0x4342);
-        a[0][1] = prmt(u1, 0x64646464u, 0x4140);
-        a[0][3] = prmt(u1, 0x64646464u, 0x4342);
-        a[1][0] = prmt(u2, 0x64646464u, 0x4140);
-        a[1][2] = prmt(u2, 0x64646464u, 0x4342);
-        a[1][1] = prmt(u3, 0x64646464u, 0x4140);
-        a[1][3] = prmt(u3, 0x64646464u, 0x4342);
+        a[0][0] = prmt(u0, 0u, 0x4140);
+        a[0][2] = prmt(u0, 0u, 0x4342);
+        a[0][1] = prmt(u1, 0u, 0x4140);
+        a[0][3] = prmt(u1, 0u, 0x4342);
+        a[1][0] = prmt(u2, 0u, 0x4140);
+        a[1][2] = prmt(u2, 0u, 0x4342);
+        a[1][1] = prmt(u3, 0u, 0x4140);
+        a[1][3] = prmt(u3, 0u, 0x4342);
       } else if constexpr (KT == KVQ_Q4_0) {
         // one x4 load covers blocks blk (regs 0, 1) and blk + 1 (regs 2, 3):
         // reg = bytes 4c..4c+3 of the block in row g (even regs) or g+8 (odd)
-        if ((blk & 1) == 0) ldmatrix_x4(kr, kc + koff[blk]);
+        if ((blk & 1) == 0) ldmatrix_x4(kr, kbase ^ blk_xor(KT, L::RBK, blk));
         const uint32_t wa = kr[(blk & 1) * 2], wb = kr[(blk & 1) * 2 + 1];
-        a[0][0] = lop_and_or(wa, 0x000F000Fu, kMagic);        // dims (4c, 4c+2)
-        a[0][2] = lop_and_or(wa >> 8, 0x000F000Fu, kMagic);   // dims (4c+1, 4c+3)
-        a[1][0] = lop_and_or(wa >> 4, 0x000F000Fu, kMagic);   // dims (4c+16, 4c+18)
-        a[1][2] = lop_and_or(wa >> 12, 0x000F000Fu, kMagic);  // dims (4c+17, 4c+19)
-        a[0][1] = lop_and_or(wb, 0x000F000Fu, kMagic);
-        a[0][3] = lop_and_or(wb >> 8, 0x000F000Fu, kMagic);
-        a[1][1] = lop_and_or(wb >> 4, 0x000F000Fu, kMagic);
-        a[1][3] = lop_and_or(wb >> 12, 0x000F000Fu, kMagic);
+        const uint32_t was = wa >> 8, wbs = wb >> 8;
+        a[0][0] = wa & 0x000F000Fu;   // dims (4c, 4c+2):       n * 2^-24
+        a[0][2] = was & 0x000F000Fu;  // dims (4c+1, 4c+3)
+        a[1][0] = wa & 0x00F000F0u;   // dims (4c+16, 4c+18):  16 n * 2^-24
+        a[1][2] = was & 0x00F000F0u;  // dims (4c+17, 4c+19)
+        a[0][1] = wb & 0x000F000Fu;
+        a[0][3] = wbs & 0x000F000Fu;
+        a[1][1] = wb & 0x00F000F0u;
+        a[1][3] = wbs & 0x00F000F0u;
       } else {  // f16
 #pragma unroll
         for (int s2 = 0; s2 < 2; ++s2) {
@@ -512,17 +532,15 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 #pragma unroll
       for (int nt = 0; nt < NTH; ++nt) {
         if constexpr (L::NSK > 0) {
-          // per-block dot products from a zero accumulator; the offset
-          // correction and the block scale are applied in fp32
+          // block dot product (k-step 0 starts from the offset correction),
+          // then the row's block scale in fp32
           float dblk[4];
-          const float z4[4] = {0.f, 0.f, 0.f, 0.f};
-          mma16816(dblk, a[0][0], a[0][1], a[0][2], a[0][3], qb[nt][blk][0][0], qb[nt][blk][0][1], z4);
+          mma16816(dblk, a[0][0], a[0][1], a[0][2], a[0][3], qb[nt][blk][0][0], qb[nt][blk][0][1], cq[nt][blk]);
           mma16816(dblk, a[1][0], a[1][1], a[1][2], a[1][3], qb[nt][blk][1][0], qb[nt][blk][1][1], dblk);
-          const float c0 = corr[nt][blk][0], c1 = corr[nt][blk][1];
-          sc[nt][0] = fmaf(dA[blk], dblk[0] + c0, sc[nt][0]);
-          sc[nt][1] = fmaf(dA[blk], dblk[1] + c1, sc[nt][1]);
-          sc[nt][2] = fmaf(dB[blk], dblk[2] + c0, sc[nt][2]);
-          sc[nt][3] = fmaf(dB[blk], dblk[3] + c1, sc[nt][3]);
+          sc[nt][0] = fmaf(dA[blk], dblk[0], sc[nt][0]);
+          sc[nt][1] = fmaf(dA[blk], dblk[1], sc[nt][1]);
+          sc[nt][2] = fmaf(dB[blk], dblk[2], sc[nt][2]);
+          sc[nt][3] = fmaf(dB[blk], dblk[3], sc[nt][3]);
         } else {
           // f16 keys: no scale, no correction; accumulate in place
           mma16816(sc[nt], a[0][0], a[0][1], a[0][2], a[0][3], qb[nt][blk][0][0], qb[nt][blk][0][1], sc[nt]);
@@ -533,14 +551,13 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 #pragma unroll
     for (int nt = 0; nt < NTH; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) sc[nt][i] *= p.qscale;
+      for (int i = 0; i < 4; ++i) sc[nt][i] *= qs;
   };
 
-  // PV of one 16-row tile with its P fragments (rows 2c, 2c+1 | 2c+8, 2c+9)
+  // PV of one 16-row tile with its P fragments (rows 2c, 2c+1 | 2c+8, 2c+9);
+  // in a tail half, pmask_lo / pmask_hi zero the P rows past the split end
   auto pv_tile = [&](const unsigned char* vc, uint32_t vc32, const __half* vsc, const uint32_t (&pb)[NTH][2],
-                     bool tail,
-                     uint32_t pmask_lo, uint32_t pmask_hi) {
-    // ---------------- PV
+                     bool tail, uint32_t pmask_lo, uint32_t pmask_hi) {
     if constexpr (VT == KVQ_F16) {
 #pragma unroll
       for (int mt = 0; mt < NMT; ++mt) {
@@ -631,8 +648,12 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       }
     } else {
       // q8_0 / q4_0 values: per 32-dim block two m-tiles; each row's block scale
-      // multiplies P.  Scales of rows (2c, 2c+1) and (2c+8, 2c+9) are adjacent.
-      uint32_t sAB[L::NSV > 0 ? L::NSV : 1], sCD[L::NSV > 0 ? L::NSV : 1];  // words: row 2c blocks | row 2c+1 blocks
+      // multiplies P.  The codes enter as subnormals ((k + 128) * 2^-24 for
+      // q8_0; n * 2^-24 and 16 n * 2^-24 for the q4_0 nibbles); the code offset
+      // (128 or 8) times sum_t d[t][blk] p[t] comes from one more MMA per half
+      // tile whose A operand is the block-scale matrix (m = block, k = row).
+      // Scales of rows (2c, 2c+1) and (2c+8, 2c+9) are adjacent.
+      uint32_t sAB[L::NSV], sCD[L::NSV];  // words: row 2c blocks | row 2c+1 blocks
       if (L::NSV == 2) {
         const uint2 x = *reinterpret_cast<const uint2*>(vsc + 2 * c * L::NSV);
         const uint2 y = *reinterpret_cast<const uint2*>(vsc + (2 * c + 8) * L::NSV);
@@ -646,10 +667,32 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           sCD[4 * i] = y.x; sCD[4 * i + 1] = y.y; sCD[4 * i + 2] = y.z; sCD[4 * i + 3] = y.w;
         }
       }
+      // row 2c's scales are words 0 .. NSV/2-1, row 2c+1's are NSV/2 ..
+      {
+        uint32_t xa = sAB[0], xb = sAB[L::NSV / 2], xc = sCD[0], xd = sCD[L::NSV / 2];
+#pragma unroll
+        for (int i = 1; i < L::NSV / 2; ++i) {
+          const bool hit = (g >> 1) == i;
+          xa = hit ? sAB[i] : xa;
+          xb = hit ? sAB[L::NSV / 2 + i] : xb;
+          xc = hit ? sCD[i] : xc;
+          xd = hit ? sCD[L::NSV / 2 + i] : xd;
+        }
+        const uint32_t oa0 = prmt(xa, xb, osel) & omask, oa2 = prmt(xc, xd, osel) & omask;
+#pragma unroll
+        for (int nt = 0; nt < NTH; ++nt) {
+          uint32_t b0 = pb[nt][0], b1 = pb[nt][1];
+          if (tail) {
+            b0 &= pmask_lo;
+            b1 &= pmask_hi;
+          }
+          mma16816(off[nt], oa0, 0u, oa2, 0u, b0, b1, off[nt]);
+        }
+      }
+      const uint32_t vbase = vc32 + voff0;
       uint32_t vr[4];  // q4_0: one x4 load per two blocks
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
-        // row 2c's scales are words 0 .. NSV/2-1, row 2c+1's are NSV/2 ..
         const uint32_t sel = (blk & 1) ? 0x7632u : 0x5410u;
         const uint32_t dAB = prmt(sAB[blk >> 1], sAB[L::NSV / 2 + (blk >> 1)], sel);
         const uint32_t dCD = prmt(sCD[blk >> 1], sCD[L::NSV / 2 + (blk >> 1)], sel);
@@ -667,34 +710,31 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         if (VT == KVQ_Q4_0) {
           // trans load: reg = [row 2c: bytes 2g, 2g+1 | row 2c+1: bytes 2g, 2g+1]
           // of the block -> dims 2g, 2g+1 (low nibbles), 2g+16, 2g+17 (high)
-          if ((blk & 1) == 0) ldmatrix_x4_trans(vr, vc32 + voff[blk]);
+          if ((blk & 1) == 0) ldmatrix_x4_trans(vr, vbase ^ blk_xor(VT, L::RBV, blk));
           const uint32_t w1 = vr[(blk & 1) * 2], w2 = vr[(blk & 1) * 2 + 1];
           const uint32_t w1s = w1 >> 8, w2s = w2 >> 8;
-          a0[0] = hsub2_u32(lop_and_or(w1, 0x000F000Fu, kMagic), kBias1032);   // dim 2g, rows 2c,2c+1
-          a0[1] = hsub2_u32(lop_and_or(w1s, 0x000F000Fu, kMagic), kBias1032);  // dim 2g+1
-          a0[2] = hsub2_u32(lop_and_or(w2, 0x000F000Fu, kMagic), kBias1032);   // dim 2g, rows 2c+8,2c+9
-          a0[3] = hsub2_u32(lop_and_or(w2s, 0x000F000Fu, kMagic), kBias1032);
-          // high nibbles: 1024 + 16 n -> (x / 16) - 72 = n - 8
-          const uint32_t sc16 = 0x2C002C00u;   // fp16 1/16
-          const uint32_t m72 = 0xD480D480u;    // fp16 -72
-          a1[0] = hfma2_u32(lop_and_or(w1, 0x00F000F0u, kMagic), sc16, m72);
-          a1[1] = hfma2_u32(lop_and_or(w1s, 0x00F000F0u, kMagic), sc16, m72);
-          a1[2] = hfma2_u32(lop_and_or(w2, 0x00F000F0u, kMagic), sc16, m72);
-          a1[3] = hfma2_u32(lop_and_or(w2s, 0x00F000F0u, kMagic), sc16, m72);
+          a0[0] = w1 & 0x000F000Fu;   // dim 2g, rows 2c, 2c+1:   n * 2^-24
+          a0[1] = w1s & 0x000F000Fu;  // dim 2g+1
+          a0[2] = w2 & 0x000F000Fu;   // dim 2g, rows 2c+8, 2c+9
+          a0[3] = w2s & 0x000F000Fu;
+          a1[0] = w1 & 0x00F000F0u;   // dim 2g+16:               16 n * 2^-24
+          a1[1] = w1s & 0x00F000F0u;
+          a1[2] = w2 & 0x00F000F0u;
+          a1[3] = w2s & 0x00F000F0u;
         } else {
           // q8_0 trans load of segments 2blk (regs 0, 1) and 2blk+1 (regs 2, 3):
           // reg = [row 2c: bytes 2g, 2g+1 | row 2c+1: bytes 2g, 2g+1]
-          ldmatrix_x4_trans(vr, vc32 + voff[blk]);
+          ldmatrix_x4_trans(vr, vbase ^ blk_xor(VT, L::RBV, blk));
           const uint32_t x0 = vr[0] ^ 0x80808080u, x1 = vr[1] ^ 0x80808080u;
           const uint32_t y0 = vr[2] ^ 0x80808080u, y1 = vr[3] ^ 0x80808080u;
-          a0[0] = hsub2_u32(prmt(x0, 0x64646464u, 0x4240), kBias1152);  // dim 2g
-          a0[1] = hsub2_u32(prmt(x0, 0x64646464u, 0x4341), kBias1152);  // dim 2g+1
-          a0[2] = hsub2_u32(prmt(x1, 0x64646464u, 0x4240), kBias1152);
-          a0[3] = hsub2_u32(prmt(x1, 0x64646464u, 0x4341), kBias1152);
-          a1[0] = hsub2_u32(prmt(y0, 0x64646464u, 0x4240), kBias1152);  // dim 16+2g
-          a1[1] = hsub2_u32(prmt(y0, 0x64646464u, 0x4341), kBias1152);  // dim 16+2g+1
-          a1[2] = hsub2_u32(prmt(y1, 0x64646464u, 0x4240), kBias1152);
-          a1[3] = hsub2_u32(prmt(y1, 0x64646464u, 0x4341), kBias1152);
+          a0[0] = prmt(x0, 0u, 0x4240);  // dim 2g
+          a0[1] = prmt(x0, 0u, 0x4341);  // dim 2g+1
+          a0[2] = prmt(x1, 0u, 0x4240);
+          a0[3] = prmt(x1, 0u, 0x4341);
+          a1[0] = prmt(y0, 0u, 0x4240);  // dim 16+2g
+          a1[1] = prmt(y0, 0u, 0x4341);  // dim 16+2g+1
+          a1[2] = prmt(y1, 0u, 0x4240);
+          a1[3] = prmt(y1, 0u, 0x4341);
         }
 #pragma unroll
         for (int nt = 0; nt < NTH; ++nt) {
@@ -704,23 +744,23 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         }
       }
     }
-
   };
 
+  int st = 0;
+  uint32_t phase = 0;
 #pragma unroll 1
   for (int j = 0; j < my_tiles; ++j) {
     // one 32-row tile per iteration, as two 16-row MMA halves (the second may
     // lie past the split end): one wait and one refill per 32 rows
-    const int st = j % S;
-    const bool ok = mbar_wait(&bars[st], (uint32_t)((j / S) & 1));
+    const bool ok = mbar_wait(&bars[st], phase);
     if (!__all_sync(0xffffffffu, ok)) {
       failed_at = j;
       break;
     }
-    const int64_t r0 = t0 + (int64_t)kSub * (warp + L::NW * j);
-    const int nv0 = (int)(t1 - r0 < kHalf ? t1 - r0 : kHalf);
-    const int64_t rem1 = t1 - r0 - kHalf;
-    const int nv1 = rem1 <= 0 ? 0 : (int)(rem1 < kHalf ? rem1 : kHalf);
+    const int r0 = t0 + kSub * (warp + L::NW * j);
+    const int rem = t1 - r0;  // rows of this tile inside the split (>= 1)
+    const int nv0 = rem < kHalf ? rem : kHalf;
+    const int nv1 = rem <= kHalf ? 0 : (rem - kHalf < kHalf ? rem - kHalf : kHalf);
     const bool two = nv1 > 0;
     const bool tail0 = nv0 < kHalf, tail1 = two && nv1 < kHalf;
     const uint32_t kc0 = wbase32 + st * L::KC;
@@ -737,7 +777,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 #pragma unroll
       for (int nt = 0; nt < NTH; ++nt) sc1[nt][0] = sc1[nt][1] = sc1[nt][2] = sc1[nt][3] = -INFINITY;
     }
-    if (tail0 || tail1 || !two) {
+    if (rem < kSub) {
 #pragma unroll
       for (int nt = 0; nt < NTH; ++nt) {
         if (g >= nv0) sc0[nt][0] = sc0[nt][1] = -INFINITY;
@@ -747,28 +787,27 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       }
     }
 
-    // ---------------- online softmax over the 32 rows (heads 2c, 2c+1)
+    // ---------------- online softmax over the 32 rows (heads 2c, 2c+1).  The
+    // running max only moves when a score passes it, which after the first
+    // tiles is rare: only then are the row maxima reduced across the warp and
+    // the state rescaled.  Every P stays <= 1 either way.
     uint32_t pb0[NTH][2], pb1[NTH][2];
 #pragma unroll
     for (int nt = 0; nt < NTH; ++nt) {
       float mx0 = fmaxf(fmaxf(sc0[nt][0], sc0[nt][2]), fmaxf(sc1[nt][0], sc1[nt][2]));
       float mx1 = fmaxf(fmaxf(sc0[nt][1], sc0[nt][3]), fmaxf(sc1[nt][1], sc1[nt][3]));
+      if (__any_sync(0xffffffffu, mx0 > m_run[nt][0] || mx1 > m_run[nt][1])) {
 #pragma unroll
-      for (int o = 4; o <= 16; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-      }
-      const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-      const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
-      m_run[nt][0] = mn0;
-      m_run[nt][1] = mn1;
-      const float p0 = fast_exp2(sc0[nt][0] - mn0), p1 = fast_exp2(sc0[nt][1] - mn1);
-      const float p2 = fast_exp2(sc0[nt][2] - mn0), p3 = fast_exp2(sc0[nt][3] - mn1);
-      const float q0 = fast_exp2(sc1[nt][0] - mn0), q1 = fast_exp2(sc1[nt][1] - mn1);
-      const float q2 = fast_exp2(sc1[nt][2] - mn0), q3 = fast_exp2(sc1[nt][3] - mn1);
-      l_run[nt][0] = fmaf(l_run[nt][0], al0, (p0 + p2) + (q0 + q2));
-      l_run[nt][1] = fmaf(l_run[nt][1], al1, (p1 + p3) + (q1 + q3));
-      if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+        for (int o = 4; o <= 16; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+        const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
+        m_run[nt][0] = mn0;
+        m_run[nt][1] = mn1;
+        l_run[nt][0] *= al0;
+        l_run[nt][1] *= al1;
 #pragma unroll
         for (int i = 0; i < NMT; ++i) {
           acc[nt][i][0] *= al0;
@@ -776,13 +815,23 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           acc[nt][i][2] *= al0;
           acc[nt][i][3] *= al1;
         }
+        if (kVQ) {
+          off[nt][0] *= al0;
+          off[nt][1] *= al1;
+        }
       }
+      const float p0 = fast_exp2(sc0[nt][0] - m_run[nt][0]), p1 = fast_exp2(sc0[nt][1] - m_run[nt][1]);
+      const float p2 = fast_exp2(sc0[nt][2] - m_run[nt][0]), p3 = fast_exp2(sc0[nt][3] - m_run[nt][1]);
+      const float q0 = fast_exp2(sc1[nt][0] - m_run[nt][0]), q1 = fast_exp2(sc1[nt][1] - m_run[nt][1]);
+      const float q2 = fast_exp2(sc1[nt][2] - m_run[nt][0]), q3 = fast_exp2(sc1[nt][3] - m_run[nt][1]);
+      l_run[nt][0] += (p0 + p2) + (q0 + q2);
+      l_run[nt][1] += (p1 + p3) + (q1 + q3);
       pb0[nt][0] = movmatrix_trans(pack_half2(p0, p1));
       pb0[nt][1] = movmatrix_trans(pack_half2(p2, p3));
       pb1[nt][0] = movmatrix_trans(pack_half2(q0, q1));
       pb1[nt][1] = movmatrix_trans(pack_half2(q2, q3));
     }
-    // In a tail tile, P rows past the split end contribute exactly 0 whatever
+    // In a tail half, P rows past the split end contribute exactly 0 whatever
     // the row's scale holds (b operand halves: rows 2c, 2c+1 | 2c+8, 2c+9).
     auto pmask = [&](int nv, uint32_t& lo, uint32_t& hi) {
       lo = (2 * c < nv ? 0x0000FFFFu : 0u) | (2 * c + 1 < nv ? 0xFFFF0000u : 0u);
@@ -800,7 +849,11 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     __syncwarp();
     if (lane == 0 && j + S < my_tiles) {
       fence_proxy_async();
-      issue(j + S);
+      issue(j + S, st);
+    }
+    if (++st == S) {
+      st = 0;
+      phase ^= 1u;
     }
   }
 
@@ -822,6 +875,29 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     for (int e = 0; e < 2; ++e)
 #pragma unroll
       for (int o = 4; o <= 16; o <<= 1) l_run[nt][e] += __shfl_xor_sync(0xffffffffu, l_run[nt][e], o);
+
+  // ---- q8_0 / q4_0 values: take the 2^24 (2^20) out and subtract the code
+  //      offset times sum_t d[t][blk] p[t] (held by lane 4 * blk + c)
+  if constexpr (kVQ) {
+    constexpr float vb = VT == KVQ_Q8_0 ? 128.f : 8.f;
+#pragma unroll
+    for (int nt = 0; nt < NTH; ++nt) {
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk) {
+        const float o0 = -vb * __shfl_sync(0xffffffffu, off[nt][0], blk * 4 + c);
+        const float o1 = -vb * __shfl_sync(0xffffffffu, off[nt][1], blk * 4 + c);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int mt = 2 * blk + h;
+          const float f = (VT == KVQ_Q4_0 && h == 1) ? kTwo20 : kTwo24;
+          acc[nt][mt][0] = fmaf(acc[nt][mt][0], f, o0);
+          acc[nt][mt][1] = fmaf(acc[nt][mt][1], f, o1);
+          acc[nt][mt][2] = fmaf(acc[nt][mt][2], f, o0);
+          acc[nt][mt][3] = fmaf(acc[nt][mt][3], f, o1);
+        }
+      }
+    }
+  }
 
   __syncthreads();  // every warp is done with its stages: reuse them for the merge
 
