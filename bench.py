@@ -251,7 +251,7 @@ def run_reference(args):
 def _config(w, args, n_layers):
     return {"workload": w.name, "layers": n_layers or w.layers, "batch": w.batch, "n_q_heads": w.n_q,
             "n_kv_heads": w.n_kv, "head_dim": w.head_dim, "ctx": w.ctx, "k_type": w.k_type,
-            "v_type": w.v_type, "step": "per layer: append 1 row + split decode + combine",
+            "v_type": w.v_type, "step": "per layer: one fused launch (append 1 row + split decode + combine)",
             "l2": "inputs larger than L2: every layer a distinct cache buffer larger than the 126 MB L2"}
 
 
@@ -325,19 +325,27 @@ def run_kvq(args):
     torch.cuda.empty_cache()
 
     S = kvq.kvq_auto_splits(desc, B, ctx)
-    ws = torch.empty(kvq.kvq_workspace_bytes(desc, B, 0), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(kvq.kvq_workspace_bytes(desc, B, 0), dtype=torch.uint8, device=dev)  # counters start at 0
     outs = [torch.empty((B, w.n_q, w.head_dim), dtype=torch.float32, device=dev) for _ in range(L)]
     scale = w.scale
 
     def step(events=None):
-        """One decode token through every layer, launched on the current stream."""
+        """One decode token through every layer, launched on the current stream:
+        per layer one fused launch (append the token's K/V row, split decode,
+        combine)."""
         for layer in range(L):
-            kvq.kvq_append_quantize(desc, kcs[layer], vcs[layer], kn[layer], vn[layer], B, ctx - 1, 1)
             if events is not None:
                 events[layer][0].record()
-            kvq.kvq_decode_attention(desc, kcs[layer], vcs[layer], qs[layer], B, ctx, scale, 0, ws)
+            kvq.kvq_decode_step(desc, kcs[layer], vcs[layer], qs[layer], kn[layer], vn[layer], B, ctx, scale, 0,
+                                ws, outs[layer])
             if events is not None:
                 events[layer][1].record()
+
+    def step_unfused():
+        """The same step as three launches per layer (append, decode, combine)."""
+        for layer in range(L):
+            kvq.kvq_append_quantize(desc, kcs[layer], vcs[layer], kn[layer], vn[layer], B, ctx - 1, 1)
+            kvq.kvq_decode_attention(desc, kcs[layer], vcs[layer], qs[layer], B, ctx, scale, 0, ws)
             kvq.kvq_combine(desc, ws, B, ctx, 0, outs[layer])
 
     def barrier():
@@ -349,14 +357,9 @@ def run_kvq(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    try:
-        dec_ev = [(torch.cuda.Event(enable_timing=True, external=True),
-                   torch.cuda.Event(enable_timing=True, external=True)) for _ in range(L)]
-    except TypeError:
-        dec_ev = None
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        step(dec_ev)
+        step()
     for _ in range(args.warmup):
         graph.replay()
     barrier()
@@ -372,21 +375,41 @@ def run_kvq(args):
     clocks.end()
     clk = clocks.stop()
     ms = t_start.elapsed_time(t_end)
-    if dec_ev is not None:
-        dec_ms = [a.elapsed_time(b) for a, b in dec_ev]   # the last timed replay's launches
-    else:
-        dec_graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(dec_graph):
-            for layer in range(L):
-                kvq.kvq_decode_attention(desc, kcs[layer], vcs[layer], qs[layer], B, ctx, scale, 0, ws)
-        dec_graph.replay()
-        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        dec_graph.replay()
-        b2.record()
-        torch.cuda.synchronize()
-        dec_ms = [a.elapsed_time(b2) / L]
     del graph
+
+    # ---- each launch bracketed by event nodes (a separate replay: the nodes
+    #      themselves add time, so the headline graph above has none)
+    try:
+        dec_ev = [(torch.cuda.Event(enable_timing=True, external=True),
+                   torch.cuda.Event(enable_timing=True, external=True)) for _ in range(L)]
+        egraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(egraph):
+            step(dec_ev)
+        for _ in range(2):
+            egraph.replay()
+        torch.cuda.synchronize()
+        ev_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_ev)
+        del egraph
+    except TypeError:
+        ev_ms = float("nan")
+
+    # ---- the same step as three launches per layer, for comparison (not the headline)
+    step_unfused()
+    torch.cuda.synchronize()
+    ugraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ugraph):
+        step_unfused()
+    for _ in range(args.warmup):
+        ugraph.replay()
+    barrier()
+    u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    u0.record()
+    for _ in range(args.steps):
+        ugraph.replay()
+    u1.record()
+    barrier()
+    unfused_ms = u0.elapsed_time(u1)
+    del ugraph
 
     # ---- end to end through the public API with host buffers: every layer's
     #      query and new K/V rows copied in from pinned host memory, every
@@ -404,9 +427,8 @@ def run_kvq(args):
             qd[layer].copy_(q_h[layer], non_blocking=True)
             knd[layer].copy_(kn_h[layer], non_blocking=True)
             vnd[layer].copy_(vn_h[layer], non_blocking=True)
-            kvq.kvq_append_quantize(desc, kcs[layer], vcs[layer], knd[layer], vnd[layer], B, ctx - 1, 1)
-            kvq.kvq_decode_attention(desc, kcs[layer], vcs[layer], qd[layer], B, ctx, scale, 0, ws)
-            kvq.kvq_combine(desc, ws, B, ctx, 0, outs[layer])
+            kvq.kvq_decode_step(desc, kcs[layer], vcs[layer], qd[layer], knd[layer], vnd[layer], B, ctx, scale, 0,
+                                ws, outs[layer])
             out_h[layer].copy_(outs[layer], non_blocking=True)
 
     e2e_step()
@@ -427,7 +449,8 @@ def run_kvq(args):
     del e2e_graph
 
     # ---- max over ranks
-    ms, e2e_ms, dec_avg = max_over_ranks([ms, e2e_ms, statistics.mean(dec_ms)], world, dev)
+    ms, e2e_ms, ev_ms, unfused_ms = max_over_ranks([ms, e2e_ms, ev_ms, unfused_ms], world, dev)
+    dec_avg = ms / (args.steps * L)   # one launch per layer step: the average launch period
 
     dec_bytes, app_bytes, step_bytes = algorithmic_bytes(w, L)
     value = whole_job_gbs(world, step_bytes, args.steps, ms)
@@ -440,7 +463,8 @@ def run_kvq(args):
     peak = peaks.get("hbm_gbs")
     peak_src = "measured" if peak else "fallback"
     peak = peak or 6650.0
-    achieved = dec_bytes / (dec_avg * 1e-3) / 1e9
+    launch_bytes = dec_bytes + app_bytes          # what one fused step launch must move
+    achieved = launch_bytes / (dec_avg * 1e-3) / 1e9
     ms_step = ms / args.steps
     traffic = _profiled_traffic(w.name)
 
@@ -454,16 +478,19 @@ def run_kvq(args):
             "tokens_per_s": round(world * B * 1e3 / ms_step, 2),
             "frac_of_8tbs": round(value / 8000.0, 4),
             "splits": S,
-            "roofline": {"bound": "hbm", "kernel": "decode split kernel", "achieved": round(achieved, 2),
+            "roofline": {"bound": "hbm", "kernel": "fused decode step (append + split decode + combine)",
+                         "achieved": round(achieved, 2),
                          "peak": peak, "peak_source": f"{peak_src} copy bandwidth", "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "algorithmic_bytes_per_launch": dec_bytes,
-                         "avg_launch_us": round(dec_avg * 1e3, 3)},
+                         "algorithmic_bytes_per_launch": launch_bytes,
+                         "avg_launch_us": round(dec_avg * 1e3, 3),
+                         "launch_us_between_event_nodes": None if ev_ms != ev_ms else round(ev_ms * 1e3, 3)},
             "e2e": {"value": round(e2e_value, 3), "unit": UNIT,
                     "h2d_bytes_per_step": L * (qs[0].numel() * 2 + kn[0].numel() * 2 + vn[0].numel() * 2),
                     "d2h_bytes_per_step": L * outs[0].numel() * 4},
-            "gpu_launches": args.steps * L * 3,
-            "timing": "CUDA-graph replays of whole steps; decode launch time from event nodes in the graph",
+            "gpu_launches": args.steps * L,
+            "step_unfused_us_per_layer": round(1e3 * unfused_ms / args.steps / L, 3),
+            "timing": "CUDA-graph replays of whole steps (no event nodes); avg launch = timed region / launches",
             "append_bulk": {"rows_per_layer": B * ctx * w.n_kv, "us_per_layer": round(1e3 * statistics.median(prefill_ms), 2),
                             "GB_per_s": round((B * w.n_kv * ctx * (2 * w.head_dim * 2 + row_bytes(w.k_type, w.head_dim)
                                                                      + row_bytes(w.v_type, w.head_dim)))

@@ -33,7 +33,7 @@ EXPORTED = (
     "kvq_status_string", "kvq_last_cuda_error", "kvq_row_bytes", "kvq_check_desc",
     "kvq_cache_layout", "kvq_cache_bytes", "kvq_auto_splits", "kvq_workspace_bytes",
     "kvq_turbo3_codebook", "kvq_turbo3_signs", "kvq_append_quantize",
-    "kvq_decode_attention", "kvq_combine", "kvq_decode_attention_noalloc",
+    "kvq_decode_attention", "kvq_combine", "kvq_decode_attention_noalloc", "kvq_decode_step",
 )
 
 
@@ -81,6 +81,8 @@ _sigs = {
                                    _P, _P]),
     "kvq_decode_attention_noalloc": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
                                                     ctypes.c_int32, _P, _P]),
+    "kvq_decode_step": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                                       ctypes.c_int32, _P, ctypes.c_size_t, _P, _P]),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -208,6 +210,19 @@ def kvq_decode_attention_noalloc(desc, k_cache, v_cache, q, batch, ctx_len, soft
                                                     batch, ctx_len, softmax_scale, n_splits, _ptr(out),
                                                     _stream(stream)),
                   "kvq_decode_attention_noalloc")
+
+
+def kvq_decode_step(desc, k_cache, v_cache, q, k_new, v_new, batch, ctx_len, softmax_scale, n_splits, workspace,
+                    out, workspace_bytes=None, stream=None):
+    """Append one row per batch entry at row ctx_len - 1, decode over rows
+    0 .. ctx_len-1 and combine into ``out``, in one launch (see include/kvq.h;
+    the workspace's counter words must be zero before its first use)."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return _check(_lib.kvq_decode_step(ctypes.byref(desc), _ptr(k_cache), _ptr(v_cache), _ptr(q), _ptr(k_new),
+                                       _ptr(v_new), batch, ctx_len, softmax_scale, n_splits, _ptr(workspace),
+                                       workspace_bytes, _ptr(out), _stream(stream)),
+                  "kvq_decode_step")
 
 
 def raw_status(name, *args):

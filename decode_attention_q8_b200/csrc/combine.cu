@@ -56,12 +56,15 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
   const float* acc = p.ws_acc + base * p.D + j;
   float num = 0.f;
   int s = 0;
-  for (; s + 4 <= p.S; s += 4) {
-    const float a0 = acc[(int64_t)(s + 0) * p.D], a1 = acc[(int64_t)(s + 1) * p.D];
-    const float a2 = acc[(int64_t)(s + 2) * p.D], a3 = acc[(int64_t)(s + 3) * p.D];
-    num += wts[s] * a0 + wts[s + 1] * a1 + wts[s + 2] * a2 + wts[s + 3] * a3;
+  constexpr int kU = 16;  // independent loads per round: the partials may come from HBM
+  for (; s + kU <= p.S; s += kU) {
+    float a[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) a[u] = acc[(int64_t)(s + u) * p.D];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) num = fmaf(wts[s + u], a[u], num);
   }
-  for (; s < p.S; ++s) num += wts[s] * acc[(int64_t)s * p.D];
+  for (; s < p.S; ++s) num = fmaf(wts[s], acc[(int64_t)s * p.D], num);
   float o = num / den;
   if (p.turbo3) {
     xs[j] = o;

@@ -107,6 +107,7 @@ bool decode_supported(int32_t k_type, int32_t v_type, int32_t G, int32_t D) {
 
 int decode_ctas_per_sm() { return 2; }
 
+
 cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p, cudaStream_t st) {
   tc::TcMaps maps;
   const int64_t planes = (int64_t)p.B * p.n_kv;

@@ -58,7 +58,7 @@
 
 #include <cuda.h>
 
-#include "kvq_internal.h"
+#include "append_rows.cuh"
 
 namespace kvq {
 namespace tc {
@@ -110,8 +110,7 @@ struct Layout {
   static constexpr int BARS = NW * kStages * 8;
   static constexpr int TX = kSub * (RBK + 2 * NSK + RBV + 2 * NSV);  // bytes landing per tile
   // CTA-level merge scratch (reuses the stage memory after the main loop)
-  static constexpr int MERGE_HEADS = 8;
-  static constexpr int MERGE = NW * MERGE_HEADS * (D + 2) * 4;
+  static constexpr int MERGE = NW * ((D / 16) * 32 * 4 + 16) * 4;  // fragment chunks + m, l per warp
   static constexpr int TOTAL = 1024 + NW * WARP + TABLE + BARS + 16;
   static_assert(MERGE <= NW * WARP, "merge area must fit in the stage memory");
   static_assert(TOTAL <= 227 * 1024, "shared memory per CTA");
@@ -170,28 +169,48 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+// Tensor copies of cache tiles carry an L2 evict-first policy: every cache
+// byte is read once per decode, so it should not displace what is read again
+// (the split partials the combine reads back, the queries).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
+                                            uint64_t pol) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-          "r"(smem_addr(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar))
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(pol)
       : "memory");
 }
 
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar,
+                                            uint64_t pol) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-      "[%5];" ::"r"(smem_addr(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar)), "l"(pol)
       : "memory");
 }
 
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
-                                            uint64_t* bar) {
+                                            uint64_t* bar, uint64_t pol) {
   asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
-      "%5}], [%6];" ::"r"(smem_addr(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar))
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar)), "l"(pol)
+      : "memory");
+}
+
+// Contiguous global -> shared copy by the bulk-copy engine (16-byte aligned
+// addresses, size a multiple of 16), completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
 
@@ -328,28 +347,51 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 
   // tile j of this warp covers rows t0 + 32*(warp + NW*j) ...
   const int my_tiles = n_sub > warp ? (n_sub - warp + L::NW - 1) / L::NW : 0;
+  const uint64_t pol = l2_evict_first_policy();
   auto issue = [&](int j, int st) {
     const int r0 = t0 + kSub * (warp + L::NW * j);
     mbar_expect_tx(&bars[st], L::TX);
     if (L::RBK > 128)
-      tma_load_4d(kc_of(st), &tm_kc, 0, 0, r0, plane, &bars[st]);
+      tma_load_4d(kc_of(st), &tm_kc, 0, 0, r0, plane, &bars[st], pol);
     else
-      tma_load_3d(kc_of(st), &tm_kc, 0, r0, plane, &bars[st]);
-    if (L::NSK) tma_load_2d(ks_of(st), &tm_ks, r0 * L::NSK / 2, plane, &bars[st]);
+      tma_load_3d(kc_of(st), &tm_kc, 0, r0, plane, &bars[st], pol);
+    if (L::NSK) tma_load_2d(ks_of(st), &tm_ks, r0 * L::NSK / 2, plane, &bars[st], pol);
     if (VT == KVQ_TURBO3) {
       if (kSub * L::RBV / 4 <= 256)
-        tma_load_2d(vc_of(st), &tm_vc, r0 * L::RBV / 4, plane, &bars[st]);
+        tma_load_2d(vc_of(st), &tm_vc, r0 * L::RBV / 4, plane, &bars[st], pol);
       else
-        tma_load_3d(vc_of(st), &tm_vc, 0, r0, plane, &bars[st]);
+        tma_load_3d(vc_of(st), &tm_vc, 0, r0, plane, &bars[st], pol);
     } else if (L::RBV > 128) {
-      tma_load_4d(vc_of(st), &tm_vc, 0, 0, r0, plane, &bars[st]);
+      tma_load_4d(vc_of(st), &tm_vc, 0, 0, r0, plane, &bars[st], pol);
     } else {
-      tma_load_3d(vc_of(st), &tm_vc, 0, r0, plane, &bars[st]);
+      tma_load_3d(vc_of(st), &tm_vc, 0, r0, plane, &bars[st], pol);
     }
-    if (L::NSV) tma_load_2d(vs_of(st), &tm_vs, r0 * L::NSV / 2, plane, &bars[st]);
+    if (L::NSV) tma_load_2d(vs_of(st), &tm_vs, r0 * L::NSV / 2, plane, &bars[st], pol);
   };
+  // Fused decode step: the new row (row append_pos) lies in tile jt of warp wt
+  // of the CTA whose split holds it.  That warp issues its other first tiles,
+  // then quantizes and writes the row of K and of V itself, makes the writes
+  // visible device-wide and to the async proxy, and only then issues the tile
+  // that reads the row back; no other warp waits.
+  const bool owner = p.append_pos >= t0l && p.append_pos < t1l;
+  const int t_new = owner ? (int)(p.append_pos - t0l) / kSub : -1;
+  const int wt = owner ? t_new % L::NW : -1, jt = owner ? t_new / L::NW : -1;
   if (lane == 0) {
-    for (int j = 0; j < S && j < my_tiles; ++j) issue(j, j);
+    for (int j = 0; j < S && j < my_tiles; ++j)
+      if (!(warp == wt && j == jt)) issue(j, j);
+  }
+  if (warp == wt) {
+    constexpr int rk = rows::row_threads(KT, D), rv = rows::row_threads(VT, D);
+#pragma unroll
+    for (int t = 0; t < rk; t += 32)
+      rows::append_any(KT, p.app_k, (int64_t)plane * rk + t + lane, (int64_t)(plane + 1) * rk);
+#pragma unroll
+    for (int t = 0; t < rv; t += 32)
+      rows::append_any(VT, p.app_v, (int64_t)plane * rv + t + lane, (int64_t)(plane + 1) * rv);
+    __threadfence();
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncwarp();
+    if (lane == 0 && jt < S && jt < my_tiles) issue(jt, jt);
   }
 
   // ---- queries: B fragments of Q^T per (block, k-step) and, for quantized
@@ -901,59 +943,240 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 
   __syncthreads();  // every warp is done with its stages: reuse them for the merge
 
-  // merge area: per warp [8 heads][D] acc, then m[8], l[8]
+  // ---- merge of the warps.  Each warp stores its accumulator fragments as
+  //      they lie in registers (16-byte chunks, lane-major: no bank conflicts)
+  //      and its per-head m and l; thread t then sums chunk t over the warps,
+  //      weighted by 2^(m_w - M) of the chunk's two heads (2c, 2c+1).
+  constexpr int CH = NMT * 32;          // 16-byte chunks per warp and n-tile
+  constexpr int WSTRIDE = CH * 4 + 16;  // floats per warp: chunks, m[8], l[8]
   float* mrg = reinterpret_cast<float*>(smem);
   auto dim_of = [&](int mt, int row) -> int {  // PV m-tile row -> head dim
     if (VT == KVQ_F16) return 16 * mt + row;                       // row in 0..15
     if (VT == KVQ_TURBO3) return (row & 7) * (D / 8) + 2 * mt + (row >> 3);
     return 32 * (mt >> 1) + 16 * (mt & 1) + 2 * (row & 7) + (row >> 3);  // q8_0, q4_0
   };
+  const bool failed = cta_failed != 0;
 #pragma unroll
   for (int nt = 0; nt < NTH; ++nt) {
-    float* wacc = mrg + warp * (8 * D + 16);
-    float* wm = wacc + 8 * D;
-    float* wl = wm + 8;
+    float* wf = mrg + warp * WSTRIDE;
 #pragma unroll
-    for (int mt = 0; mt < NMT; ++mt) {
-      wacc[(2 * c) * D + dim_of(mt, g)] = acc[nt][mt][0];
-      wacc[(2 * c + 1) * D + dim_of(mt, g)] = acc[nt][mt][1];
-      wacc[(2 * c) * D + dim_of(mt, g + 8)] = acc[nt][mt][2];
-      wacc[(2 * c + 1) * D + dim_of(mt, g + 8)] = acc[nt][mt][3];
-    }
+    for (int mt = 0; mt < NMT; ++mt)
+      *reinterpret_cast<float4*>(wf + (mt * 32 + lane) * 4) =
+          make_float4(acc[nt][mt][0], acc[nt][mt][1], acc[nt][mt][2], acc[nt][mt][3]);
     if (g == 0) {
-      wm[2 * c] = m_run[nt][0];
-      wm[2 * c + 1] = m_run[nt][1];
-      wl[2 * c] = l_run[nt][0];
-      wl[2 * c + 1] = l_run[nt][1];
+      wf[CH * 4 + 2 * c] = m_run[nt][0];
+      wf[CH * 4 + 2 * c + 1] = m_run[nt][1];
+      wf[CH * 4 + 8 + 2 * c] = l_run[nt][0];
+      wf[CH * 4 + 8 + 2 * c + 1] = l_run[nt][1];
     }
     __syncthreads();
     const int heads_here = min(8, p.G - nt * 8);
-    for (int i = threadIdx.x; i < heads_here * D; i += L::NW * 32) {
-      const int h = i / D, dd = i % D;
-      float M = -INFINITY;
+    const int64_t row0 = ((int64_t)b * p.n_q + (int64_t)kvh * p.G + nt * 8) * p.S + s_idx;  // head 0's row
+    for (int i = threadIdx.x; i < CH; i += L::NW * 32) {
+      const int mt = i >> 5, gg = (i >> 2) & 7, cc = i & 3;
+      const int hA = 2 * cc, hB = 2 * cc + 1;
+      float MA = -INFINITY, MB = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < L::NW; ++w) M = fmaxf(M, mrg[w * (8 * D + 16) + 8 * D + h]);
-      float a = 0.f, l = 0.f;
-      if (M != -INFINITY) {
+      for (int w = 0; w < L::NW; ++w) {
+        MA = fmaxf(MA, mrg[w * WSTRIDE + CH * 4 + hA]);
+        MB = fmaxf(MB, mrg[w * WSTRIDE + CH * 4 + hB]);
+      }
+      float fA[L::NW], fB[L::NW];
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < L::NW; ++w) {
+        // a warp without rows has m = -inf: weight 0 (all weights 0 if no warp has rows)
+        fA[w] = MA == -INFINITY ? 0.f : fast_exp2(mrg[w * WSTRIDE + CH * 4 + hA] - MA);
+        fB[w] = MB == -INFINITY ? 0.f : fast_exp2(mrg[w * WSTRIDE + CH * 4 + hB] - MB);
+        const float4 x = *reinterpret_cast<const float4*>(mrg + w * WSTRIDE + i * 4);
+        sum.x = fmaf(fA[w], x.x, sum.x);
+        sum.y = fmaf(fB[w], x.y, sum.y);
+        sum.z = fmaf(fA[w], x.z, sum.z);
+        sum.w = fmaf(fB[w], x.w, sum.w);
+      }
+      if (failed) sum = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                                    __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+      const int dA = dim_of(mt, gg), dB = dim_of(mt, gg + 8);
+      if (hA < heads_here) {
+        p.ws_acc[(row0 + (int64_t)hA * p.S) * D + dA] = sum.x;
+        p.ws_acc[(row0 + (int64_t)hA * p.S) * D + dB] = sum.z;
+      }
+      if (hB < heads_here) {
+        p.ws_acc[(row0 + (int64_t)hB * p.S) * D + dA] = sum.y;
+        p.ws_acc[(row0 + (int64_t)hB * p.S) * D + dB] = sum.w;
+      }
+      if (mt == 0 && gg == 0) {  // one thread per head pair: m and l
+        float lA = 0.f, lB = 0.f;
 #pragma unroll
         for (int w = 0; w < L::NW; ++w) {
-          const float* base = mrg + w * (8 * D + 16);
-          const float mw = base[8 * D + h];
-          if (mw == -INFINITY) continue;
-          const float f = exp2f(mw - M);
-          a = fmaf(f, base[h * D + dd], a);
-          l = fmaf(f, base[8 * D + 8 + h], l);
+          lA = fmaf(fA[w], mrg[w * WSTRIDE + CH * 4 + 8 + hA], lA);
+          lB = fmaf(fB[w], mrg[w * WSTRIDE + CH * 4 + 8 + hB], lB);
         }
-      }
-      if (cta_failed) a = l = M = __int_as_float(0x7fc00000);  // NaN
-      const int64_t row = ((int64_t)b * p.n_q + (int64_t)kvh * p.G + nt * 8 + h) * p.S + s_idx;
-      p.ws_acc[row * D + dd] = a;
-      if (dd == 0) {
-        p.ws_m[row] = M;
-        p.ws_l[row] = l;
+        const float nan = __int_as_float(0x7fc00000);
+        if (hA < heads_here) {
+          p.ws_m[row0 + (int64_t)hA * p.S] = failed ? nan : MA;
+          p.ws_l[row0 + (int64_t)hA * p.S] = failed ? nan : lA;
+        }
+        if (hB < heads_here) {
+          p.ws_m[row0 + (int64_t)hB * p.S] = failed ? nan : MB;
+          p.ws_l[row0 + (int64_t)hB * p.S] = failed ? nan : lB;
+        }
       }
     }
     __syncthreads();
+  }
+
+  // ---- fused decode step: the last CTA of this (batch row, KV head) to
+  //      finish merges the S split partials of the group's G heads into the
+  //      output (the arithmetic of kvq_combine, with the inverse rotation of a
+  //      turbo3 value cache).  The arrival counter wraps to 0 at S.
+  if (p.out != nullptr) {
+    __shared__ unsigned int last_cta;
+    __threadfence();  // this CTA's partials are visible device-wide ...
+    __syncthreads();
+    if (threadIdx.x == 0)  // ... before its arrival is counted
+      last_cta = atomicInc(p.counters + plane, (unsigned)(p.S - 1)) == (unsigned)(p.S - 1);
+    __syncthreads();
+    if (last_cta) {
+      __threadfence();
+      // The partials of the group (G heads x S splits x D floats) come into the
+      // free stage memory by bulk copies, one per head and round of up to 32
+      // splits; m and l are read alongside.  One warp per head then folds the
+      // round into its running (max, sum, weighted acc), D/32 consecutive dims
+      // per lane.
+      constexpr int E = D / 32;                        // dims per lane
+      constexpr int HPW = (16 + L::NW - 1) / L::NW;    // heads per warp, G <= 16
+      constexpr int kAvail = L::NW * L::WARP / 4;      // floats of stage memory
+      const int G = p.G, S_ = p.S;
+      float* buf = reinterpret_cast<float*>(smem);     // [G][SC][D]
+      const int SC = max(1, min(32, min(S_, kAvail / (G * D))));
+      const int64_t grow0 = ((int64_t)b * p.n_q + (int64_t)kvh * G) * S_;  // (head 0, split 0)
+      // one mbarrier for the rounds' bulk copies (the pipeline's are idle now)
+      __shared__ uint64_t comb_bar[1];
+      uint64_t* cbar = comb_bar;
+      uint32_t cphase = 0;
+      int comb_failed = 0;
+      if (threadIdx.x == 0) {
+        mbar_init(cbar, 1);
+        fence_barrier_init();
+      }
+      fence_proxy_async();  // the merge's generic writes to the stage memory come before the copies into it
+      __syncthreads();
+      float Mh[HPW], den[HPW], num[HPW][E];
+#pragma unroll
+      for (int hi = 0; hi < HPW; ++hi) {
+        Mh[hi] = -INFINITY;
+        den[hi] = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) num[hi][e] = 0.f;
+      }
+      for (int s0 = 0; s0 < S_; s0 += SC) {
+        const int sc = min(SC, S_ - s0);
+        if (threadIdx.x == 0) {
+          mbar_expect_tx(cbar, (uint32_t)(G * sc * D * 4));
+          for (int h = 0; h < G; ++h)
+            bulk_load(buf + h * SC * D, p.ws_acc + (grow0 + (int64_t)h * S_ + s0) * D, (uint32_t)(sc * D * 4), cbar);
+        }
+        float mj[HPW], lj[HPW];  // this round's m, l of split s0 + lane
+#pragma unroll
+        for (int hi = 0; hi < HPW; ++hi) {
+          const int h = warp + hi * L::NW;
+          mj[hi] = -INFINITY;
+          lj[hi] = 0.f;
+          if (h < G && lane < sc) {
+            mj[hi] = __ldcg(p.ws_m + grow0 + (int64_t)h * S_ + s0 + lane);
+            lj[hi] = __ldcg(p.ws_l + grow0 + (int64_t)h * S_ + s0 + lane);
+          }
+        }
+        const bool landed = mbar_wait(cbar, cphase);
+        if (!__syncthreads_and(landed)) {
+          // a copy did not land within the limit: let it drain (bounded
+          // again) so nothing writes shared memory after the CTA exits; the
+          // group's outputs read NaN
+          if (threadIdx.x == 0) (void)mbar_wait(cbar, cphase);
+          __syncthreads();
+          comb_failed = 1;
+          break;
+        }
+        cphase ^= 1u;
+#pragma unroll
+        for (int hi = 0; hi < HPW; ++hi) {
+          const int h = warp + hi * L::NW;
+          if (h >= G) break;
+          float mc = mj[hi];
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+          const float mn = fmaxf(Mh[hi], mc);
+          // an empty split (m = -inf) weighs 0; so does the old state while no split had rows
+          const float alpha = Mh[hi] == -INFINITY ? 0.f : exp2f(Mh[hi] - mn);
+          const float wl = mj[hi] == -INFINITY ? 0.f : exp2f(mj[hi] - mn);
+          float dl = wl * lj[hi];
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
+          den[hi] = fmaf(den[hi], alpha, dl);
+#pragma unroll
+          for (int e = 0; e < E; ++e) num[hi][e] *= alpha;
+          const float* hb = buf + h * SC * D + lane * E;
+          for (int j = 0; j < sc; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, wl, j);
+#pragma unroll
+            for (int e4 = 0; e4 < E; e4 += 2) {
+              const float2 x2 = *reinterpret_cast<const float2*>(hb + j * D + e4);
+              num[hi][e4] = fmaf(wj, x2.x, num[hi][e4]);
+              num[hi][e4 + 1] = fmaf(wj, x2.y, num[hi][e4 + 1]);
+            }
+          }
+          Mh[hi] = mn;
+        }
+        fence_proxy_async();  // this round's reads of the buffer come before the next round's copies
+        __syncthreads();
+      }
+#pragma unroll
+      for (int hi = 0; hi < HPW; ++hi) {
+        const int h = warp + hi * L::NW;
+        if (h >= G) break;
+        float o_v[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) o_v[e] = comb_failed ? __int_as_float(0x7fc00000) : num[hi][e] / den[hi];
+        if (VT == KVQ_TURBO3) {
+          // o <- s * H_un * o / D: butterflies of strides 1 .. E/2 in registers,
+          // E .. D/2 across lanes
+#pragma unroll
+          for (int hs = 1; hs < E; hs <<= 1)
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+              if ((e & hs) == 0) {
+                const float a0 = o_v[e], a1 = o_v[e + hs];
+                o_v[e] = a0 + a1;
+                o_v[e + hs] = a0 - a1;
+              }
+#pragma unroll
+          for (int hs = E; hs < D; hs <<= 1) {
+            const int lm = hs / E;
+            const bool upper = (lane & lm) != 0;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              const float other = __shfl_xor_sync(0xffffffffu, o_v[e], lm);
+              o_v[e] = upper ? other - o_v[e] : o_v[e] + other;
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const int d = lane * E + e;
+            const float sgn = ((p.t3.sign_bits[d >> 5] >> (d & 31)) & 1u) ? -1.f : 1.f;
+            o_v[e] = o_v[e] * sgn / (float)D;
+          }
+        }
+        float* dst = p.out + ((int64_t)b * p.n_q + (int64_t)kvh * G + h) * D + lane * E;
+        if constexpr (E == 2) {
+          *reinterpret_cast<float2*>(dst) = make_float2(o_v[0], o_v[1]);
+        } else {
+#pragma unroll
+          for (int e4 = 0; e4 < E; e4 += 4)
+            *reinterpret_cast<float4*>(dst + e4) = make_float4(o_v[e4], o_v[e4 + 1], o_v[e4 + 2], o_v[e4 + 3]);
+        }
+      }
+    }
   }
 }
 

@@ -182,14 +182,17 @@ int32_t resolve_splits(const kvq_cache_desc* d, int32_t batch, int64_t ctx, int3
 }
 
 struct WsLayout {
-  int64_t m_off, l_off, acc_off, total;
+  int64_t m_off, l_off, acc_off, cnt_off, total;
 };
 
+// Counters first: their place depends on batch and n_kv only, so calls with
+// different split counts on one workspace keep them intact.
 WsLayout ws_layout(const kvq_cache_desc* d, int32_t batch, int32_t S) {
   WsLayout w;
   const int64_t rows = (int64_t)batch * d->n_q_heads * S;
-  w.m_off = 0;
-  w.l_off = round_up(rows * 4, 256);
+  w.cnt_off = 0;
+  w.m_off = round_up((int64_t)batch * d->n_kv_heads * 4, 256);
+  w.l_off = w.m_off + round_up(rows * 4, 256);
   w.acc_off = w.l_off + round_up(rows * 4, 256);
   w.total = w.acc_off + rows * d->head_dim * 4;
   return w;
@@ -207,6 +210,49 @@ Plane plane_of(const kvq_cache_desc* d, int32_t batch, int which, void* base) {
   return p;
 }
 
+
+// Checks and fills the parameters of a decode launch (kvq_decode_attention and
+// kvq_decode_step); a plain decode appends nothing and writes partials only.
+kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void* v_cache, const void* q,
+                       int32_t batch, int64_t ctx_len, float softmax_scale, int32_t n_splits, void* workspace,
+                       size_t workspace_bytes, DecodeParams* out) {
+  kvq_status st = kvq_check_desc(d);
+  if (st != KVQ_OK) return st;
+  if (!k_cache || !v_cache || !q || !workspace) return KVQ_ERR_INVALID;
+  if (batch < 1 || batch > 65535 || ctx_len < 1 || ctx_len > d->max_ctx) return KVQ_ERR_INVALID;
+  if (n_splits < 0 || n_splits > kMaxSplits || !std::isfinite(softmax_scale)) return KVQ_ERR_INVALID;
+  if (!aligned(k_cache, 256) || !aligned(v_cache, 256) || !aligned(q, 16) || !aligned(workspace, 256))
+    return KVQ_ERR_INVALID;
+  const int32_t G = d->n_q_heads / d->n_kv_heads;
+  if (!decode_supported(d->k_type, d->v_type, G, d->head_dim)) return KVQ_ERR_UNSUPPORTED;
+  const int32_t S = resolve_splits(d, batch, ctx_len, n_splits);
+  const WsLayout w = ws_layout(d, batch, S);
+  if (workspace_bytes < (size_t)w.total) return KVQ_ERR_WORKSPACE;
+
+  DecodeParams& p = *out;
+  p = DecodeParams{};
+  p.k = plane_of(d, batch, 0, const_cast<void*>(k_cache));
+  p.v = plane_of(d, batch, 1, const_cast<void*>(v_cache));
+  p.q = static_cast<const __half*>(q);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.ws_m = reinterpret_cast<float*>(ws + w.m_off);
+  p.ws_l = reinterpret_cast<float*>(ws + w.l_off);
+  p.ws_acc = reinterpret_cast<float*>(ws + w.acc_off);
+  p.B = batch;
+  p.n_q = d->n_q_heads;
+  p.n_kv = d->n_kv_heads;
+  p.G = G;
+  p.D = d->head_dim;
+  p.S = S;
+  p.ctx = ctx_len;
+  p.chunk = chunk_rows(ctx_len, S);
+  p.qscale = softmax_scale * 1.4426950408889634f;
+  if (d->v_type == KVQ_TURBO3) p.t3 = turbo3_consts(d);
+  p.append_pos = -1;
+  p.out = nullptr;
+  p.counters = nullptr;
+  return KVQ_OK;
+}
 }  // namespace
 
 void set_last_cuda_error(cudaError_t e) { g_last_cuda_error = cudaGetErrorString(e); }
@@ -337,37 +383,39 @@ kvq_status kvq_append_quantize(const kvq_cache_desc* d, void* k_cache, void* v_c
 kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* k_cache, const void* v_cache, const void* q,
                                 int32_t batch, int64_t ctx_len, float softmax_scale, int32_t n_splits,
                                 void* workspace, size_t workspace_bytes, void* stream) {
-  kvq_status st = kvq_check_desc(d);
-  if (st != KVQ_OK) return st;
-  if (!k_cache || !v_cache || !q || !workspace) return KVQ_ERR_INVALID;
-  if (batch < 1 || batch > 65535 || ctx_len < 1 || ctx_len > d->max_ctx) return KVQ_ERR_INVALID;
-  if (n_splits < 0 || n_splits > kMaxSplits || !std::isfinite(softmax_scale)) return KVQ_ERR_INVALID;
-  if (!aligned(k_cache, 256) || !aligned(v_cache, 256) || !aligned(q, 16) || !aligned(workspace, 256))
-    return KVQ_ERR_INVALID;
-  const int32_t G = d->n_q_heads / d->n_kv_heads;
-  if (!decode_supported(d->k_type, d->v_type, G, d->head_dim)) return KVQ_ERR_UNSUPPORTED;
-  const int32_t S = resolve_splits(d, batch, ctx_len, n_splits);
-  const WsLayout w = ws_layout(d, batch, S);
-  if (workspace_bytes < (size_t)w.total) return KVQ_ERR_WORKSPACE;
-
   DecodeParams p{};
-  p.k = plane_of(d, batch, 0, const_cast<void*>(k_cache));
-  p.v = plane_of(d, batch, 1, const_cast<void*>(v_cache));
-  p.q = static_cast<const __half*>(q);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  p.ws_m = reinterpret_cast<float*>(ws + w.m_off);
-  p.ws_l = reinterpret_cast<float*>(ws + w.l_off);
-  p.ws_acc = reinterpret_cast<float*>(ws + w.acc_off);
-  p.B = batch;
-  p.n_q = d->n_q_heads;
-  p.n_kv = d->n_kv_heads;
-  p.G = G;
-  p.D = d->head_dim;
-  p.S = S;
-  p.ctx = ctx_len;
-  p.chunk = chunk_rows(ctx_len, S);
-  p.qscale = softmax_scale * 1.4426950408889634f;
-  if (d->v_type == KVQ_TURBO3) p.t3 = turbo3_consts(d);
+  const kvq_status st = fill_decode(d, k_cache, v_cache, q, batch, ctx_len, softmax_scale, n_splits, workspace,
+                                    workspace_bytes, &p);
+  if (st != KVQ_OK) return st;
+  const cudaError_t e = launch_decode(d->k_type, d->v_type, p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_step(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* q, const void* k_new,
+                           const void* v_new, int32_t batch, int64_t ctx_len, float softmax_scale, int32_t n_splits,
+                           void* workspace, size_t workspace_bytes, float* out, void* stream) {
+  if (!k_new || !v_new || !out) return KVQ_ERR_INVALID;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(out, 16)) return KVQ_ERR_INVALID;
+  DecodeParams p{};
+  const kvq_status st = fill_decode(d, k_cache, v_cache, q, batch, ctx_len, softmax_scale, n_splits, workspace,
+                                    workspace_bytes, &p);
+  if (st != KVQ_OK) return st;
+  const WsLayout w = ws_layout(d, batch, p.S);
+  p.append_pos = ctx_len - 1;
+  for (int which = 0; which < 2; ++which) {
+    AppendParams& a = which ? p.app_v : p.app_k;
+    a.src = static_cast<const __half*>(which ? v_new : k_new);
+    a.dst = which ? p.v : p.k;
+    a.B = batch;
+    a.H = d->n_kv_heads;
+    a.D = d->head_dim;
+    a.n_tok = 1;
+    a.pos = p.append_pos;
+    if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) a.t3 = turbo3_consts(d);
+  }
+  p.out = out;
+  p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + w.cnt_off);
   const cudaError_t e = launch_decode(d->k_type, d->v_type, p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return KVQ_OK;

@@ -47,7 +47,14 @@ struct DecodeParams {
   int32_t B, n_q, n_kv, G, D, S;
   int64_t ctx, chunk;
   float qscale;        // softmax_scale * log2(e)
-  Turbo3Consts t3;
+  Turbo3Consts t3;     // V sign bits and codebook (turbo3 values)
+  // Fused decode step (kvq_decode_step); a plain decode has append_pos < 0 and
+  // out == null.
+  int64_t append_pos;    // row the new K/V rows are written to first (< 0: none)
+  AppendParams app_k;    // that append: B = batch, H = n_kv, n_tok = 1
+  AppendParams app_v;
+  float* out;            // [B][n_q][D] combined output, or null (partials only)
+  uint32_t* counters;    // [B][n_kv] split arrival counters, zero between calls
 };
 
 struct CombineParams {

@@ -150,10 +150,12 @@ KVQ_API size_t kvq_cache_bytes(const kvq_cache_desc* desc, int32_t batch, int32_
  * (n_splits = 0 in kvq_decode_attention means this value); >= 1, or 0 on error. */
 KVQ_API int32_t kvq_auto_splits(const kvq_cache_desc* desc, int32_t batch, int64_t ctx_len);
 
-/* Workspace bytes kvq_decode_attention / kvq_combine need for n_splits
- * (0 = automatic, resolved as kvq_auto_splits would for ctx_len = max_ctx);
- * 0 on error.  Layout: m and l fp32 [batch][n_q][S] each, then acc fp32
- * [batch][n_q][S][head_dim], each part 256-byte aligned. */
+/* Workspace bytes kvq_decode_attention / kvq_combine / kvq_decode_step need
+ * for n_splits (0 = automatic, resolved as kvq_auto_splits would for ctx_len =
+ * max_ctx); 0 on error.  Layout: uint32 counters [batch][n_kv_heads] (used by
+ * kvq_decode_step only; their place does not depend on n_splits), then m and l
+ * fp32 [batch][n_q][S] each, then acc fp32 [batch][n_q][S][head_dim], each part
+ * 256-byte aligned. */
 KVQ_API size_t kvq_workspace_bytes(const kvq_cache_desc* desc, int32_t batch, int32_t n_splits);
 
 /* The turbo3 codebook this library uses: 8 binary32 levels (ascending) and
@@ -234,6 +236,30 @@ KVQ_API kvq_status kvq_decode_attention_noalloc(const kvq_cache_desc* desc, cons
                                                 const void* v_cache, const void* q, int32_t batch,
                                                 int64_t ctx_len, float softmax_scale, int32_t n_splits,
                                                 float* out, void* cuda_stream);
+
+/*
+ * Fused decode step: one launch that does what kvq_append_quantize (one new
+ * row per batch entry, at row ctx_len - 1), kvq_decode_attention (rows
+ * 0 .. ctx_len-1, the new row included) and kvq_combine do one after the
+ * other.  The pages have no such call: it is the decode loop's "append, then
+ * attend" (the CPY step before flash attention in the llama.cpp issue,
+ * "Possibly related") in one kernel, so a layer step costs one launch.
+ *   k_new, v_new   device fp16 [batch][n_kv_heads][head_dim], 16-byte aligned
+ *   out            device fp32 [batch][n_q_heads][head_dim], 16-byte aligned
+ *   other arguments as in kvq_decode_attention; ctx_len counts the new row.
+ * The CTA whose split holds row ctx_len - 1 writes the new rows before it reads
+ * any cache row; the last CTA of each (batch, KV head) to finish combines the
+ * group's splits.  The workspace counters (see kvq_workspace_bytes) must be zero
+ * before the first call with a workspace; every completed call leaves them
+ * zero.  Calls sharing a workspace must be ordered (one stream).
+ * Cached bytes are identical to kvq_append_quantize's; out agrees with
+ * kvq_decode_attention + kvq_combine up to fp32 rounding order.
+ */
+KVQ_API kvq_status kvq_decode_step(const kvq_cache_desc* desc, void* k_cache, void* v_cache,
+                                   const void* q, const void* k_new, const void* v_new,
+                                   int32_t batch, int64_t ctx_len, float softmax_scale,
+                                   int32_t n_splits, void* workspace, size_t workspace_bytes,
+                                   float* out, void* cuda_stream);
 
 #ifdef __cplusplus
 }

@@ -129,6 +129,12 @@ def _combine(desc, ws=FAKE, ws_bytes=1 << 40, batch=1, ctx=16, S=0, out=FAKE):
     return kvq.raw_status("kvq_combine", ctypes.byref(desc), ws, ws_bytes, batch, ctx, S, out, None)
 
 
+def _step(desc, k=FAKE, v=FAKE, q=FAKE, k_new=FAKE, v_new=FAKE, batch=1, ctx=16, scale=0.1, S=0, ws=FAKE,
+          ws_bytes=1 << 40, out=FAKE):
+    return kvq.raw_status("kvq_decode_step", ctypes.byref(desc), k, v, q, k_new, v_new, batch, ctx, scale, S, ws,
+                          ws_bytes, out, None)
+
+
 def test_append_rejects_before_launch():
     d = kvq.make_desc(8, 2, 64, "q8_0", "q4_0", 256)
     assert _append(d, pos=250, n_tok=7) == kvq.KVQ_ERR_INVALID     # past max_ctx
@@ -160,12 +166,28 @@ def test_decode_and_combine_reject_before_launch():
     assert _decode(kvq.make_desc(32, 8, 128, "turbo3", "q4_0", 64)) == kvq.KVQ_ERR_UNSUPPORTED
 
 
+def test_decode_step_rejects_before_launch():
+    d = kvq.make_desc(32, 8, 128, "q8_0", "q4_0", 8192)
+    assert _step(d, k_new=None) == kvq.KVQ_ERR_INVALID
+    assert _step(d, v_new=None) == kvq.KVQ_ERR_INVALID
+    assert _step(d, out=None) == kvq.KVQ_ERR_INVALID
+    assert _step(d, k_new=FAKE + 2) == kvq.KVQ_ERR_INVALID         # new rows not 16-aligned
+    assert _step(d, out=FAKE + 4) == kvq.KVQ_ERR_INVALID
+    assert _step(d, ctx=0) == kvq.KVQ_ERR_INVALID                  # the new row needs ctx_len >= 1
+    assert _step(d, ctx=8193) == kvq.KVQ_ERR_INVALID
+    assert _step(d, k=FAKE + 16) == kvq.KVQ_ERR_INVALID
+    need = kvq.kvq_workspace_bytes(d, 1, 4)
+    assert _step(d, S=4, ws_bytes=need - 1) == kvq.KVQ_ERR_WORKSPACE  # the counters are part of it
+    assert _step(kvq.make_desc(32, 8, 128, "turbo3", "q4_0", 64)) == kvq.KVQ_ERR_UNSUPPORTED
+
+
 def test_workspace_bytes_formula():
     d = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 32768)
     B, S = 4, 9
     rows = B * 64 * S
     r256 = lambda v: (v + 255) // 256 * 256
-    assert kvq.kvq_workspace_bytes(d, B, S) == 2 * r256(rows * 4) + rows * 128 * 4
+    # the fused step's counters [B][n_kv] (uint32), then m, l, acc, each part 256-aligned
+    assert kvq.kvq_workspace_bytes(d, B, S) == r256(B * 8 * 4) + 2 * r256(rows * 4) + rows * 128 * 4
     assert kvq.kvq_workspace_bytes(d, 0, S) == 0
     # the automatic split count never needs more workspace than n_splits = 0 reserves
     auto_ws = kvq.kvq_workspace_bytes(d, B, 0)
