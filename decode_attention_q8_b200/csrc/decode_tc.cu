@@ -105,7 +105,27 @@ bool decode_supported(int32_t k_type, int32_t v_type, int32_t G, int32_t D) {
   return true;
 }
 
-int decode_ctas_per_sm() { return 2; }
+namespace {
+template <int KT>
+int ctas_k(int32_t v_type, int32_t D) {
+  switch (v_type) {
+    case KVQ_F16: return tc::ctas_per_sm_for(KT, KVQ_F16, D);
+    case KVQ_Q8_0: return tc::ctas_per_sm_for(KT, KVQ_Q8_0, D);
+    case KVQ_Q4_0: return tc::ctas_per_sm_for(KT, KVQ_Q4_0, D);
+    case KVQ_TURBO3: return tc::ctas_per_sm_for(KT, KVQ_TURBO3, D);
+  }
+  return 1;
+}
+}  // namespace
+
+int decode_ctas_per_sm(int32_t k_type, int32_t v_type, int32_t D) {
+  switch (k_type) {
+    case KVQ_F16: return ctas_k<KVQ_F16>(v_type, D);
+    case KVQ_Q8_0: return ctas_k<KVQ_Q8_0>(v_type, D);
+    case KVQ_Q4_0: return ctas_k<KVQ_Q4_0>(v_type, D);
+  }
+  return 1;
+}
 
 
 cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p, cudaStream_t st) {

@@ -84,14 +84,32 @@ __host__ __device__ constexpr int stage_bytes(int kt, int vt, int d) {
          round_up_c(kSub * code_bytes(vt, d), vt == KVQ_TURBO3 ? 128 : 1024) +
          round_up_c(kSub * n_scales(kt, d) * 2, 128) + round_up_c(kSub * n_scales(vt, d) * 2, 128);
 }
-// Warps per CTA: 8 while two 2-stage rings per warp fit in ~110 KB (two CTAs per
-// SM), else 4 (one CTA per SM).  Stages per warp ring: up to 4, as many as fit.
+// Shared memory of one CTA: the 1024-byte alignment pad, one ring of `stages`
+// stages per warp (rounded to the 1024-byte swizzle atom), the turbo3 pair
+// table, the ring barriers and a few bytes of slack.
+__host__ __device__ constexpr int cta_smem(int kt, int vt, int d, int nw, int stages) {
+  return 1024 + nw * round_up_c(stages * stage_bytes(kt, vt, d), 1024) + (vt == KVQ_TURBO3 ? 64 * 32 * 4 : 0) +
+         nw * stages * 8 + 16;
+}
+// An SM has 228 KB of shared memory and reserves 1 KB per resident CTA; the
+// kernel's static shared variables take a few bytes more.
+constexpr int kSmemTwoCtas = 228 * 1024 / 2 - 1024 - 64;  // per CTA, two CTAs per SM
+constexpr int kSmemOneCta = 227 * 1024 - 64;               // per CTA, one CTA per SM
+// Warps per CTA: 8 while 8 two-stage rings leave room for a second CTA on the
+// SM, else 4.  Stages per warp ring: as many (2 to 4) as keep the CTA count
+// per SM (two if two fit at 2 stages, else one).
 __host__ __device__ constexpr int warps_for(int kt, int vt, int d) {
-  return kNWMax * 2 * stage_bytes(kt, vt, d) <= 112640 ? kNWMax : kNWMax / 2;
+  return cta_smem(kt, vt, d, kNWMax, 2) <= kSmemTwoCtas ? kNWMax : kNWMax / 2;
+}
+__host__ __device__ constexpr int ctas_per_sm_for(int kt, int vt, int d) {
+  return cta_smem(kt, vt, d, warps_for(kt, vt, d), 2) <= kSmemTwoCtas ? 2 : 1;
 }
 __host__ __device__ constexpr int stages_for(int kt, int vt, int d) {
-  return (112640 / (warps_for(kt, vt, d) * stage_bytes(kt, vt, d))) >= 4 ? 4
-         : (112640 / (warps_for(kt, vt, d) * stage_bytes(kt, vt, d))) >= 3 ? 3 : 2;
+  return cta_smem(kt, vt, d, warps_for(kt, vt, d), 4) <= (ctas_per_sm_for(kt, vt, d) == 2 ? kSmemTwoCtas : kSmemOneCta)
+             ? 4
+         : cta_smem(kt, vt, d, warps_for(kt, vt, d), 3) <= (ctas_per_sm_for(kt, vt, d) == 2 ? kSmemTwoCtas : kSmemOneCta)
+             ? 3
+             : 2;
 }
 
 template <int KT, int VT, int D>
@@ -112,6 +130,7 @@ struct Layout {
   // CTA-level merge scratch (reuses the stage memory after the main loop)
   static constexpr int MERGE = NW * ((D / 16) * 32 * 4 + 16) * 4;  // fragment chunks + m, l per warp
   static constexpr int TOTAL = 1024 + NW * WARP + TABLE + BARS + 16;
+  static_assert(TOTAL == cta_smem(KT, VT, D, NW, kStages), "layout and budget agree");
   static_assert(MERGE <= NW * WARP, "merge area must fit in the stage memory");
   static_assert(TOTAL <= 227 * 1024, "shared memory per CTA");
 };
@@ -293,7 +312,7 @@ struct TcArgs {
 
 template <int KT, int VT, int NB, int NTH>
 __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
-                                  (NB >= 8 || NTH == 2 || warps_for(KT, VT, NB * 32) < kNWMax) ? 1 : 2)
+                                  (NB >= 8 || NTH == 2 || ctas_per_sm_for(KT, VT, NB * 32) < 2) ? 1 : 2)
     decode_tc_kernel(const TcArgs args, const __grid_constant__ CUtensorMap tm_kc,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vc,
                      const __grid_constant__ CUtensorMap tm_vs) {

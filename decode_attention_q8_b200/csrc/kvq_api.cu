@@ -169,7 +169,8 @@ int64_t chunk_rows(int64_t ctx, int32_t S) { return round_up((ctx + S - 1) / S, 
 // Upper bound of the automatic split count over ctx_len <= ctx (sizes the
 // workspace for n_splits = 0).
 int32_t auto_splits_bound(const kvq_cache_desc* d, int32_t batch, int64_t ctx) {
-  return choose_splits((int64_t)batch * d->n_kv_heads, ctx, sm_count(), decode_ctas_per_sm());
+  return choose_splits((int64_t)batch * d->n_kv_heads, ctx, sm_count(),
+                       decode_ctas_per_sm(d->k_type, d->v_type, d->head_dim));
 }
 
 // Explicit counts are used as given (trailing splits may be empty); the
