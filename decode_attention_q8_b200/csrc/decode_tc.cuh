@@ -52,7 +52,8 @@
 //        one more MMA per 16 rows whose A operand is the block-scale matrix
 //        (m = block, k = row); it and the 2^24 are taken out once at the end.
 //        turbo3 codes become codebook levels through a per-lane replicated
-//        64-entry pair table.
+//        64-entry table of one row's two consecutive dims, paired across rows
+//        by a byte permute.
 //   turbo3 values accumulate in the rotated domain; kvq_combine rotates back.
 #pragma once
 
@@ -351,7 +352,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     fence_barrier_init();
   }
   if (VT == KVQ_TURBO3) {
-    // table[idx6 * 32 + lane] = half2(c[idx6 & 7], c[idx6 >> 3]); one copy per bank
+    // table[x * 32 + lane] = half2(c[x & 7], c[x >> 3]) for a 6-bit code pair x; one copy per bank
     for (int e = threadIdx.x; e < 64 * 32; e += L::NW * 32) {
       const int idx = e >> 5;
       table[e] = pack_half2(p.t3.levels[idx & 7], p.t3.levels[idx >> 3]);
@@ -662,18 +663,23 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           pbw[nt][1] &= pmask_hi;
         }
       }
+      // table[x * 32 + lane] = half2(c[x & 7], c[x >> 3]): the levels of one
+      // row's two consecutive dims; a byte permute pairs rows 2c and 2c+1
+      const uint32_t* tl = table + lane;
       if (D <= 128) {
         const unsigned long long fA = field(2 * c), fB = field(2 * c + 1);
         const unsigned long long fC = field(2 * c + 8), fD = field(2 * c + 9);
 #pragma unroll
         for (int mt = 0; mt < NMT; ++mt) {
-          const uint32_t xA = (uint32_t)(fA >> (6 * mt)) & 63u, xB = (uint32_t)(fB >> (6 * mt)) & 63u;
-          const uint32_t xC = (uint32_t)(fC >> (6 * mt)) & 63u, xD = (uint32_t)(fD >> (6 * mt)) & 63u;
+          const uint32_t tA = tl[((uint32_t)(fA >> (6 * mt)) & 63u) << 5];
+          const uint32_t tB = tl[((uint32_t)(fB >> (6 * mt)) & 63u) << 5];
+          const uint32_t tC = tl[((uint32_t)(fC >> (6 * mt)) & 63u) << 5];
+          const uint32_t tD = tl[((uint32_t)(fD >> (6 * mt)) & 63u) << 5];
           uint32_t a[4];
-          a[0] = table[(((xA & 7u) | ((xB & 7u) << 3)) << 5) + lane];
-          a[1] = table[(((xA >> 3) | (xB & 0x38u)) << 5) + lane];
-          a[2] = table[(((xC & 7u) | ((xD & 7u) << 3)) << 5) + lane];
-          a[3] = table[(((xC >> 3) | (xD & 0x38u)) << 5) + lane];
+          a[0] = prmt(tA, tB, 0x5410);  // dim 2mt:   rows 2c, 2c+1
+          a[1] = prmt(tA, tB, 0x7632);  // dim 2mt+1
+          a[2] = prmt(tC, tD, 0x5410);  // dim 2mt:   rows 2c+8, 2c+9
+          a[3] = prmt(tC, tD, 0x7632);
 #pragma unroll
           for (int nt = 0; nt < NTH; ++nt)
             mma16816(acc[nt][mt], a[0], a[1], a[2], a[3], pbw[nt][0], pbw[nt][1], acc[nt][mt]);
@@ -694,13 +700,15 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const int mt = half * 8 + k;
-            const uint32_t xA = (uint32_t)(fA >> (6 * k)) & 63u, xB = (uint32_t)(fB >> (6 * k)) & 63u;
-            const uint32_t xC = (uint32_t)(fC >> (6 * k)) & 63u, xD = (uint32_t)(fD >> (6 * k)) & 63u;
+            const uint32_t tA = tl[((uint32_t)(fA >> (6 * k)) & 63u) << 5];
+            const uint32_t tB = tl[((uint32_t)(fB >> (6 * k)) & 63u) << 5];
+            const uint32_t tC = tl[((uint32_t)(fC >> (6 * k)) & 63u) << 5];
+            const uint32_t tD = tl[((uint32_t)(fD >> (6 * k)) & 63u) << 5];
             uint32_t a[4];
-            a[0] = table[(((xA & 7u) | ((xB & 7u) << 3)) << 5) + lane];
-            a[1] = table[(((xA >> 3) | (xB & 0x38u)) << 5) + lane];
-            a[2] = table[(((xC & 7u) | ((xD & 7u) << 3)) << 5) + lane];
-            a[3] = table[(((xC >> 3) | (xD & 0x38u)) << 5) + lane];
+            a[0] = prmt(tA, tB, 0x5410);
+            a[1] = prmt(tA, tB, 0x7632);
+            a[2] = prmt(tC, tD, 0x5410);
+            a[3] = prmt(tC, tD, 0x7632);
 #pragma unroll
             for (int nt = 0; nt < NTH; ++nt)
               mma16816(acc[nt][mt], a[0], a[1], a[2], a[3], pbw[nt][0], pbw[nt][1], acc[nt][mt]);
