@@ -411,25 +411,31 @@ def run_kvq(args):
     unfused_ms = u0.elapsed_time(u1)
     del ugraph
 
-    # ---- end to end through the public API with host buffers: every layer's
-    #      query and new K/V rows copied in from pinned host memory, every
-    #      layer's output copied back, all inside the timed region
-    q_h = [x.cpu().pin_memory() for x in qs]
-    kn_h = [x.cpu().pin_memory() for x in kn]
-    vn_h = [x.cpu().pin_memory() for x in vn]
-    out_h = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
-    qd = [torch.empty_like(x) for x in qs]
-    knd = [torch.empty_like(x) for x in kn]
-    vnd = [torch.empty_like(x) for x in vn]
+    # ---- end to end through the public API with host buffers: the step's
+    #      inputs (every layer's query and new K/V rows) copied in from pinned
+    #      host memory in one transfer, every layer's output copied back in
+    #      one, all inside the timed region
+    n_q_el, n_k_el = qs[0].numel(), kn[0].numel()
+    per_layer = n_q_el + 2 * n_k_el
+    in_h = torch.empty(L * per_layer, dtype=torch.float16).pin_memory()
+    for layer in range(L):
+        base = layer * per_layer
+        in_h[base:base + n_q_el] = qs[layer].reshape(-1).cpu()
+        in_h[base + n_q_el:base + n_q_el + n_k_el] = kn[layer].reshape(-1).cpu()
+        in_h[base + n_q_el + n_k_el:base + per_layer] = vn[layer].reshape(-1).cpu()
+    in_d = torch.empty_like(in_h, device=dev)
+    out_d = torch.empty((L,) + tuple(outs[0].shape), dtype=torch.float32, device=dev)
+    out_h = torch.empty_like(out_d, device="cpu").pin_memory()
+    qd = [in_d[l * per_layer:l * per_layer + n_q_el].view(qs[0].shape) for l in range(L)]
+    knd = [in_d[l * per_layer + n_q_el:l * per_layer + n_q_el + n_k_el].view(kn[0].shape) for l in range(L)]
+    vnd = [in_d[l * per_layer + n_q_el + n_k_el:(l + 1) * per_layer].view(vn[0].shape) for l in range(L)]
 
     def e2e_step():
+        in_d.copy_(in_h, non_blocking=True)
         for layer in range(L):
-            qd[layer].copy_(q_h[layer], non_blocking=True)
-            knd[layer].copy_(kn_h[layer], non_blocking=True)
-            vnd[layer].copy_(vn_h[layer], non_blocking=True)
             kvq.kvq_decode_step(desc, kcs[layer], vcs[layer], qd[layer], knd[layer], vnd[layer], B, ctx, scale, 0,
-                                ws, outs[layer])
-            out_h[layer].copy_(outs[layer], non_blocking=True)
+                                ws, out_d[layer])
+        out_h.copy_(out_d, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -486,8 +492,8 @@ def run_kvq(args):
                          "avg_launch_us": round(dec_avg * 1e3, 3),
                          "launch_us_between_event_nodes": None if ev_ms != ev_ms else round(ev_ms * 1e3, 3)},
             "e2e": {"value": round(e2e_value, 3), "unit": UNIT,
-                    "h2d_bytes_per_step": L * (qs[0].numel() * 2 + kn[0].numel() * 2 + vn[0].numel() * 2),
-                    "d2h_bytes_per_step": L * outs[0].numel() * 4},
+                    "h2d_bytes_per_step": in_h.numel() * in_h.element_size(),
+                    "d2h_bytes_per_step": out_h.numel() * out_h.element_size()},
             "gpu_launches": args.steps * L,
             "step_unfused_us_per_layer": round(1e3 * unfused_ms / args.steps / L, 3),
             "timing": "CUDA-graph replays of whole steps (no event nodes); avg launch = timed region / launches",
