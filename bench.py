@@ -134,10 +134,20 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def _sample_now(self):
+        if self._thread is not None:
+            try:
+                sm, reasons = self._query()
+                self.samples.append((time.perf_counter(), sm, reasons))
+            except Exception:
+                pass
+
     def begin(self):
         self.window[0] = time.perf_counter()
+        self._sample_now()  # a short timed region still gets samples at its ends
 
     def end(self):
+        self._sample_now()
         self.window[1] = time.perf_counter()
 
     def stop(self):
