@@ -1,34 +1,113 @@
 // Quantize-on-append kernel: fp16 K/V rows -> f16 / q8_0 / q4_0 / turbo3 cache
 // rows, K and V of one call in one launch.  The row bodies (formats, rounding,
 // work mapping) are in append_rows.cuh.
+#include <algorithm>
+
 #include "append_rows.cuh"
 
 namespace kvq {
 namespace {
 
 constexpr int kAppendThreads = 256;
+constexpr int kAppendRound = 4;  // work items per thread and round: loads in flight
+constexpr int kBlockRound = 1;   // q8_0 / q4_0 blocks per thread and round (a block is 4 loads)
 
-// CTAs a tensor of `type` needs (each CTA: 256 threads).
-int64_t append_ctas(int32_t type, const AppendParams& p) {
-  const int64_t rows = (int64_t)p.B * p.n_tok * p.H;
-  const int64_t threads = rows * rows::row_threads(type, p.D);
-  return (threads + kAppendThreads - 1) / kAppendThreads;
+// Work items of one row in this kernel: a 32-element block for q8_0 / q4_0,
+// otherwise the row bodies' threads.
+__host__ __device__ constexpr int bulk_items(int32_t type, int d) {
+  return type == KVQ_Q8_0 || type == KVQ_Q4_0 ? d / kBlock : rows::row_threads(type, d);
 }
 
-// K and V rows of one append call in one launch: CTAs [0, ctas0) quantize the
-// first tensor, the rest the second; the branch on the type is uniform per CTA.
+// K and V rows of one append call in one launch.  Every CTA takes its share of
+// the first tensor's rows, then of the second's (the branch on the type is
+// uniform per CTA), so the two parts stay balanced whatever their cost.  Each
+// part runs grid-stride over its flat work: a thread loads several items
+// (stride apart) before it quantizes and stores them, so a grid of one
+// resident wave keeps enough reads in flight to stream at HBM rates.  Strides
+// are multiples of 32, so each lane keeps its place in the 8-lane block groups
+// and the warps of the shuffles stay whole.
 struct AppendPair {
   AppendParams p[2];
   int32_t type[2];
-  int64_t ctas0;
+  int32_t n;  // tensors in the call (1 or 2)
 };
 
+template <int TYPE, int E>
+__device__ __forceinline__ void append_stream(const AppendParams& p, int64_t first, int64_t stride, int64_t gend) {
+  for (int64_t base = first; (base & ~(int64_t)31) < gend; base += kAppendRound * stride) {
+    uint4 raw[kAppendRound];
+#pragma unroll
+    for (int u = 0; u < kAppendRound; ++u) raw[u] = rows::load_raw<TYPE, E>(p, base + u * stride, gend);
+#pragma unroll
+    for (int u = 0; u < kAppendRound; ++u) {
+      const int64_t g = base + u * stride;
+      if ((g & ~(int64_t)31) < gend) rows::finish<TYPE, E>(p, g, gend, raw[u]);  // warp-uniform
+    }
+  }
+}
+
+// q8_0 / q4_0: one thread per 32-element block; kBlockRound blocks (four
+// 16-byte loads each) in flight per thread.  One block per round measured
+// fastest: the smaller body keeps the instruction cache warm and the
+// registers at 64 (four CTAs per SM).
+template <int TYPE>
+__device__ __forceinline__ void append_blocks(const AppendParams& p, int64_t first, int64_t stride, int64_t nblk) {
+  for (int64_t base = first; base < nblk; base += kBlockRound * stride) {
+    rows::BlockRaw raw[kBlockRound];
+#pragma unroll
+    for (int u = 0; u < kBlockRound; ++u) raw[u] = rows::load_block(p, base + u * stride, nblk);
+#pragma unroll
+    for (int u = 0; u < kBlockRound; ++u) {
+      const int64_t g = base + u * stride;
+      if (g < nblk) {
+        if constexpr (TYPE == KVQ_Q8_0) rows::q8_0_block(p, g, raw[u]);
+        else rows::q4_0_block(p, g, raw[u]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void append_part(const AppendParams& p, int32_t type, int64_t first, int64_t stride) {
+  const int64_t gend = (int64_t)p.B * p.n_tok * p.H * bulk_items(type, p.D);
+  switch (type) {
+    case KVQ_F16: append_stream<KVQ_F16, 0>(p, first, stride, gend); break;
+    case KVQ_Q8_0: append_blocks<KVQ_Q8_0>(p, first, stride, gend); break;
+    case KVQ_Q4_0: append_blocks<KVQ_Q4_0>(p, first, stride, gend); break;
+    case KVQ_TURBO3:
+      switch (p.D) {
+        case 32: append_stream<KVQ_TURBO3, 1>(p, first, stride, gend); break;
+        case 64: append_stream<KVQ_TURBO3, 2>(p, first, stride, gend); break;
+        case 128: append_stream<KVQ_TURBO3, 4>(p, first, stride, gend); break;
+        case 256: append_stream<KVQ_TURBO3, 8>(p, first, stride, gend); break;
+      }
+      break;
+  }
+}
+
 __global__ void __launch_bounds__(kAppendThreads) append_pair_kernel(const AppendPair pp) {
-  const int which = (int64_t)blockIdx.x < pp.ctas0 ? 0 : 1;
-  const int64_t cta = which ? (int64_t)blockIdx.x - pp.ctas0 : (int64_t)blockIdx.x;
-  const AppendParams& p = pp.p[which];
-  const int64_t gend = (int64_t)p.B * p.n_tok * p.H * rows::row_threads(pp.type[which], p.D);
-  rows::append_any(pp.type[which], p, cta * blockDim.x + threadIdx.x, gend);
+  const int64_t first = (int64_t)blockIdx.x * kAppendThreads + threadIdx.x;
+  const int64_t stride = (int64_t)gridDim.x * kAppendThreads;
+  append_part(pp.p[0], pp.type[0], first, stride);
+  if (pp.n == 2) append_part(pp.p[1], pp.type[1], first, stride);
+}
+
+// Resident 256-thread CTAs of the append kernel on the whole current device
+// (one wave); 148 SMs x 4 if the device cannot be asked.
+int64_t resident_ctas() {
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, append_pair_kernel, kAppendThreads, 0) != cudaSuccess ||
+      sms <= 0 || per_sm <= 0) {
+    (void)cudaGetLastError();
+    return 148 * 4;
+  }
+  return (int64_t)sms * per_sm;
+}
+
+// CTAs the work of a tensor needs (one item per thread).
+int64_t append_ctas(int32_t type, const AppendParams& p) {
+  const int64_t threads = (int64_t)p.B * p.n_tok * p.H * bulk_items(type, p.D);
+  return (threads + kAppendThreads - 1) / kAppendThreads;
 }
 
 }  // namespace
@@ -37,23 +116,21 @@ cudaError_t launch_append(const AppendParams* k, int32_t k_type, const AppendPar
                           cudaStream_t st) {
   AppendPair pp{};
   int n = 0;
-  int64_t ctas[2] = {0, 0};
-  if (k) {
-    pp.p[n] = *k;
-    pp.type[n] = k_type;
-    ctas[n++] = append_ctas(k_type, *k);
-  }
-  if (v) {
-    pp.p[n] = *v;
-    pp.type[n] = v_type;
-    ctas[n++] = append_ctas(v_type, *v);
+  const AppendParams* ps[2] = {k, v};
+  const int32_t ts[2] = {k_type, v_type};
+  for (int i = 0; i < 2; ++i) {
+    if (!ps[i]) continue;
+    pp.p[n] = *ps[i];
+    pp.type[n] = ts[i];
+    ++n;
   }
   if (n == 0) return cudaSuccess;
-  if (n == 1) ctas[1] = 0;
-  pp.ctas0 = ctas[0];
-  const int64_t total = ctas[0] + ctas[1];
-  if (total <= 0 || total > 0x7fffffff) return cudaErrorInvalidValue;
-  append_pair_kernel<<<(unsigned)total, kAppendThreads, 0, st>>>(pp);
+  pp.n = n;
+  int64_t need = append_ctas(pp.type[0], pp.p[0]);
+  if (n == 2) need = std::max(need, append_ctas(pp.type[1], pp.p[1]));
+  const int64_t ctas = std::min(need, resident_ctas());
+  if (ctas <= 0) return cudaSuccess;  // no rows
+  append_pair_kernel<<<(unsigned)ctas, kAppendThreads, 0, st>>>(pp);
   return cudaGetLastError();
 }
 

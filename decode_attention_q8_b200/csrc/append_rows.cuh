@@ -15,7 +15,8 @@
 // warps share a gtid range aligned to 32): q8_0 / q4_0 give each 32-element
 // block to 8 consecutive threads holding 4 contiguous elements each (one 8-byte
 // load per thread; the block max is a 3-step xor-shuffle reduction inside the 8
-// lanes).  turbo3 gives each row to one warp, D/32 contiguous elements per lane;
+// lanes).  Loading (load_raw) and quantizing (finish) are separate steps, so a
+// thread can have several loads in flight.  turbo3 gives each row to one warp, D/32 contiguous elements per lane;
 // the Walsh-Hadamard butterflies run in registers for strides below D/32 and
 // as xor-shuffles above.  Threads past the work still take part in the
 // shuffles and then return.
@@ -26,46 +27,98 @@
 namespace kvq {
 namespace rows {
 
-__device__ __forceinline__ void load4_f16(const __half* src, float x[4]) {
-  uint2 raw = __ldg(reinterpret_cast<const uint2*>(src));
-  __half2 a = *reinterpret_cast<__half2*>(&raw.x);
-  __half2 b = *reinterpret_cast<__half2*>(&raw.y);
-  x[0] = __low2float(a);
-  x[1] = __high2float(a);
-  x[2] = __low2float(b);
-  x[3] = __high2float(b);
+// The fp16 input bytes thread gtid of a call's flat work needs (zero past
+// gend): q8_0 / q4_0 4 elements (8 bytes), f16 8 elements (16 bytes), turbo3
+// D/32 elements.  Work item gtid's elements start at element 4, 8 or D/32 times
+// gtid of the call's [rows][D] input.
+template <int TYPE, int E>
+__device__ __forceinline__ uint4 load_raw(const AppendParams& p, int64_t gtid, int64_t gend) {
+  uint4 r = make_uint4(0u, 0u, 0u, 0u);
+  if (gtid >= gend) return r;
+  if constexpr (TYPE == KVQ_Q8_0 || TYPE == KVQ_Q4_0) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.src + gtid * 4));
+    r.x = v.x;
+    r.y = v.y;
+  } else if constexpr (TYPE == KVQ_F16) {
+    r = __ldg(reinterpret_cast<const uint4*>(p.src + gtid * 8));
+  } else {  // turbo3
+    if constexpr (E == 8) {
+      r = __ldg(reinterpret_cast<const uint4*>(p.src + gtid * 8));
+    } else if constexpr (E == 4) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.src + gtid * 4));
+      r.x = v.x;
+      r.y = v.y;
+    } else if constexpr (E == 2) {
+      r.x = __ldg(reinterpret_cast<const unsigned int*>(p.src + gtid * 2));
+    } else {
+      r.x = __ldg(reinterpret_cast<const unsigned short*>(p.src + gtid));
+    }
+  }
+  return r;
+}
+
+__device__ __forceinline__ float raw_elem(const uint4& r, int i) {  // fp16 element i of r as float
+  const uint32_t w = i < 2 ? r.x : i < 4 ? r.y : i < 6 ? r.z : r.w;
+  const uint16_t h = (uint16_t)(w >> (16 * (i & 1)));
+  return __half2float(__ushort_as_half(h));
 }
 
 // Destination row index of flat input row `row` = ((b * n_tok + t) * H + h).
+// 32-bit division when the call's rows fit (the 64-bit one is a long routine).
 __device__ __forceinline__ int64_t dst_row(const AppendParams& p, int64_t row) {
-  int64_t h = row % p.H;
-  int64_t t = (row / p.H) % p.n_tok;
-  int64_t b = row / ((int64_t)p.H * p.n_tok);
+  int64_t h, t, b;
+  if ((int64_t)p.B * p.n_tok * p.H <= 0xffffffffll) {
+    const uint64_t r32 = (uint64_t)(uint32_t)row;
+    const uint64_t bt = p.h_mul ? __umul64hi(r32, p.h_mul) : r32;
+    h = (int64_t)(r32 - bt * (uint64_t)p.H);
+    b = (int64_t)(p.t_mul ? __umul64hi(bt, p.t_mul) : bt);
+    t = (int64_t)bt - b * p.n_tok;
+  } else {
+    h = row % p.H;
+    t = (row / p.H) % p.n_tok;
+    b = row / ((int64_t)p.H * p.n_tok);
+  }
   return (b * p.H + h) * p.dst.T + p.pos + t;
 }
 
+// log2 of the 32-element blocks per row (head_dim is 32 times a power of two)
+__device__ __forceinline__ int log2_blocks(const AppendParams& p) { return 31 - __clz(p.D / kBlock); }
+
 // q8_0: d = amax/127; q = roundf(x / d) (IEEE divide per element); d == 0 -> 0.
-__device__ __forceinline__ void append_q8_0(const AppendParams& p, int64_t gtid, int64_t gend) {
+__device__ __forceinline__ void append_q8_0(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
   const int nb = p.D / kBlock;
   const int64_t gblk = gtid >> 3;
   const int sub = (int)(gtid & 7);
   const bool active = gtid < gend;
-  float x[4] = {0.f, 0.f, 0.f, 0.f};
-  if (active) load4_f16(p.src + gblk * kBlock + sub * 4, x);
+  float x[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) x[i] = raw_elem(raw, i);  // zeros past gend
   float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
   for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if (!active) return;
   const float d = __fdiv_rn(amax, 127.0f);
+  // q = roundf of the IEEE quotient x / d.  x * fl(1/d) is within 2^-15 of that
+  // quotient (|x / d| <= 127, two roundings of 2^-24 relative), so it rounds to
+  // the same integer unless it lies within 2^-14 of a half-integer; only then
+  // is the exact divide taken.  Away from a tie round-to-nearest is roundf.
+  const float rd = d != 0.0f ? __frcp_rn(d) : 0.0f;
   uint32_t packed = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     int q = 0;
-    if (d != 0.0f) q = (int)roundf(__fdiv_rn(x[i], d));
+    if (d != 0.0f) {
+      const float t = __fmul_rn(x[i], rd);
+      const float a = fabsf(t);
+      if (fabsf(a - floorf(a) - 0.5f) > 6.103515625e-05f)  // 2^-14
+        q = __float2int_rn(t);
+      else
+        q = (int)roundf(__fdiv_rn(x[i], d));
+    }
     packed |= (uint32_t)(q & 0xFF) << (8 * i);
   }
-  const int64_t row = gblk / nb;
-  const int blk = (int)(gblk % nb);
+  const int64_t row = gblk >> log2_blocks(p);
+  const int blk = (int)(gblk & (nb - 1));
   const int64_t r = dst_row(p, row);
   *reinterpret_cast<uint32_t*>(p.dst.codes + r * p.dst.code_bytes + blk * kBlock + sub * 4) = packed;
   if (sub == 0) p.dst.scales[r * p.dst.n_scales + blk] = __float2half_rn(d);
@@ -73,13 +126,14 @@ __device__ __forceinline__ void append_q8_0(const AppendParams& p, int64_t gtid,
 
 // q4_0: m = signed max-magnitude element (lowest index on ties); d = m / -8;
 // q = min(15, trunc(fl(fl(x * fl(1/d)) + 8.5))); byte j = q_j | q_{j+16} << 4.
-__device__ __forceinline__ void append_q4_0(const AppendParams& p, int64_t gtid, int64_t gend) {
+__device__ __forceinline__ void append_q4_0(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
   const int nb = p.D / kBlock;
   const int64_t gblk = gtid >> 3;
   const int sub = (int)(gtid & 7);
   const bool active = gtid < gend;
-  float x[4] = {0.f, 0.f, 0.f, 0.f};
-  if (active) load4_f16(p.src + gblk * kBlock + sub * 4, x);
+  float x[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) x[i] = raw_elem(raw, i);  // zeros past gend
   // local best: largest |x|, first index on ties
   float bm = x[0];
   int bi = sub * 4;
@@ -106,38 +160,160 @@ __device__ __forceinline__ void append_q4_0(const AppendParams& p, int64_t gtid,
   const uint32_t hi = __shfl_xor_sync(0xffffffffu, nib, 4);
   if (!active || sub >= 4) return;
   const uint32_t bytes = nib | (hi << 4);
-  const int64_t row = gblk / nb;
-  const int blk = (int)(gblk % nb);
+  const int64_t row = gblk >> log2_blocks(p);
+  const int blk = (int)(gblk & (nb - 1));
   const int64_t r = dst_row(p, row);
   *reinterpret_cast<uint32_t*>(p.dst.codes + r * p.dst.code_bytes + blk * 16 + sub * 4) = bytes;
   if (sub == 0) p.dst.scales[r * p.dst.n_scales + blk] = __float2half_rn(d);
 }
 
+// ---- Bulk mapping for q8_0 / q4_0: one thread per 32-element block ----------
+// The 8-lane bodies above keep the latency of one row low (the fused decode
+// step appends one row per KV head).  Many rows at once are bound by
+// instruction issue instead, so the bulk append gives a whole block to one
+// thread: four 16-byte loads, no shuffles, and the block's scale, divide and
+// index math paid once per 32 elements.  The arithmetic is the same as above,
+// so the stored bytes are identical.
+
+struct BlockRaw {
+  uint4 w[4];  // the block's 32 fp16 inputs, two per word
+};
+
+// Block gblk of the call's [rows][D] input (zeros past nblk).
+__device__ __forceinline__ BlockRaw load_block(const AppendParams& p, int64_t gblk, int64_t nblk) {
+  BlockRaw r;
+  if (gblk < nblk) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.src + gblk * kBlock);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) r.w[j] = __ldg(src + j);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) r.w[j] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  return r;
+}
+
+__device__ __forceinline__ float block_elem(const BlockRaw& r, int i) {  // element i (0..31) as float
+  const uint4& v = r.w[i >> 3];
+  const int k = (i >> 1) & 3;
+  const uint32_t w = k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
+  return __half2float(__ushort_as_half((uint16_t)(w >> (16 * (i & 1)))));
+}
+
+__device__ __forceinline__ __half2 block_pair(const BlockRaw& r, int k) {  // elements 2k, 2k+1
+  const uint4& v = r.w[k >> 2];
+  const int c = k & 3;
+  const uint32_t w = c == 0 ? v.x : c == 1 ? v.y : c == 2 ? v.z : v.w;
+  return *reinterpret_cast<const __half2*>(&w);
+}
+
+// Where block gblk's row lands in the cache, and the block's index in its row.
+__device__ __forceinline__ void block_dst(const AppendParams& p, int64_t gblk, int64_t& r, int& blk) {
+  const int lb = log2_blocks(p);
+  r = dst_row(p, gblk >> lb);
+  blk = (int)(gblk & ((1 << lb) - 1));
+}
+
+// q8_0 of one block (same definition as append_q8_0).  Rounding without the
+// conversion pipe: s = fl(t + 1.5 * 2^23) holds t rounded to an integer (ties
+// to even) in its low mantissa bits, so its low byte is the two's-complement
+// code and s - 1.5 * 2^23 is that integer as a float.  Away from a tie this is
+// roundf; if any t of the block lies within 2^-14 of a half-integer, the whole
+// block takes the exact divide instead.
+__device__ __forceinline__ void q8_0_block(const AppendParams& p, int64_t gblk, const BlockRaw& raw) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  __half2 m2 = __habs2(block_pair(raw, 0));
+#pragma unroll
+  for (int k = 1; k < 16; ++k) m2 = __hmax2(m2, __habs2(block_pair(raw, k)));
+  const float amax = fmaxf(__low2float(m2), __high2float(m2));  // max of fp16 values: exact
+  const float d = __fdiv_rn(amax, 127.0f);
+  const float rd = d != 0.0f ? __frcp_rn(d) : 0.0f;
+  uint32_t code[8];
+  bool near = false;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    uint32_t s4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float t = __fmul_rn(block_elem(raw, 4 * w + i), rd);
+      const float s = __fadd_rn(t, kMagic);
+      near |= fabsf(__fsub_rn(t, __fsub_rn(s, kMagic))) >= 0.49993896484375f;  // 0.5 - 2^-14
+      s4[i] = __float_as_uint(s);
+    }
+    code[w] = __byte_perm(__byte_perm(s4[0], s4[1], 0x0040), __byte_perm(s4[2], s4[3], 0x0040), 0x5410);
+  }
+  if (near) {  // rare: some quotient is close to a tie
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      uint32_t b = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        b |= (uint32_t)((int)roundf(__fdiv_rn(block_elem(raw, 4 * w + i), d)) & 0xFF) << (8 * i);
+      code[w] = b;
+    }
+  }
+  int64_t r;
+  int blk;
+  block_dst(p, gblk, r, blk);
+  uint4* dst = reinterpret_cast<uint4*>(p.dst.codes + r * p.dst.code_bytes + blk * kBlock);
+  dst[0] = make_uint4(code[0], code[1], code[2], code[3]);
+  dst[1] = make_uint4(code[4], code[5], code[6], code[7]);
+  p.dst.scales[r * p.dst.n_scales + blk] = __float2half_rn(d);
+}
+
+// q4_0 of one block (same definition as append_q4_0).
+__device__ __forceinline__ void q4_0_block(const AppendParams& p, int64_t gblk, const BlockRaw& raw) {
+  float bm = block_elem(raw, 0);
+#pragma unroll
+  for (int i = 1; i < kBlock; ++i) {
+    const float x = block_elem(raw, i);
+    if (fabsf(x) > fabsf(bm)) bm = x;  // strictly larger: the first index wins ties
+  }
+  const float d = __fdiv_rn(bm, -8.0f);
+  const float id = d != 0.0f ? __frcp_rn(d) : 0.0f;
+  uint32_t q[kBlock];
+#pragma unroll
+  for (int i = 0; i < kBlock; ++i)
+    q[i] = (uint32_t)min(15, __float2int_rz(__fadd_rn(__fmul_rn(block_elem(raw, i), id), 8.5f)));
+  uint32_t word[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {  // byte j = q_j | q_{j+16} << 4
+    uint32_t b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) b[i] = q[4 * w + i] | (q[4 * w + i + 16] << 4);
+    word[w] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+  }
+  int64_t r;
+  int blk;
+  block_dst(p, gblk, r, blk);
+  *reinterpret_cast<uint4*>(p.dst.codes + r * p.dst.code_bytes + blk * (kBlock / 2)) =
+      make_uint4(word[0], word[1], word[2], word[3]);
+  p.dst.scales[r * p.dst.n_scales + blk] = __float2half_rn(d);
+}
+
 // f16: copy rows, 16 bytes per thread.
-__device__ __forceinline__ void append_f16(const AppendParams& p, int64_t gtid, int64_t gend) {
-  const int per_row = p.D / 8;  // 16-byte chunks per row
+__device__ __forceinline__ void append_f16(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
+  const int per_row = p.D / 8;  // 16-byte chunks per row (a power of two)
   const int64_t i = gtid;
   if (i >= gend) return;
-  const int64_t row = i / per_row;
-  const int c = (int)(i % per_row);
-  const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.src + row * p.D) + c);
+  const int64_t row = i >> (31 - __clz(per_row));
+  const int c = (int)(i & (per_row - 1));
   const int64_t r = dst_row(p, row);
-  reinterpret_cast<uint4*>(p.dst.codes + r * p.dst.code_bytes)[c] = v;
+  reinterpret_cast<uint4*>(p.dst.codes + r * p.dst.code_bytes)[c] = raw;
 }
 
 // turbo3: one warp per row, E = D/32 contiguous elements per lane.
 template <int E>
-__device__ __forceinline__ void append_turbo3(const AppendParams& p, int64_t gtid, int64_t gend) {
+__device__ __forceinline__ void append_turbo3(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
   constexpr int D = 32 * E;
   const int64_t row = gtid >> 5;
   const int lane = (int)(gtid & 31);
   if (gtid >= gend) return;  // whole warps exit together (gend is a multiple of 32)
-  const __half* src = p.src + row * D + lane * E;
   float v[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const int i = lane * E + e;
-    const float x = __half2float(src[e]);
+    const float x = raw_elem(raw, e);
     v[e] = ((p.t3.sign_bits[i >> 5] >> (i & 31)) & 1u) ? -x : x;
   }
   // |v|^2 by the strided pairwise tree a[i] += a[i+h], h = D/2 ... 1
@@ -215,19 +391,34 @@ __device__ __forceinline__ void append_turbo3(const AppendParams& p, int64_t gti
   if (lane == 0) p.dst.scales[r_dst] = __float2half_rn(fminf(norm, 65504.0f));
 }
 
+// Quantize and store work item gtid from its loaded bytes (every lane of the
+// warp calls this: the bodies shuffle; items at or past gend store nothing).
+template <int TYPE, int E>
+__device__ __forceinline__ void finish(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
+  if constexpr (TYPE == KVQ_Q8_0) append_q8_0(p, gtid, gend, raw);
+  else if constexpr (TYPE == KVQ_Q4_0) append_q4_0(p, gtid, gend, raw);
+  else if constexpr (TYPE == KVQ_F16) append_f16(p, gtid, gend, raw);
+  else append_turbo3<E>(p, gtid, gend, raw);
+}
+
+template <int TYPE, int E>
+__device__ __forceinline__ void append_one(const AppendParams& p, int64_t gtid, int64_t gend) {
+  finish<TYPE, E>(p, gtid, gend, load_raw<TYPE, E>(p, gtid, gend));
+}
+
 // Thread gtid of the flat work of one call's rows of a tensor of `type`;
 // threads at or past gend do no work (but still take part in shuffles).
 __device__ __forceinline__ void append_any(int32_t type, const AppendParams& p, int64_t gtid, int64_t gend) {
   switch (type) {
-    case KVQ_F16: append_f16(p, gtid, gend); break;
-    case KVQ_Q8_0: append_q8_0(p, gtid, gend); break;
-    case KVQ_Q4_0: append_q4_0(p, gtid, gend); break;
+    case KVQ_F16: append_one<KVQ_F16, 0>(p, gtid, gend); break;
+    case KVQ_Q8_0: append_one<KVQ_Q8_0, 0>(p, gtid, gend); break;
+    case KVQ_Q4_0: append_one<KVQ_Q4_0, 0>(p, gtid, gend); break;
     case KVQ_TURBO3:
       switch (p.D) {
-        case 32: append_turbo3<1>(p, gtid, gend); break;
-        case 64: append_turbo3<2>(p, gtid, gend); break;
-        case 128: append_turbo3<4>(p, gtid, gend); break;
-        case 256: append_turbo3<8>(p, gtid, gend); break;
+        case 32: append_one<KVQ_TURBO3, 1>(p, gtid, gend); break;
+        case 64: append_one<KVQ_TURBO3, 2>(p, gtid, gend); break;
+        case 128: append_one<KVQ_TURBO3, 4>(p, gtid, gend); break;
+        case 256: append_one<KVQ_TURBO3, 8>(p, gtid, gend); break;
       }
       break;
   }

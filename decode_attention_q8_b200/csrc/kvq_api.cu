@@ -374,6 +374,8 @@ kvq_status kvq_append_quantize(const kvq_cache_desc* d, void* k_cache, void* v_c
     p.D = d->head_dim;
     p.n_tok = n_tok;
     p.pos = pos;
+    p.h_mul = div_multiplier((uint64_t)p.H);
+    p.t_mul = div_multiplier((uint64_t)n_tok);
     if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) p.t3 = turbo3_consts(d);
   }
   const cudaError_t e = launch_append(do_k ? &ap[0] : nullptr, d->k_type, do_v ? &ap[1] : nullptr, d->v_type, s);
@@ -413,6 +415,8 @@ kvq_status kvq_decode_step(const kvq_cache_desc* d, void* k_cache, void* v_cache
     a.D = d->head_dim;
     a.n_tok = 1;
     a.pos = p.append_pos;
+    a.h_mul = div_multiplier((uint64_t)a.H);
+    a.t_mul = div_multiplier(1);
     if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) a.t3 = turbo3_consts(d);
   }
   p.out = out;

@@ -35,8 +35,15 @@ struct AppendParams {
   Plane dst;
   int32_t B, H, D, n_tok;
   int64_t pos;
+  // n / H and n / n_tok for 32-bit n as the high half of n * mul (mul = 0: divisor 1)
+  uint64_t h_mul, t_mul;
   Turbo3Consts t3;
 };
+
+// Multiplier for exact division of any 32-bit n by d (d >= 1): n / d equals the
+// high 64 bits of n * (floor((2^64 - 1) / d) + 1), since the added n / 2^64 per
+// unit of error stays below 1 / d; 0 stands for d = 1.
+inline uint64_t div_multiplier(uint64_t d) { return d <= 1 ? 0 : ~0ull / d + 1; }
 
 struct DecodeParams {
   Plane k, v;
