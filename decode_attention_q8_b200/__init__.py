@@ -34,6 +34,7 @@ EXPORTED = (
     "kvq_cache_layout", "kvq_cache_bytes", "kvq_auto_splits", "kvq_workspace_bytes",
     "kvq_turbo3_codebook", "kvq_turbo3_signs", "kvq_append_quantize",
     "kvq_decode_attention", "kvq_combine", "kvq_decode_attention_noalloc", "kvq_decode_step",
+    "kvq_decode_attention_varlen", "kvq_decode_step_varlen", "kvq_append_quantize_varlen",
 )
 
 
@@ -83,6 +84,11 @@ _sigs = {
                                                     ctypes.c_int32, _P, _P]),
     "kvq_decode_step": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
                                        ctypes.c_int32, _P, ctypes.c_size_t, _P, _P]),
+    "kvq_decode_attention_varlen": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, _P, ctypes.c_int64,
+                                                   ctypes.c_float, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
+    "kvq_decode_step_varlen": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, ctypes.c_int32, _P, ctypes.c_int64,
+                                              ctypes.c_float, ctypes.c_int32, _P, ctypes.c_size_t, _P, _P]),
+    "kvq_append_quantize_varlen": (ctypes.c_int, [_D, _P, _P, _P, _P, ctypes.c_int32, _P, ctypes.c_int32, _P]),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -223,6 +229,39 @@ def kvq_decode_step(desc, k_cache, v_cache, q, k_new, v_new, batch, ctx_len, sof
                                        _ptr(v_new), batch, ctx_len, softmax_scale, n_splits, _ptr(workspace),
                                        workspace_bytes, _ptr(out), _stream(stream)),
                   "kvq_decode_step")
+
+
+def kvq_append_quantize_varlen(desc, k_cache, v_cache, k_new, v_new, batch, lens, n_tok, stream=None):
+    """Append n_tok rows per batch entry at rows lens[b] - n_tok .. lens[b] - 1
+    (``lens``: device int32 [batch], each sequence's length after the append)."""
+    return _check(_lib.kvq_append_quantize_varlen(ctypes.byref(desc), _ptr(k_cache), _ptr(v_cache), _ptr(k_new),
+                                                  _ptr(v_new), batch, _ptr(lens), n_tok, _stream(stream)),
+                  "kvq_append_quantize_varlen")
+
+
+def kvq_decode_attention_varlen(desc, k_cache, v_cache, q, batch, ctx_lens, max_ctx_len, softmax_scale, n_splits,
+                                workspace, workspace_bytes=None, stream=None):
+    """Split-KV decode where batch row b attends rows 0 .. ctx_lens[b]-1
+    (``ctx_lens``: device int32 [batch]; ``max_ctx_len`` bounds them)."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return _check(_lib.kvq_decode_attention_varlen(ctypes.byref(desc), _ptr(k_cache), _ptr(v_cache), _ptr(q), batch,
+                                                   _ptr(ctx_lens), max_ctx_len, softmax_scale, n_splits,
+                                                   _ptr(workspace), workspace_bytes, _stream(stream)),
+                  "kvq_decode_attention_varlen")
+
+
+def kvq_decode_step_varlen(desc, k_cache, v_cache, q, k_new, v_new, batch, ctx_lens, max_ctx_len, softmax_scale,
+                           n_splits, workspace, out, workspace_bytes=None, stream=None):
+    """kvq_decode_step with per-sequence lengths: row b's new K/V row lands at
+    ctx_lens[b] - 1 and rows 0 .. ctx_lens[b]-1 are attended."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return _check(_lib.kvq_decode_step_varlen(ctypes.byref(desc), _ptr(k_cache), _ptr(v_cache), _ptr(q),
+                                              _ptr(k_new), _ptr(v_new), batch, _ptr(ctx_lens), max_ctx_len,
+                                              softmax_scale, n_splits, _ptr(workspace), workspace_bytes, _ptr(out),
+                                              _stream(stream)),
+                  "kvq_decode_step_varlen")
 
 
 def raw_status(name, *args):

@@ -63,7 +63,8 @@ __device__ __forceinline__ float raw_elem(const uint4& r, int i) {  // fp16 elem
   return __half2float(__ushort_as_half(h));
 }
 
-// Destination row index of flat input row `row` = ((b * n_tok + t) * H + h).
+// Destination row index of flat input row `row` = ((b * n_tok + t) * H + h),
+// or -1 when batch row b's length (per-sequence lengths) is out of range.
 // 32-bit division when the call's rows fit (the 64-bit one is a long routine).
 __device__ __forceinline__ int64_t dst_row(const AppendParams& p, int64_t row) {
   int64_t h, t, b;
@@ -78,7 +79,13 @@ __device__ __forceinline__ int64_t dst_row(const AppendParams& p, int64_t row) {
     t = (row / p.H) % p.n_tok;
     b = row / ((int64_t)p.H * p.n_tok);
   }
-  return (b * p.H + h) * p.dst.T + p.pos + t;
+  int64_t pos = p.pos;
+  if (p.lens != nullptr) {
+    const int64_t len = p.lens[b];
+    if (len < p.n_tok || len > p.len_max) return -1;
+    pos = len - p.n_tok;
+  }
+  return (b * p.H + h) * p.dst.T + pos + t;
 }
 
 // log2 of the 32-element blocks per row (head_dim is 32 times a power of two)
@@ -120,6 +127,7 @@ __device__ __forceinline__ void append_q8_0(const AppendParams& p, int64_t gtid,
   const int64_t row = gblk >> log2_blocks(p);
   const int blk = (int)(gblk & (nb - 1));
   const int64_t r = dst_row(p, row);
+  if (r < 0) return;
   *reinterpret_cast<uint32_t*>(p.dst.codes + r * p.dst.code_bytes + blk * kBlock + sub * 4) = packed;
   if (sub == 0) p.dst.scales[r * p.dst.n_scales + blk] = __float2half_rn(d);
 }
@@ -163,6 +171,7 @@ __device__ __forceinline__ void append_q4_0(const AppendParams& p, int64_t gtid,
   const int64_t row = gblk >> log2_blocks(p);
   const int blk = (int)(gblk & (nb - 1));
   const int64_t r = dst_row(p, row);
+  if (r < 0) return;
   *reinterpret_cast<uint32_t*>(p.dst.codes + r * p.dst.code_bytes + blk * 16 + sub * 4) = bytes;
   if (sub == 0) p.dst.scales[r * p.dst.n_scales + blk] = __float2half_rn(d);
 }
@@ -207,7 +216,8 @@ __device__ __forceinline__ __half2 block_pair(const BlockRaw& r, int k) {  // el
   return *reinterpret_cast<const __half2*>(&w);
 }
 
-// Where block gblk's row lands in the cache, and the block's index in its row.
+// Where block gblk's row lands in the cache (-1: not written), and the block's
+// index in its row.
 __device__ __forceinline__ void block_dst(const AppendParams& p, int64_t gblk, int64_t& r, int& blk) {
   const int lb = log2_blocks(p);
   r = dst_row(p, gblk >> lb);
@@ -255,6 +265,7 @@ __device__ __forceinline__ void q8_0_block(const AppendParams& p, int64_t gblk, 
   int64_t r;
   int blk;
   block_dst(p, gblk, r, blk);
+  if (r < 0) return;
   uint4* dst = reinterpret_cast<uint4*>(p.dst.codes + r * p.dst.code_bytes + blk * kBlock);
   dst[0] = make_uint4(code[0], code[1], code[2], code[3]);
   dst[1] = make_uint4(code[4], code[5], code[6], code[7]);
@@ -286,6 +297,7 @@ __device__ __forceinline__ void q4_0_block(const AppendParams& p, int64_t gblk, 
   int64_t r;
   int blk;
   block_dst(p, gblk, r, blk);
+  if (r < 0) return;
   *reinterpret_cast<uint4*>(p.dst.codes + r * p.dst.code_bytes + blk * (kBlock / 2)) =
       make_uint4(word[0], word[1], word[2], word[3]);
   p.dst.scales[r * p.dst.n_scales + blk] = __float2half_rn(d);
@@ -299,6 +311,7 @@ __device__ __forceinline__ void append_f16(const AppendParams& p, int64_t gtid, 
   const int64_t row = i >> (31 - __clz(per_row));
   const int c = (int)(i & (per_row - 1));
   const int64_t r = dst_row(p, row);
+  if (r < 0) return;
   reinterpret_cast<uint4*>(p.dst.codes + r * p.dst.code_bytes)[c] = raw;
 }
 
@@ -372,6 +385,7 @@ __device__ __forceinline__ void append_turbo3(const AppendParams& p, int64_t gti
     word |= o << (3 * E * j);
   }
   const int64_t r_dst = dst_row(p, row);
+  if (r_dst < 0) return;  // after the last shuffle
   uint8_t* codes = p.dst.codes + r_dst * p.dst.code_bytes;
   if (E >= 8) {
 #pragma unroll

@@ -338,8 +338,16 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::NW * L::WARP + L::TABLE) + warp * S;
 
   const int s_idx = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int64_t t0l = (int64_t)s_idx * p.chunk;
-  const int64_t t1l = min(p.ctx, t0l + p.chunk);
+  // rows of this batch row, and its split length (a multiple of 16 rows)
+  int64_t ctx = p.ctx, chunk = p.chunk, append_pos = p.append_pos;
+  if (p.ctx_lens != nullptr) {
+    const int64_t len = p.ctx_lens[b];
+    ctx = len >= 1 && len <= p.ctx ? len : 0;  // out of range: attends nothing
+    chunk = ((ctx + p.S - 1) / p.S + kSplitAlign - 1) / kSplitAlign * kSplitAlign;
+    if (append_pos >= 0) append_pos = ctx - 1;
+  }
+  const int64_t t0l = (int64_t)s_idx * chunk;
+  const int64_t t1l = min(ctx, t0l + chunk);
   const int n_sub = t0l < t1l ? (int)((t1l - t0l + kSub - 1) / kSub) : 0;
   // row indices fit in 32 bits (the tensor-map coordinates are 32-bit)
   const int t0 = (int)t0l, t1 = (int)t1l;
@@ -393,8 +401,8 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   // then quantizes and writes the row of K and of V itself, makes the writes
   // visible device-wide and to the async proxy, and only then issues the tile
   // that reads the row back; no other warp waits.
-  const bool owner = p.append_pos >= t0l && p.append_pos < t1l;
-  const int t_new = owner ? (int)(p.append_pos - t0l) / kSub : -1;
+  const bool owner = append_pos >= t0l && append_pos < t1l;
+  const int t_new = owner ? (int)(append_pos - t0l) / kSub : -1;
   const int wt = owner ? t_new % L::NW : -1, jt = owner ? t_new / L::NW : -1;
   if (lane == 0) {
     for (int j = 0; j < S && j < my_tiles; ++j)

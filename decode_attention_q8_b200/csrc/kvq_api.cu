@@ -213,10 +213,11 @@ Plane plane_of(const kvq_cache_desc* d, int32_t batch, int which, void* base) {
 
 
 // Checks and fills the parameters of a decode launch (kvq_decode_attention and
-// kvq_decode_step); a plain decode appends nothing and writes partials only.
+// kvq_decode_step, and their per-sequence-length forms, where ctx_len is the
+// bound on the lengths); a plain decode appends nothing and writes partials only.
 kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void* v_cache, const void* q,
-                       int32_t batch, int64_t ctx_len, float softmax_scale, int32_t n_splits, void* workspace,
-                       size_t workspace_bytes, DecodeParams* out) {
+                       int32_t batch, int64_t ctx_len, const int32_t* ctx_lens, float softmax_scale,
+                       int32_t n_splits, void* workspace, size_t workspace_bytes, DecodeParams* out) {
   kvq_status st = kvq_check_desc(d);
   if (st != KVQ_OK) return st;
   if (!k_cache || !v_cache || !q || !workspace) return KVQ_ERR_INVALID;
@@ -224,6 +225,7 @@ kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void*
   if (n_splits < 0 || n_splits > kMaxSplits || !std::isfinite(softmax_scale)) return KVQ_ERR_INVALID;
   if (!aligned(k_cache, 256) || !aligned(v_cache, 256) || !aligned(q, 16) || !aligned(workspace, 256))
     return KVQ_ERR_INVALID;
+  if (ctx_lens != nullptr && !aligned(ctx_lens, 4)) return KVQ_ERR_INVALID;
   const int32_t G = d->n_q_heads / d->n_kv_heads;
   if (!decode_supported(d->k_type, d->v_type, G, d->head_dim)) return KVQ_ERR_UNSUPPORTED;
   const int32_t S = resolve_splits(d, batch, ctx_len, n_splits);
@@ -247,6 +249,7 @@ kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void*
   p.S = S;
   p.ctx = ctx_len;
   p.chunk = chunk_rows(ctx_len, S);
+  p.ctx_lens = ctx_lens;
   p.qscale = softmax_scale * 1.4426950408889634f;
   if (d->v_type == KVQ_TURBO3) p.t3 = turbo3_consts(d);
   p.append_pos = -1;
@@ -254,6 +257,91 @@ kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void*
   p.counters = nullptr;
   return KVQ_OK;
 }
+kvq_status append_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                       int32_t batch, int64_t pos, const int32_t* lens, int32_t n_tok, void* stream) {
+  kvq_status st = kvq_check_desc(d);
+  if (st != KVQ_OK) return st;
+  if (batch < 1 || batch > 65535 || n_tok < 1 || n_tok > d->max_ctx) return KVQ_ERR_INVALID;
+  if (lens == nullptr && (pos < 0 || pos + n_tok > d->max_ctx)) return KVQ_ERR_INVALID;
+  if (lens != nullptr && !aligned(lens, 4)) return KVQ_ERR_INVALID;
+  const bool do_k = k_cache != nullptr, do_v = v_cache != nullptr;
+  if (do_k != (k_new != nullptr) || do_v != (v_new != nullptr) || (!do_k && !do_v)) return KVQ_ERR_INVALID;
+  if ((do_k && (!aligned(k_cache, 256) || !aligned(k_new, 16))) ||
+      (do_v && (!aligned(v_cache, 256) || !aligned(v_new, 16))))
+    return KVQ_ERR_INVALID;
+  const int64_t rows = (int64_t)batch * n_tok * d->n_kv_heads;
+  if (rows * (d->head_dim / 4) > ((int64_t)1 << 40)) return KVQ_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  AppendParams ap[2];
+  for (int which = 0; which < 2; ++which) {
+    void* cache = which ? v_cache : k_cache;
+    if (!cache) continue;
+    AppendParams& p = ap[which];
+    p = AppendParams{};
+    p.src = static_cast<const __half*>(which ? v_new : k_new);
+    p.dst = plane_of(d, batch, which, cache);
+    p.B = batch;
+    p.H = d->n_kv_heads;
+    p.D = d->head_dim;
+    p.n_tok = n_tok;
+    p.pos = lens ? 0 : pos;
+    p.lens = lens;
+    p.len_max = d->max_ctx;
+    p.h_mul = div_multiplier((uint64_t)p.H);
+    p.t_mul = div_multiplier((uint64_t)n_tok);
+    if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) p.t3 = turbo3_consts(d);
+  }
+  const cudaError_t e = launch_append(do_k ? &ap[0] : nullptr, d->k_type, do_v ? &ap[1] : nullptr, d->v_type, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KVQ_OK;
+}
+
+kvq_status decode_impl(const kvq_cache_desc* d, const void* k_cache, const void* v_cache, const void* q,
+                       int32_t batch, int64_t ctx_len, const int32_t* ctx_lens, float softmax_scale,
+                       int32_t n_splits, void* workspace, size_t workspace_bytes, void* stream) {
+  DecodeParams p{};
+  const kvq_status st = fill_decode(d, k_cache, v_cache, q, batch, ctx_len, ctx_lens, softmax_scale, n_splits,
+                                    workspace, workspace_bytes, &p);
+  if (st != KVQ_OK) return st;
+  const cudaError_t e = launch_decode(d->k_type, d->v_type, p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KVQ_OK;
+}
+
+kvq_status step_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* q, const void* k_new,
+                     const void* v_new, int32_t batch, int64_t ctx_len, const int32_t* ctx_lens,
+                     float softmax_scale, int32_t n_splits, void* workspace, size_t workspace_bytes, float* out,
+                     void* stream) {
+  if (!k_new || !v_new || !out) return KVQ_ERR_INVALID;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(out, 16)) return KVQ_ERR_INVALID;
+  DecodeParams p{};
+  const kvq_status st = fill_decode(d, k_cache, v_cache, q, batch, ctx_len, ctx_lens, softmax_scale, n_splits,
+                                    workspace, workspace_bytes, &p);
+  if (st != KVQ_OK) return st;
+  const WsLayout w = ws_layout(d, batch, p.S);
+  p.append_pos = ctx_len - 1;  // with ctx_lens the kernel takes ctx_lens[b] - 1
+  for (int which = 0; which < 2; ++which) {
+    AppendParams& a = which ? p.app_v : p.app_k;
+    a.src = static_cast<const __half*>(which ? v_new : k_new);
+    a.dst = which ? p.v : p.k;
+    a.B = batch;
+    a.H = d->n_kv_heads;
+    a.D = d->head_dim;
+    a.n_tok = 1;
+    a.pos = p.append_pos;
+    a.lens = ctx_lens;
+    a.len_max = ctx_len;
+    a.h_mul = div_multiplier((uint64_t)a.H);
+    a.t_mul = div_multiplier(1);
+    if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) a.t3 = turbo3_consts(d);
+  }
+  p.out = out;
+  p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + w.cnt_off);
+  const cudaError_t e = launch_decode(d->k_type, d->v_type, p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KVQ_OK;
+}
+
 }  // namespace
 
 void set_last_cuda_error(cudaError_t e) { g_last_cuda_error = cudaGetErrorString(e); }
@@ -350,80 +438,46 @@ kvq_status kvq_turbo3_signs(uint64_t seed, int32_t head_dim, float* signs) {
 
 kvq_status kvq_append_quantize(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* k_new,
                                const void* v_new, int32_t batch, int64_t pos, int32_t n_tok, void* stream) {
-  kvq_status st = kvq_check_desc(d);
-  if (st != KVQ_OK) return st;
-  if (batch < 1 || batch > 65535 || n_tok < 1 || pos < 0 || pos + n_tok > d->max_ctx) return KVQ_ERR_INVALID;
-  const bool do_k = k_cache != nullptr, do_v = v_cache != nullptr;
-  if (do_k != (k_new != nullptr) || do_v != (v_new != nullptr) || (!do_k && !do_v)) return KVQ_ERR_INVALID;
-  if ((do_k && (!aligned(k_cache, 256) || !aligned(k_new, 16))) ||
-      (do_v && (!aligned(v_cache, 256) || !aligned(v_new, 16))))
-    return KVQ_ERR_INVALID;
-  const int64_t rows = (int64_t)batch * n_tok * d->n_kv_heads;
-  if (rows * (d->head_dim / 4) > ((int64_t)1 << 40)) return KVQ_ERR_UNSUPPORTED;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  AppendParams ap[2];
-  for (int which = 0; which < 2; ++which) {
-    void* cache = which ? v_cache : k_cache;
-    if (!cache) continue;
-    AppendParams& p = ap[which];
-    p = AppendParams{};
-    p.src = static_cast<const __half*>(which ? v_new : k_new);
-    p.dst = plane_of(d, batch, which, cache);
-    p.B = batch;
-    p.H = d->n_kv_heads;
-    p.D = d->head_dim;
-    p.n_tok = n_tok;
-    p.pos = pos;
-    p.h_mul = div_multiplier((uint64_t)p.H);
-    p.t_mul = div_multiplier((uint64_t)n_tok);
-    if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) p.t3 = turbo3_consts(d);
-  }
-  const cudaError_t e = launch_append(do_k ? &ap[0] : nullptr, d->k_type, do_v ? &ap[1] : nullptr, d->v_type, s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  return KVQ_OK;
+  return append_impl(d, k_cache, v_cache, k_new, v_new, batch, pos, nullptr, n_tok, stream);
+}
+
+kvq_status kvq_append_quantize_varlen(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* k_new,
+                                      const void* v_new, int32_t batch, const int32_t* lens, int32_t n_tok,
+                                      void* stream) {
+  if (!lens) return KVQ_ERR_INVALID;
+  return append_impl(d, k_cache, v_cache, k_new, v_new, batch, 0, lens, n_tok, stream);
 }
 
 kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* k_cache, const void* v_cache, const void* q,
                                 int32_t batch, int64_t ctx_len, float softmax_scale, int32_t n_splits,
                                 void* workspace, size_t workspace_bytes, void* stream) {
-  DecodeParams p{};
-  const kvq_status st = fill_decode(d, k_cache, v_cache, q, batch, ctx_len, softmax_scale, n_splits, workspace,
-                                    workspace_bytes, &p);
-  if (st != KVQ_OK) return st;
-  const cudaError_t e = launch_decode(d->k_type, d->v_type, p, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e);
-  return KVQ_OK;
+  return decode_impl(d, k_cache, v_cache, q, batch, ctx_len, nullptr, softmax_scale, n_splits, workspace,
+                     workspace_bytes, stream);
+}
+
+kvq_status kvq_decode_attention_varlen(const kvq_cache_desc* d, const void* k_cache, const void* v_cache,
+                                       const void* q, int32_t batch, const int32_t* ctx_lens, int64_t max_ctx_len,
+                                       float softmax_scale, int32_t n_splits, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  if (!ctx_lens) return KVQ_ERR_INVALID;
+  return decode_impl(d, k_cache, v_cache, q, batch, max_ctx_len, ctx_lens, softmax_scale, n_splits, workspace,
+                     workspace_bytes, stream);
 }
 
 kvq_status kvq_decode_step(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* q, const void* k_new,
                            const void* v_new, int32_t batch, int64_t ctx_len, float softmax_scale, int32_t n_splits,
                            void* workspace, size_t workspace_bytes, float* out, void* stream) {
-  if (!k_new || !v_new || !out) return KVQ_ERR_INVALID;
-  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(out, 16)) return KVQ_ERR_INVALID;
-  DecodeParams p{};
-  const kvq_status st = fill_decode(d, k_cache, v_cache, q, batch, ctx_len, softmax_scale, n_splits, workspace,
-                                    workspace_bytes, &p);
-  if (st != KVQ_OK) return st;
-  const WsLayout w = ws_layout(d, batch, p.S);
-  p.append_pos = ctx_len - 1;
-  for (int which = 0; which < 2; ++which) {
-    AppendParams& a = which ? p.app_v : p.app_k;
-    a.src = static_cast<const __half*>(which ? v_new : k_new);
-    a.dst = which ? p.v : p.k;
-    a.B = batch;
-    a.H = d->n_kv_heads;
-    a.D = d->head_dim;
-    a.n_tok = 1;
-    a.pos = p.append_pos;
-    a.h_mul = div_multiplier((uint64_t)a.H);
-    a.t_mul = div_multiplier(1);
-    if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) a.t3 = turbo3_consts(d);
-  }
-  p.out = out;
-  p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + w.cnt_off);
-  const cudaError_t e = launch_decode(d->k_type, d->v_type, p, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e);
-  return KVQ_OK;
+  return step_impl(d, k_cache, v_cache, q, k_new, v_new, batch, ctx_len, nullptr, softmax_scale, n_splits,
+                   workspace, workspace_bytes, out, stream);
+}
+
+kvq_status kvq_decode_step_varlen(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* q,
+                                  const void* k_new, const void* v_new, int32_t batch, const int32_t* ctx_lens,
+                                  int64_t max_ctx_len, float softmax_scale, int32_t n_splits, void* workspace,
+                                  size_t workspace_bytes, float* out, void* stream) {
+  if (!ctx_lens) return KVQ_ERR_INVALID;
+  return step_impl(d, k_cache, v_cache, q, k_new, v_new, batch, max_ctx_len, ctx_lens, softmax_scale, n_splits,
+                   workspace, workspace_bytes, out, stream);
 }
 
 kvq_status kvq_combine(const kvq_cache_desc* d, const void* workspace, size_t workspace_bytes, int32_t batch,

@@ -35,6 +35,11 @@ struct AppendParams {
   Plane dst;
   int32_t B, H, D, n_tok;
   int64_t pos;
+  // Per-sequence lengths (device int32 [B], or null: every row at pos): batch
+  // row b's tokens land at lens[b] - n_tok .. lens[b] - 1; a row whose length
+  // lies outside [n_tok, len_max] is not written.
+  const int32_t* lens;
+  int64_t len_max;
   // n / H and n / n_tok for 32-bit n as the high half of n * mul (mul = 0: divisor 1)
   uint64_t h_mul, t_mul;
   Turbo3Consts t3;
@@ -53,11 +58,16 @@ struct DecodeParams {
   float* ws_acc;       // [B][n_q][S][D]
   int32_t B, n_q, n_kv, G, D, S;
   int64_t ctx, chunk;
+  // Per-sequence lengths (device int32 [B], or null: every row attends ctx
+  // rows): batch row b attends rows [0, ctx_lens[b]) in S chunks of its own;
+  // ctx is then the bound, and a length outside [1, ctx] attends nothing.
+  const int32_t* ctx_lens;
   float qscale;        // softmax_scale * log2(e)
   Turbo3Consts t3;     // V sign bits and codebook (turbo3 values)
   // Fused decode step (kvq_decode_step); a plain decode has append_pos < 0 and
   // out == null.
-  int64_t append_pos;    // row the new K/V rows are written to first (< 0: none)
+  int64_t append_pos;    // row the new K/V rows are written to first (< 0: none;
+                         // with ctx_lens, batch row b's is ctx_lens[b] - 1)
   AppendParams app_k;    // that append: B = batch, H = n_kv, n_tok = 1
   AppendParams app_v;
   float* out;            // [B][n_q][D] combined output, or null (partials only)

@@ -261,6 +261,54 @@ KVQ_API kvq_status kvq_decode_step(const kvq_cache_desc* desc, void* k_cache, vo
                                    int32_t n_splits, void* workspace, size_t workspace_bytes,
                                    float* out, void* cuda_stream);
 
+/*
+ * Per-sequence context lengths.  A server's cache holds several sequences (the
+ * llama.cpp issue "Eval bug: Metal fails mixed quantized KV on Apple Silicon
+ * when Flash Attention is unavailable, ...": the kv-cache line in a comment's
+ * "Relevant output" reports 4/1 sequences), and the sequences of one batch need
+ * not have equal lengths.  These forms take the lengths from device memory, so a
+ * captured CUDA graph can be replayed as the lengths grow, with no host round
+ * trip.
+ *   ctx_lens      device int32 [batch], 4-byte aligned; read by the kernels when
+ *                 they run.
+ *   max_ctx_len   host bound on the lengths, 1 <= max_ctx_len <= max_ctx.  It
+ *                 takes ctx_len's place in the split choice (n_splits = 0),
+ *                 in kvq_workspace_bytes and in kvq_combine.
+ * Batch row b attends rows [0, ctx_lens[b]), cut into n_splits chunks of its
+ * own (a multiple of 16 rows each; trailing splits may be empty).  A length
+ * outside [1, max_ctx_len] attends no row: that row reads no cache byte, every
+ * split partial is empty (m = -inf, l = 0), and the combined output is NaN.
+ * Nothing is read or written out of bounds, whatever the lengths hold.
+ */
+KVQ_API kvq_status kvq_decode_attention_varlen(const kvq_cache_desc* desc, const void* k_cache,
+                                               const void* v_cache, const void* q, int32_t batch,
+                                               const int32_t* ctx_lens, int64_t max_ctx_len,
+                                               float softmax_scale, int32_t n_splits, void* workspace,
+                                               size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * kvq_decode_step with per-sequence lengths: batch row b's new K/V row is
+ * written at row ctx_lens[b] - 1, then rows [0, ctx_lens[b]) are attended.  A
+ * row whose length lies outside [1, max_ctx_len] writes nothing to the caches,
+ * and its output is NaN.
+ */
+KVQ_API kvq_status kvq_decode_step_varlen(const kvq_cache_desc* desc, void* k_cache, void* v_cache,
+                                          const void* q, const void* k_new, const void* v_new,
+                                          int32_t batch, const int32_t* ctx_lens, int64_t max_ctx_len,
+                                          float softmax_scale, int32_t n_splits, void* workspace,
+                                          size_t workspace_bytes, float* out, void* cuda_stream);
+
+/*
+ * kvq_append_quantize with per-sequence positions: batch row b's n_tok rows
+ * land at rows lens[b] - n_tok .. lens[b] - 1.  lens holds each sequence's
+ * length after the append: device int32 [batch], 4-byte aligned, read by the
+ * kernel.  A row whose lens[b] lies outside [n_tok, max_ctx] is not written.
+ * The stored bytes are those kvq_append_quantize writes at the same positions.
+ */
+KVQ_API kvq_status kvq_append_quantize_varlen(const kvq_cache_desc* desc, void* k_cache, void* v_cache,
+                                              const void* k_new, const void* v_new, int32_t batch,
+                                              const int32_t* lens, int32_t n_tok, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

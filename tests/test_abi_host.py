@@ -181,6 +181,51 @@ def test_decode_step_rejects_before_launch():
     assert _step(kvq.make_desc(32, 8, 128, "turbo3", "q4_0", 64)) == kvq.KVQ_ERR_UNSUPPORTED
 
 
+def _decode_varlen(desc, lens=FAKE, max_ctx=16, q=FAKE, S=0, ws=FAKE, ws_bytes=1 << 40):
+    return kvq.raw_status("kvq_decode_attention_varlen", ctypes.byref(desc), FAKE, FAKE, q, 1, lens, max_ctx,
+                          0.1, S, ws, ws_bytes, None)
+
+
+def _step_varlen(desc, lens=FAKE, max_ctx=16, k_new=FAKE, S=0, ws_bytes=1 << 40, out=FAKE):
+    return kvq.raw_status("kvq_decode_step_varlen", ctypes.byref(desc), FAKE, FAKE, FAKE, k_new, FAKE, 1, lens,
+                          max_ctx, 0.1, S, FAKE, ws_bytes, out, None)
+
+
+def _append_varlen(desc, lens=FAKE, n_tok=1, batch=1, k_new=FAKE):
+    return kvq.raw_status("kvq_append_quantize_varlen", ctypes.byref(desc), FAKE, FAKE, k_new, FAKE, batch, lens,
+                          n_tok, None)
+
+
+def test_varlen_entry_points_reject_before_launch():
+    d = kvq.make_desc(32, 8, 128, "q8_0", "q4_0", 8192)
+    # the lengths pointer: required, 4-byte aligned
+    assert _decode_varlen(d, lens=None) == kvq.KVQ_ERR_INVALID
+    assert _decode_varlen(d, lens=FAKE + 2) == kvq.KVQ_ERR_INVALID
+    assert _step_varlen(d, lens=None) == kvq.KVQ_ERR_INVALID
+    assert _step_varlen(d, lens=FAKE + 1) == kvq.KVQ_ERR_INVALID
+    assert _append_varlen(d, lens=None) == kvq.KVQ_ERR_INVALID
+    assert _append_varlen(d, lens=FAKE + 3) == kvq.KVQ_ERR_INVALID
+    # the host bound on the lengths takes ctx_len's checks
+    assert _decode_varlen(d, max_ctx=0) == kvq.KVQ_ERR_INVALID
+    assert _decode_varlen(d, max_ctx=8193) == kvq.KVQ_ERR_INVALID
+    assert _step_varlen(d, max_ctx=0) == kvq.KVQ_ERR_INVALID
+    assert _step_varlen(d, max_ctx=8193) == kvq.KVQ_ERR_INVALID
+    # everything else as in the uniform-length forms
+    assert _decode_varlen(d, q=None) == kvq.KVQ_ERR_INVALID
+    need = kvq.kvq_workspace_bytes(d, 1, 4)
+    assert _decode_varlen(d, S=4, ws_bytes=need - 1) == kvq.KVQ_ERR_WORKSPACE
+    assert _step_varlen(d, S=4, ws_bytes=need - 1) == kvq.KVQ_ERR_WORKSPACE
+    assert _step_varlen(d, k_new=None) == kvq.KVQ_ERR_INVALID
+    assert _step_varlen(d, out=FAKE + 4) == kvq.KVQ_ERR_INVALID
+    assert _append_varlen(d, n_tok=0) == kvq.KVQ_ERR_INVALID
+    assert _append_varlen(d, n_tok=8193) == kvq.KVQ_ERR_INVALID     # no sequence can hold them
+    assert _append_varlen(d, batch=0) == kvq.KVQ_ERR_INVALID
+    assert _append_varlen(d, k_new=FAKE + 8) == kvq.KVQ_ERR_INVALID
+    t3k = kvq.make_desc(32, 8, 128, "turbo3", "q4_0", 64)
+    assert _decode_varlen(t3k) == kvq.KVQ_ERR_UNSUPPORTED
+    assert _append_varlen(t3k) == kvq.KVQ_ERR_UNSUPPORTED
+
+
 def test_workspace_bytes_formula():
     d = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 32768)
     B, S = 4, 9
