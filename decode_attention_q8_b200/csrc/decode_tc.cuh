@@ -353,6 +353,38 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   const int t0 = (int)t0l, t1 = (int)t1l;
   const int plane = b * p.n_kv + kvh;
 
+  // The queries are read before any cache tile is requested: issued after the
+  // tiles, these few bytes would wait behind every warp's first stages on the
+  // SM's return path (several microseconds when the stages hold most of a
+  // split).  Raw words here; their fragment form is built further down.
+  //   q8_0 / q4_0: 16-byte segments 2*blk, 2*blk+1, lane c's bytes 4c..4c+3
+  //   f16: dims 32*blk + 8*i + 2c, +1 for i = 0..3
+  uint32_t qraw[NTH][NB][4];
+#pragma unroll
+  for (int nt = 0; nt < NTH; ++nt) {
+    const int head = nt * 8 + g;
+    const bool hv = head < p.G;
+    const __half* qrow = p.q + ((int64_t)b * p.n_q + (int64_t)kvh * p.G + (hv ? head : 0)) * D;
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
+      uint32_t* w = qraw[nt][blk];
+      w[0] = w[1] = w[2] = w[3] = 0u;
+      if (hv) {
+        if (KT == KVQ_F16) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) w[i] = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 8 * i + 2 * c);
+        } else {
+          const uint2 s0 = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 4 * c);
+          const uint2 s1 = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 16 + 4 * c);
+          w[0] = s0.x;
+          w[1] = s0.y;
+          w[2] = s1.x;
+          w[3] = s1.y;
+        }
+      }
+    }
+  }
+
   if (threadIdx.x == 0) cta_failed = 0;
   if (lane == 0) {
 #pragma unroll
@@ -441,33 +473,15 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   constexpr float kBiasK = KT == KVQ_Q8_0 ? 128.f : KT == KVQ_Q4_0 ? 8.f : 0.f;
 #pragma unroll
   for (int nt = 0; nt < NTH; ++nt) {
-    const int head = nt * 8 + g;
-    const bool hv = head < p.G;
-    const __half* qrow = p.q + ((int64_t)b * p.n_q + (int64_t)kvh * p.G + (hv ? head : 0)) * D;
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk) {
-      uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
-      if (hv) {
-        if (KT == KVQ_Q4_0) {
-          const uint2 lo = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 4 * c);       // dims 4c..4c+3
-          const uint2 hi = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 16 + 4 * c);  // 4c+16..
-          w0 = prmt(lo.x, lo.y, 0x5410);  // (4c, 4c+2)
-          w1 = prmt(lo.x, lo.y, 0x7632);  // (4c+1, 4c+3)
-          w2 = prmt(hi.x, hi.y, 0x5410);
-          w3 = prmt(hi.x, hi.y, 0x7632);
-        } else if (KT == KVQ_Q8_0) {
-          const uint2 s0 = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 4 * c);       // segment 0
-          const uint2 s1 = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 16 + 4 * c);  // segment 1
-          w0 = s0.x;
-          w1 = s0.y;
-          w2 = s1.x;
-          w3 = s1.y;
-        } else {
-          w0 = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 2 * c);
-          w1 = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 8 + 2 * c);
-          w2 = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 16 + 2 * c);
-          w3 = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 24 + 2 * c);
-        }
+      const uint32_t* r = qraw[nt][blk];
+      uint32_t w0 = r[0], w1 = r[1], w2 = r[2], w3 = r[3];
+      if (KT == KVQ_Q4_0) {
+        w0 = prmt(r[0], r[1], 0x5410);  // (4c, 4c+2)
+        w1 = prmt(r[0], r[1], 0x7632);  // (4c+1, 4c+3)
+        w2 = prmt(r[2], r[3], 0x5410);
+        w3 = prmt(r[2], r[3], 0x7632);
       }
       // partial sum of this lane's 8 dims of head g, then over the 4 lanes of the group
       float part = 0.f;
@@ -1061,36 +1075,71 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     __syncthreads();
   }
 
-  // ---- fused decode step: the last CTA of this (batch row, KV head) to
-  //      finish merges the S split partials of the group's G heads into the
+  // ---- fused decode step: the last CTAs of this (batch row, KV head) to
+  //      finish merge the S split partials of the group's G heads into the
   //      output (the arithmetic of kvq_combine, with the inverse rotation of a
-  //      turbo3 value cache).  The arrival counter wraps to 0 at S.
+  //      turbo3 value cache).  Arrivals are counted modulo S (the counter
+  //      returns to 0).  The last arrival (rank 0) may combine at once; the
+  //      arrivals of rank 1 .. comb_ctas-1 wait for it through the group's epoch
+  //      word, which rank 0 bumps once every partial is visible, so the G heads
+  //      are combined by comb_ctas CTAs at a time.  (The host enables that only
+  //      when the waiting CTAs leave most of the GPU's CTA slots free, so the
+  //      CTAs they wait for can always run; each wait is bounded.)
   if (p.out != nullptr) {
-    __shared__ unsigned int last_cta;
+    __shared__ unsigned int comb_rank;
+    __shared__ int comb_wait_failed;
     __threadfence();  // this CTA's partials are visible device-wide ...
     __syncthreads();
-    if (threadIdx.x == 0)  // ... before its arrival is counted
-      last_cta = atomicInc(p.counters + plane, (unsigned)(p.S - 1)) == (unsigned)(p.S - 1);
+    if (threadIdx.x == 0) {  // ... before its arrival is counted
+      // the epoch is read before this CTA arrives: rank 0 bumps it only after
+      // the last arrival, so a waiter cannot miss the bump
+      const unsigned int e0 = p.comb_ctas > 1 ? *reinterpret_cast<volatile unsigned int*>(p.epochs + plane) : 0u;
+      if (p.comb_ctas > 1) __threadfence();
+      const unsigned int ticket = atomicInc(p.counters + plane, (unsigned)(p.S - 1));
+      const unsigned int rank = (unsigned)(p.S - 1) - ticket;
+      int failed = 0;
+      if (rank == 0) {
+        __threadfence();
+        if (p.comb_ctas > 1) atomicAdd(p.epochs + plane, 1u);
+      } else if ((int)rank < p.comb_ctas) {
+        const unsigned long long w0 = global_ns();
+        while (*reinterpret_cast<volatile unsigned int*>(p.epochs + plane) == e0) {
+          if (global_ns() - w0 > kWaitLimitNs) {
+            failed = 1;
+            break;
+          }
+          __nanosleep(64);
+        }
+        __threadfence();
+      }
+      comb_rank = rank;
+      comb_wait_failed = failed;
+    }
     __syncthreads();
-    if (last_cta) {
+    const int rank = (int)comb_rank;
+    if (rank < p.comb_ctas) {
       __threadfence();
-      // The partials of the group (G heads x S splits x D floats) come into the
-      // free stage memory by bulk copies, one per head and round of up to 32
-      // splits; m and l are read alongside.  One warp per head then folds the
-      // round into its running (max, sum, weighted acc), D/32 consecutive dims
-      // per lane.
+      // the partials were written through the generic proxy by other CTAs and
+      // are read here by bulk copies (the async proxy)
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      // This CTA's heads [h0, h0 + nh) of the group.  Their partials (nh heads x
+      // S splits x D floats) come into the free stage memory by bulk copies,
+      // one per head and round of up to 64 splits; m and l are read alongside.
+      // One warp per head then folds the round into its running (max, sum,
+      // weighted acc), D/32 consecutive dims per lane.
       constexpr int E = D / 32;                        // dims per lane
       constexpr int HPW = (16 + L::NW - 1) / L::NW;    // heads per warp, G <= 16
       constexpr int kAvail = L::NW * L::WARP / 4;      // floats of stage memory
       const int G = p.G, S_ = p.S;
-      float* buf = reinterpret_cast<float*>(smem);     // [G][SC][D]
-      const int SC = max(1, min(32, min(S_, kAvail / (G * D))));
-      const int64_t grow0 = ((int64_t)b * p.n_q + (int64_t)kvh * G) * S_;  // (head 0, split 0)
+      const int h0 = rank * G / p.comb_ctas, nh = (rank + 1) * G / p.comb_ctas - h0;
+      float* buf = reinterpret_cast<float*>(smem);     // [nh][SC][D]
+      const int SC = max(1, min(64, min(S_, kAvail / (nh * D))));
+      const int64_t grow0 = ((int64_t)b * p.n_q + (int64_t)kvh * G + h0) * S_;  // (head h0, split 0)
       // one mbarrier for the rounds' bulk copies (the pipeline's are idle now)
       __shared__ uint64_t comb_bar[1];
       uint64_t* cbar = comb_bar;
       uint32_t cphase = 0;
-      int comb_failed = 0;
+      int comb_failed = comb_wait_failed;
       if (threadIdx.x == 0) {
         mbar_init(cbar, 1);
         fence_barrier_init();
@@ -1105,29 +1154,35 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 #pragma unroll
         for (int e = 0; e < E; ++e) num[hi][e] = 0.f;
       }
-      for (int s0 = 0; s0 < S_; s0 += SC) {
+      for (int s0 = 0; !comb_failed && s0 < S_; s0 += SC) {  // comb_failed is uniform
         const int sc = min(SC, S_ - s0);
         if (threadIdx.x == 0) {
-          mbar_expect_tx(cbar, (uint32_t)(G * sc * D * 4));
-          for (int h = 0; h < G; ++h)
-            bulk_load(buf + h * SC * D, p.ws_acc + (grow0 + (int64_t)h * S_ + s0) * D, (uint32_t)(sc * D * 4), cbar);
+          mbar_expect_tx(cbar, (uint32_t)(nh * sc * D * 4));
+          for (int hl = 0; hl < nh; ++hl)
+            bulk_load(buf + hl * SC * D, p.ws_acc + (grow0 + (int64_t)hl * S_ + s0) * D, (uint32_t)(sc * D * 4),
+                      cbar);
         }
-        float mj[HPW], lj[HPW];  // this round's m, l of split s0 + lane
+        // this round's m, l of splits s0 + lane and s0 + 32 + lane
+        float mj[HPW][2], lj[HPW][2];
 #pragma unroll
         for (int hi = 0; hi < HPW; ++hi) {
-          const int h = warp + hi * L::NW;
-          mj[hi] = -INFINITY;
-          lj[hi] = 0.f;
-          if (h < G && lane < sc) {
-            mj[hi] = __ldcg(p.ws_m + grow0 + (int64_t)h * S_ + s0 + lane);
-            lj[hi] = __ldcg(p.ws_l + grow0 + (int64_t)h * S_ + s0 + lane);
+          const int hl = warp + hi * L::NW;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int j = lane + 32 * u;
+            mj[hi][u] = -INFINITY;
+            lj[hi][u] = 0.f;
+            if (hl < nh && j < sc) {
+              mj[hi][u] = __ldcg(p.ws_m + grow0 + (int64_t)hl * S_ + s0 + j);
+              lj[hi][u] = __ldcg(p.ws_l + grow0 + (int64_t)hl * S_ + s0 + j);
+            }
           }
         }
         const bool landed = mbar_wait(cbar, cphase);
         if (!__syncthreads_and(landed)) {
           // a copy did not land within the limit: let it drain (bounded
           // again) so nothing writes shared memory after the CTA exits; the
-          // group's outputs read NaN
+          // heads' outputs read NaN
           if (threadIdx.x == 0) (void)mbar_wait(cbar, cphase);
           __syncthreads();
           comb_failed = 1;
@@ -1136,24 +1191,28 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         cphase ^= 1u;
 #pragma unroll
         for (int hi = 0; hi < HPW; ++hi) {
-          const int h = warp + hi * L::NW;
-          if (h >= G) break;
-          float mc = mj[hi];
+          const int hl = warp + hi * L::NW;
+          if (hl >= nh) break;
+          float mc = fmaxf(mj[hi][0], mj[hi][1]);
 #pragma unroll
           for (int o = 16; o >= 1; o >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
           const float mn = fmaxf(Mh[hi], mc);
           // an empty split (m = -inf) weighs 0; so does the old state while no split had rows
           const float alpha = Mh[hi] == -INFINITY ? 0.f : exp2f(Mh[hi] - mn);
-          const float wl = mj[hi] == -INFINITY ? 0.f : exp2f(mj[hi] - mn);
-          float dl = wl * lj[hi];
+          float wl[2], dl = 0.f;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            wl[u] = mj[hi][u] == -INFINITY ? 0.f : exp2f(mj[hi][u] - mn);
+            dl += wl[u] * lj[hi][u];
+          }
 #pragma unroll
           for (int o = 16; o >= 1; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
           den[hi] = fmaf(den[hi], alpha, dl);
 #pragma unroll
           for (int e = 0; e < E; ++e) num[hi][e] *= alpha;
-          const float* hb = buf + h * SC * D + lane * E;
+          const float* hb = buf + hl * SC * D + lane * E;
           for (int j = 0; j < sc; ++j) {
-            const float wj = __shfl_sync(0xffffffffu, wl, j);
+            const float wj = __shfl_sync(0xffffffffu, j < 32 ? wl[0] : wl[1], j & 31);
 #pragma unroll
             for (int e4 = 0; e4 < E; e4 += 2) {
               const float2 x2 = *reinterpret_cast<const float2*>(hb + j * D + e4);
@@ -1168,8 +1227,9 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       }
 #pragma unroll
       for (int hi = 0; hi < HPW; ++hi) {
-        const int h = warp + hi * L::NW;
-        if (h >= G) break;
+        const int hl = warp + hi * L::NW;
+        if (hl >= nh) break;
+        const int h = h0 + hl;
         float o_v[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) o_v[e] = comb_failed ? __int_as_float(0x7fc00000) : num[hi][e] / den[hi];

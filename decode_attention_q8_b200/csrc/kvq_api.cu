@@ -166,6 +166,24 @@ int32_t choose_splits(int64_t units, int64_t ctx, int sms, int per_sm) {
 
 int64_t chunk_rows(int64_t ctx, int32_t S) { return round_up((ctx + S - 1) / S, kSplitAlign); }
 
+// CTAs per (batch row, KV head) that share the fused step's combine: the last
+// arrivals, one per 48 (head, split) partials of the group (at most one per
+// head), once a group has more than 200 of them.  Waking a waiting CTA costs
+// about a microsecond, which pays only when one CTA would pull the partials
+// through its shared memory in several rounds (measured: 8 heads x 37 splits
+// 0.6-0.9 us faster; 4 x 37 and 8 x 9 as fast or slower).  All but the last
+// arrival wait for it, so the waiting CTAs may hold at most half of the GPU's
+// CTA slots; the CTAs they wait for can then always be scheduled.
+int32_t combining_ctas(const kvq_cache_desc* d, int32_t batch, int32_t S) {
+  const int32_t G = d->n_q_heads / d->n_kv_heads;
+  const int64_t groups = (int64_t)batch * d->n_kv_heads;
+  const int64_t slots = (int64_t)sm_count() * decode_ctas_per_sm(d->k_type, d->v_type, d->head_dim);
+  if ((int64_t)G * S <= 200) return 1;
+  int32_t k = (int32_t)std::min<int64_t>(G, (int64_t)G * S / 48);
+  while (k > 1 && (int64_t)(k - 1) * groups * 2 > slots) --k;
+  return std::max(k, 1);
+}
+
 // Upper bound of the automatic split count over ctx_len <= ctx (sizes the
 // workspace for n_splits = 0).
 int32_t auto_splits_bound(const kvq_cache_desc* d, int32_t batch, int64_t ctx) {
@@ -186,13 +204,14 @@ struct WsLayout {
   int64_t m_off, l_off, acc_off, cnt_off, total;
 };
 
-// Counters first: their place depends on batch and n_kv only, so calls with
-// different split counts on one workspace keep them intact.
+// Counters first (arrival counters, then epoch words, one of each per group):
+// their place depends on batch and n_kv only, so calls with different split
+// counts on one workspace keep them intact.
 WsLayout ws_layout(const kvq_cache_desc* d, int32_t batch, int32_t S) {
   WsLayout w;
   const int64_t rows = (int64_t)batch * d->n_q_heads * S;
   w.cnt_off = 0;
-  w.m_off = round_up((int64_t)batch * d->n_kv_heads * 4, 256);
+  w.m_off = round_up((int64_t)batch * d->n_kv_heads * 8, 256);
   w.l_off = w.m_off + round_up(rows * 4, 256);
   w.acc_off = w.l_off + round_up(rows * 4, 256);
   w.total = w.acc_off + rows * d->head_dim * 4;
@@ -337,6 +356,8 @@ kvq_status step_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, cons
   }
   p.out = out;
   p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + w.cnt_off);
+  p.epochs = p.counters + (int64_t)batch * d->n_kv_heads;
+  p.comb_ctas = combining_ctas(d, batch, p.S);
   const cudaError_t e = launch_decode(d->k_type, d->v_type, p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return KVQ_OK;

@@ -72,6 +72,8 @@ struct DecodeParams {
   AppendParams app_v;
   float* out;            // [B][n_q][D] combined output, or null (partials only)
   uint32_t* counters;    // [B][n_kv] split arrival counters, zero between calls
+  uint32_t* epochs;      // [B][n_kv] bumped by each group's last arrival (any start value)
+  int32_t comb_ctas;     // CTAs per group that combine (the last arrivals), 1 .. G
 };
 
 struct CombineParams {

@@ -152,10 +152,10 @@ KVQ_API int32_t kvq_auto_splits(const kvq_cache_desc* desc, int32_t batch, int64
 
 /* Workspace bytes kvq_decode_attention / kvq_combine / kvq_decode_step need
  * for n_splits (0 = automatic, resolved as kvq_auto_splits would for ctx_len =
- * max_ctx); 0 on error.  Layout: uint32 counters [batch][n_kv_heads] (used by
- * kvq_decode_step only; their place does not depend on n_splits), then m and l
- * fp32 [batch][n_q][S] each, then acc fp32 [batch][n_q][S][head_dim], each part
- * 256-byte aligned. */
+ * max_ctx); 0 on error.  Layout: uint32 arrival counters [batch][n_kv_heads]
+ * and uint32 epoch words [batch][n_kv_heads] (used by kvq_decode_step only;
+ * their place does not depend on n_splits), then m and l fp32 [batch][n_q][S]
+ * each, then acc fp32 [batch][n_q][S][head_dim], each part 256-byte aligned. */
 KVQ_API size_t kvq_workspace_bytes(const kvq_cache_desc* desc, int32_t batch, int32_t n_splits);
 
 /* The turbo3 codebook this library uses: 8 binary32 levels (ascending) and
@@ -248,10 +248,11 @@ KVQ_API kvq_status kvq_decode_attention_noalloc(const kvq_cache_desc* desc, cons
  *   out            device fp32 [batch][n_q_heads][head_dim], 16-byte aligned
  *   other arguments as in kvq_decode_attention; ctx_len counts the new row.
  * The CTA whose split holds row ctx_len - 1 writes the new rows before it reads
- * any cache row; the last CTA of each (batch, KV head) to finish combines the
- * group's splits.  The workspace counters (see kvq_workspace_bytes) must be zero
- * before the first call with a workspace; every completed call leaves them
- * zero.  Calls sharing a workspace must be ordered (one stream).
+ * any cache row; the last CTAs of each (batch, KV head) to finish combine the
+ * group's splits, a share of its query heads each.  The workspace's arrival
+ * counters (see kvq_workspace_bytes) must be zero before the first call with a
+ * workspace, and every completed call leaves them zero; the epoch words may
+ * hold any value.  Calls sharing a workspace must be ordered (one stream).
  * Cached bytes are identical to kvq_append_quantize's; out agrees with
  * kvq_decode_attention + kvq_combine up to fp32 rounding order.
  */

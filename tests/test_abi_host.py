@@ -231,8 +231,9 @@ def test_workspace_bytes_formula():
     B, S = 4, 9
     rows = B * 64 * S
     r256 = lambda v: (v + 255) // 256 * 256
-    # the fused step's counters [B][n_kv] (uint32), then m, l, acc, each part 256-aligned
-    assert kvq.kvq_workspace_bytes(d, B, S) == r256(B * 8 * 4) + 2 * r256(rows * 4) + rows * 128 * 4
+    # the fused step's arrival counters and epoch words, [B][n_kv] uint32 each, then m, l, acc,
+    # each part 256-aligned
+    assert kvq.kvq_workspace_bytes(d, B, S) == r256(B * 8 * 8) + 2 * r256(rows * 4) + rows * 128 * 4
     assert kvq.kvq_workspace_bytes(d, 0, S) == 0
     # the automatic split count never needs more workspace than n_splits = 0 reserves
     auto_ws = kvq.kvq_workspace_bytes(d, B, 0)

@@ -209,3 +209,29 @@ def test_many_splits_and_empty_ones(S):
     out = _step(desc, kc, vc, q, k, v, B, ctx, 0.09, S, ws)
     _check_out(desc, q, k, v, out, ctx, 0.09, f"S={S}")
     assert not ws[:4 * B * n_kv].cpu().numpy().any()
+
+
+@pytest.mark.parametrize("B,n_q,n_kv", [(1, 64, 8), (1, 16, 1), (2, 48, 4), (64, 32, 8)])
+def test_combine_shared_by_the_last_arrivals(B, n_q, n_kv):
+    """With many (head, split) partials per group the last arrivals share the
+    combine, a share of the G heads each (at batch 64 the waiting CTAs would
+    hold too many slots, so one CTA combines): every head matches the oracle,
+    whatever value the epoch words held before, over consecutive calls on one
+    workspace, with automatic and with 40 explicit splits."""
+    D, ctx = 128, 16384
+    desc, q, k, v = _inputs("q8_0", "q4_0", B, n_q, n_kv, D, ctx, seed=B + n_q)
+    kc, vc = alloc_cache(desc, B, 0), alloc_cache(desc, B, 1)
+    kvq.kvq_append_quantize(desc, kc, vc, k[:, :ctx - 1].contiguous(), v[:, :ctx - 1].contiguous(), B, 0, ctx - 1)
+    scale = 1 / math.sqrt(D)
+    groups = [(b, g) for b in range(B) for g in range(n_kv)]
+    if B > 4:
+        groups = [(0, 0), (B // 2, 3), (B - 1, n_kv - 1)]
+    for S in (0, 40):
+        ws = _workspace(desc, B, S)
+        words = ws.view(torch.int32)
+        words[B * n_kv:2 * B * n_kv] = torch.randint(-2**31, 2**31 - 1, (B * n_kv,), dtype=torch.int32,
+                                                     device="cuda")
+        for call in range(2):
+            out = _step(desc, kc, vc, q, k, v, B, ctx, scale, S, ws)
+            _check_out(desc, q, k, v, out, ctx, scale, f"B{B} G{n_q // n_kv} S={S} call {call}", groups=groups)
+            assert not ws[:4 * B * n_kv].cpu().numpy().any()
