@@ -35,6 +35,8 @@ EXPORTED = (
     "kvq_turbo3_codebook", "kvq_turbo3_signs", "kvq_append_quantize",
     "kvq_decode_attention", "kvq_combine", "kvq_decode_attention_noalloc", "kvq_decode_step",
     "kvq_decode_attention_varlen", "kvq_decode_step_varlen", "kvq_append_quantize_varlen",
+    "kvq_paged_layout", "kvq_paged_cache_bytes", "kvq_append_quantize_paged", "kvq_decode_attention_paged",
+    "kvq_decode_step_paged",
 )
 
 
@@ -61,8 +63,18 @@ class kvq_plane_layout(ctypes.Structure):
     ]
 
 
+class kvq_paged(ctypes.Structure):
+    _fields_ = [
+        ("block_table", ctypes.c_void_p),
+        ("max_pages", ctypes.c_int32),
+        ("page_rows", ctypes.c_int32),
+        ("n_pages", ctypes.c_int64),
+    ]
+
+
 _P = ctypes.c_void_p
 _D = ctypes.POINTER(kvq_cache_desc)
+_PG = ctypes.POINTER(kvq_paged)
 _sigs = {
     "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvq_last_cuda_error": (ctypes.c_char_p, []),
@@ -89,6 +101,15 @@ _sigs = {
     "kvq_decode_step_varlen": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, ctypes.c_int32, _P, ctypes.c_int64,
                                               ctypes.c_float, ctypes.c_int32, _P, ctypes.c_size_t, _P, _P]),
     "kvq_append_quantize_varlen": (ctypes.c_int, [_D, _P, _P, _P, _P, ctypes.c_int32, _P, ctypes.c_int32, _P]),
+    "kvq_paged_layout": (ctypes.c_int, [_D, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                                        ctypes.POINTER(kvq_plane_layout)]),
+    "kvq_paged_cache_bytes": (ctypes.c_size_t, [_D, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32]),
+    "kvq_append_quantize_paged": (ctypes.c_int, [_D, _P, _P, _P, _P, ctypes.c_int32, _PG, _P, ctypes.c_int32,
+                                                 _P]),
+    "kvq_decode_attention_paged": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, _PG, _P, ctypes.c_int64,
+                                                  ctypes.c_float, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
+    "kvq_decode_step_paged": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, ctypes.c_int32, _PG, _P, ctypes.c_int64,
+                                             ctypes.c_float, ctypes.c_int32, _P, ctypes.c_size_t, _P, _P]),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -262,6 +283,54 @@ def kvq_decode_step_varlen(desc, k_cache, v_cache, q, k_new, v_new, batch, ctx_l
                                               softmax_scale, n_splits, _ptr(workspace), workspace_bytes, _ptr(out),
                                               _stream(stream)),
                   "kvq_decode_step_varlen")
+
+
+def make_paged(block_table, page_rows, n_pages):
+    """kvq_paged for a device int32 block table [batch][max_pages] (the caller
+    keeps the tensor alive while the description is in use)."""
+    assert block_table.dtype.itemsize == 4 and block_table.dim() == 2 and block_table.is_contiguous()
+    return kvq_paged(block_table.data_ptr(), block_table.shape[1], page_rows, n_pages)
+
+
+def kvq_paged_layout(desc, page_rows, n_pages, which):
+    out = kvq_plane_layout()
+    _check(_lib.kvq_paged_layout(ctypes.byref(desc), page_rows, n_pages, which, ctypes.byref(out)),
+           "kvq_paged_layout")
+    return out
+
+
+def kvq_paged_cache_bytes(desc, page_rows, n_pages, which):
+    return _lib.kvq_paged_cache_bytes(ctypes.byref(desc), page_rows, n_pages, which)
+
+
+def kvq_append_quantize_paged(desc, k_pool, v_pool, k_new, v_new, batch, pages, lens, n_tok, stream=None):
+    """Append n_tok rows per sequence at logical rows lens[b] - n_tok .. lens[b] - 1
+    of a paged pool (``pages``: kvq_paged)."""
+    return _check(_lib.kvq_append_quantize_paged(ctypes.byref(desc), _ptr(k_pool), _ptr(v_pool), _ptr(k_new),
+                                                 _ptr(v_new), batch, ctypes.byref(pages), _ptr(lens), n_tok,
+                                                 _stream(stream)),
+                  "kvq_append_quantize_paged")
+
+
+def kvq_decode_attention_paged(desc, k_pool, v_pool, q, batch, pages, ctx_lens, max_ctx_len, softmax_scale,
+                               n_splits, workspace, workspace_bytes=None, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return _check(_lib.kvq_decode_attention_paged(ctypes.byref(desc), _ptr(k_pool), _ptr(v_pool), _ptr(q), batch,
+                                                  ctypes.byref(pages), _ptr(ctx_lens), max_ctx_len, softmax_scale,
+                                                  n_splits, _ptr(workspace), workspace_bytes, _stream(stream)),
+                  "kvq_decode_attention_paged")
+
+
+def kvq_decode_step_paged(desc, k_pool, v_pool, q, k_new, v_new, batch, pages, ctx_lens, max_ctx_len, softmax_scale,
+                          n_splits, workspace, out, workspace_bytes=None, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return _check(_lib.kvq_decode_step_paged(ctypes.byref(desc), _ptr(k_pool), _ptr(v_pool), _ptr(q), _ptr(k_new),
+                                             _ptr(v_new), batch, ctypes.byref(pages), _ptr(ctx_lens), max_ctx_len,
+                                             softmax_scale, n_splits, _ptr(workspace), workspace_bytes, _ptr(out),
+                                             _stream(stream)),
+                  "kvq_decode_step_paged")
 
 
 def raw_status(name, *args):

@@ -64,7 +64,8 @@ __device__ __forceinline__ float raw_elem(const uint4& r, int i) {  // fp16 elem
 }
 
 // Destination row index of flat input row `row` = ((b * n_tok + t) * H + h),
-// or -1 when batch row b's length (per-sequence lengths) is out of range.
+// or -1 when batch row b's length (per-sequence lengths) is out of range or
+// its page id (paged pool) is not a page of the pool.
 // 32-bit division when the call's rows fit (the 64-bit one is a long routine).
 __device__ __forceinline__ int64_t dst_row(const AppendParams& p, int64_t row) {
   int64_t h, t, b;
@@ -85,7 +86,13 @@ __device__ __forceinline__ int64_t dst_row(const AppendParams& p, int64_t row) {
     if (len < p.n_tok || len > p.len_max) return -1;
     pos = len - p.n_tok;
   }
-  return (b * p.H + h) * p.dst.T + pos + t;
+  const int64_t lr = pos + t;  // logical row of sequence b
+  if (p.block_table != nullptr) {
+    const int64_t pg = p.block_table[b * p.max_pages + (lr >> p.log2_page)];
+    if (pg < 0 || pg >= p.n_pages) return -1;
+    return (pg * p.H + h) * p.dst.T + (lr & ((1ll << p.log2_page) - 1));
+  }
+  return (b * p.H + h) * p.dst.T + lr;
 }
 
 // log2 of the 32-element blocks per row (head_dim is 32 times a power of two)

@@ -130,9 +130,12 @@ int decode_ctas_per_sm(int32_t k_type, int32_t v_type, int32_t D) {
 
 cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p, cudaStream_t st) {
   tc::TcMaps maps;
-  const int64_t planes = (int64_t)p.B * p.n_kv;
-  if (!plane_maps(p.k, k_type, planes, p.ctx, &maps.kc, &maps.ks) ||
-      !plane_maps(p.v, v_type, planes, p.ctx, &maps.vc, &maps.vs))
+  // a paged pool is a cache of n_pages "batch rows" of one page each
+  const bool paged = p.block_table != nullptr;
+  const int64_t planes = (paged ? p.n_pages : (int64_t)p.B) * p.n_kv;
+  const int64_t rows = paged ? ((int64_t)1 << p.log2_page) : p.ctx;
+  if (!plane_maps(p.k, k_type, planes, rows, &maps.kc, &maps.ks) ||
+      !plane_maps(p.v, v_type, planes, rows, &maps.vc, &maps.vs))
     return cudaErrorInvalidValue;
   tc::TcArgs a;
   a.p = p;

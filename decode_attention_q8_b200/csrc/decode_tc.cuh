@@ -311,7 +311,9 @@ struct TcArgs {
   DecodeParams p;
 };
 
-template <int KT, int VT, int NB, int NTH>
+// PAGED: the cache planes are pages of a pool, reached through the block table
+// (a separate instantiation, so the contiguous kernel carries none of it).
+template <int KT, int VT, int NB, int NTH, bool PAGED>
 __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
                                   (NB >= 8 || NTH == 2 || ctas_per_sm_for(KT, VT, NB * 32) < 2) ? 1 : 2)
     decode_tc_kernel(const TcArgs args, const __grid_constant__ CUtensorMap tm_kc,
@@ -338,7 +340,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::NW * L::WARP + L::TABLE) + warp * S;
 
   const int s_idx = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  // rows of this batch row, and its split length (a multiple of 16 rows)
+  // rows of this batch row, and its split length (whole 32-row tiles)
   int64_t ctx = p.ctx, chunk = p.chunk, append_pos = p.append_pos;
   if (p.ctx_lens != nullptr) {
     const int64_t len = p.ctx_lens[b];
@@ -385,6 +387,19 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     }
   }
 
+  // Paged pool: the page of each of this warp's tiles, a window of 32 tiles
+  // per register (lane i: tile j0 + i), read with the queries, before any tile
+  // is requested; the next window is read 32 tiles ahead of its first use.
+  constexpr bool paged = PAGED;
+  const int my_tiles = n_sub > warp ? (n_sub - warp + L::NW - 1) / L::NW : 0;
+  auto page_load = [&](int j0) -> int {  // page id of tile j0 + lane (0 past the last tile)
+    const int j = j0 + lane;
+    if (!paged || j >= my_tiles) return 0;
+    const int r0 = t0 + kSub * (warp + L::NW * j);
+    return p.block_table[(int64_t)b * p.max_pages + (r0 >> p.log2_page)];
+  };
+  int pg_win = page_load(0), pg_next = my_tiles > 32 ? page_load(32) : 0;
+
   if (threadIdx.x == 0) cta_failed = 0;
   if (lane == 0) {
 #pragma unroll
@@ -405,28 +420,45 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   auto ks_of = [&](int st) { return wbase + S * (L::KC + L::VC) + st * L::KS; };
   auto vs_of = [&](int st) { return wbase + S * (L::KC + L::VC + L::KS) + st * L::VS; };
 
-  // tile j of this warp covers rows t0 + 32*(warp + NW*j) ...
-  const int my_tiles = n_sub > warp ? (n_sub - warp + L::NW - 1) / L::NW : 0;
+  // tile j of this warp covers rows t0 + 32*(warp + NW*j) ... (logical rows of
+  // the sequence; in a paged pool, page pg's rows from r0 mod the page size)
   const uint64_t pol = l2_evict_first_policy();
-  auto issue = [&](int j, int st) {
-    const int r0 = t0 + kSub * (warp + L::NW * j);
+  // an id that is not a page of the pool: load page 0 instead, partials NaN
+  auto page_ok = [&](int pg) -> int {
+    if (pg < 0 || pg >= p.n_pages) {
+      atomicExch(&cta_failed, 1);
+      return 0;
+    }
+    return pg;
+  };
+  if (paged) {
+    pg_win = page_ok(pg_win);
+    pg_next = page_ok(pg_next);
+  }
+  auto issue = [&](int j, int st, int pg) {
+    int r0 = t0 + kSub * (warp + L::NW * j);
+    int tplane = plane;
+    if (paged) {
+      r0 &= (1 << p.log2_page) - 1;
+      tplane = pg * p.n_kv + kvh;
+    }
     mbar_expect_tx(&bars[st], L::TX);
     if (L::RBK > 128)
-      tma_load_4d(kc_of(st), &tm_kc, 0, 0, r0, plane, &bars[st], pol);
+      tma_load_4d(kc_of(st), &tm_kc, 0, 0, r0, tplane, &bars[st], pol);
     else
-      tma_load_3d(kc_of(st), &tm_kc, 0, r0, plane, &bars[st], pol);
-    if (L::NSK) tma_load_2d(ks_of(st), &tm_ks, r0 * L::NSK / 2, plane, &bars[st], pol);
+      tma_load_3d(kc_of(st), &tm_kc, 0, r0, tplane, &bars[st], pol);
+    if (L::NSK) tma_load_2d(ks_of(st), &tm_ks, r0 * L::NSK / 2, tplane, &bars[st], pol);
     if (VT == KVQ_TURBO3) {
       if (kSub * L::RBV / 4 <= 256)
-        tma_load_2d(vc_of(st), &tm_vc, r0 * L::RBV / 4, plane, &bars[st], pol);
+        tma_load_2d(vc_of(st), &tm_vc, r0 * L::RBV / 4, tplane, &bars[st], pol);
       else
-        tma_load_3d(vc_of(st), &tm_vc, 0, r0, plane, &bars[st], pol);
+        tma_load_3d(vc_of(st), &tm_vc, 0, r0, tplane, &bars[st], pol);
     } else if (L::RBV > 128) {
-      tma_load_4d(vc_of(st), &tm_vc, 0, 0, r0, plane, &bars[st], pol);
+      tma_load_4d(vc_of(st), &tm_vc, 0, 0, r0, tplane, &bars[st], pol);
     } else {
-      tma_load_3d(vc_of(st), &tm_vc, 0, r0, plane, &bars[st], pol);
+      tma_load_3d(vc_of(st), &tm_vc, 0, r0, tplane, &bars[st], pol);
     }
-    if (L::NSV) tma_load_2d(vs_of(st), &tm_vs, r0 * L::NSV / 2, plane, &bars[st], pol);
+    if (L::NSV) tma_load_2d(vs_of(st), &tm_vs, r0 * L::NSV / 2, tplane, &bars[st], pol);
   };
   // Fused decode step: the new row (row append_pos) lies in tile jt of warp wt
   // of the CTA whose split holds it.  That warp issues its other first tiles,
@@ -436,9 +468,10 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   const bool owner = append_pos >= t0l && append_pos < t1l;
   const int t_new = owner ? (int)(append_pos - t0l) / kSub : -1;
   const int wt = owner ? t_new % L::NW : -1, jt = owner ? t_new / L::NW : -1;
-  if (lane == 0) {
-    for (int j = 0; j < S && j < my_tiles; ++j)
-      if (!(warp == wt && j == jt)) issue(j, j);
+#pragma unroll
+  for (int j = 0; j < S; ++j) {
+    const int pg = paged ? __shfl_sync(0xffffffffu, pg_win, j) : 0;
+    if (lane == 0 && j < my_tiles && !(warp == wt && j == jt)) issue(j, j, pg);
   }
   if (warp == wt) {
     constexpr int rk = rows::row_threads(KT, D), rv = rows::row_threads(VT, D);
@@ -451,7 +484,8 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     __threadfence();
     asm volatile("fence.proxy.async.global;" ::: "memory");
     __syncwarp();
-    if (lane == 0 && jt < S && jt < my_tiles) issue(jt, jt);
+    const int pgt = paged ? __shfl_sync(0xffffffffu, pg_win, jt & 31) : 0;
+    if (lane == 0 && jt < S && jt < my_tiles) issue(jt, jt, pgt);
   }
 
   // ---- queries: B fragments of Q^T per (block, k-step) and, for quantized
@@ -938,9 +972,18 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 
     // release the stage and refill it with this warp's tile j + S
     __syncwarp();
+    int pg = 0;
+    if (paged) {
+      const int jn = j + S;
+      if ((jn & 31) == 0 && jn < my_tiles) {  // next window: read the one after it
+        pg_win = pg_next;
+        pg_next = page_ok(page_load(jn + 32));
+      }
+      pg = __shfl_sync(0xffffffffu, pg_win, jn & 31);
+    }
     if (lane == 0 && j + S < my_tiles) {
       fence_proxy_async();
-      issue(j + S, st);
+      issue(j + S, st, pg);
     }
     if (++st == S) {
       st = 0;
@@ -1281,10 +1324,10 @@ struct TcMaps {
   CUtensorMap kc, ks, vc, vs;
 };
 
-template <int KT, int VT, int NB, int NTH>
+template <int KT, int VT, int NB, int NTH, bool PAGED>
 cudaError_t launch_one(const TcArgs& a, const TcMaps& m, cudaStream_t st) {
   using L = Layout<KT, VT, NB * 32>;
-  auto kern = decode_tc_kernel<KT, VT, NB, NTH>;
+  auto kern = decode_tc_kernel<KT, VT, NB, NTH, PAGED>;
   static bool attr_set = false;  // idempotent; a race only repeats the call
   if (!attr_set) {
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
@@ -1298,7 +1341,9 @@ cudaError_t launch_one(const TcArgs& a, const TcMaps& m, cudaStream_t st) {
 
 template <int KT, int VT, int NB>
 cudaError_t launch_nb(int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st) {
-  return nth == 1 ? launch_one<KT, VT, NB, 1>(a, m, st) : launch_one<KT, VT, NB, 2>(a, m, st);
+  if (a.p.block_table != nullptr)
+    return nth == 1 ? launch_one<KT, VT, NB, 1, true>(a, m, st) : launch_one<KT, VT, NB, 2, true>(a, m, st);
+  return nth == 1 ? launch_one<KT, VT, NB, 1, false>(a, m, st) : launch_one<KT, VT, NB, 2, false>(a, m, st);
 }
 
 template <int KT, int VT>

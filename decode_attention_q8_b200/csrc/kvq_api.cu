@@ -192,7 +192,7 @@ int32_t auto_splits_bound(const kvq_cache_desc* d, int32_t batch, int64_t ctx) {
 }
 
 // Explicit counts are used as given (trailing splits may be empty); the
-// automatic count drops the splits that rounding the chunk to 16 rows leaves
+// automatic count drops the splits that rounding the chunk to 32 rows leaves
 // empty, so it never exceeds auto_splits_bound(max_ctx).
 int32_t resolve_splits(const kvq_cache_desc* d, int32_t batch, int64_t ctx, int32_t n_splits) {
   if (n_splits > 0) return n_splits;
@@ -218,6 +218,56 @@ WsLayout ws_layout(const kvq_cache_desc* d, int32_t batch, int32_t S) {
   return w;
 }
 
+// Byte layout of `planes` planes of T rows of a tensor of `type`.
+void fill_layout(int32_t type, int32_t D, int64_t planes, int64_t T, kvq_plane_layout* out) {
+  const int64_t cb = code_bytes_of(type, D);
+  const int64_t ns = n_scales_of(type, D);
+  out->rows_per_plane = T;
+  out->code_bytes = cb;
+  out->n_scales = ns;
+  out->scale_offset = round_up(planes * T * cb, 256);
+  out->total_bytes = out->scale_offset + planes * T * ns * 2;
+}
+
+// A paged pool's layout: the contiguous layout with the pages as batch rows and
+// the page rows as the rows per plane.
+kvq_status check_pool(const kvq_cache_desc* d, int32_t page_rows, int64_t n_pages) {
+  if (n_pages < 1) return KVQ_ERR_INVALID;
+  if (page_rows < 32 || page_rows > (1 << 20) || !pow2(page_rows)) return KVQ_ERR_UNSUPPORTED;
+  if (n_pages * d->n_kv_heads >= ((int64_t)1 << 31)) return KVQ_ERR_UNSUPPORTED;  // 32-bit plane coordinates
+  const double approx = (double)n_pages * d->n_kv_heads * (double)page_rows * (2.0 * d->head_dim + 16.0);
+  if (approx > 9.0e18) return KVQ_ERR_INVALID;
+  return KVQ_OK;
+}
+
+kvq_status check_paged(const kvq_cache_desc* d, const kvq_paged* pg) {
+  if (!pg || !pg->block_table || !aligned(pg->block_table, 4) || pg->max_pages < 1) return KVQ_ERR_INVALID;
+  return check_pool(d, pg->page_rows, pg->n_pages);
+}
+
+int32_t log2_of(int64_t v) {
+  int32_t l = 0;
+  while (((int64_t)1 << l) < v) ++l;
+  return l;
+}
+
+// Longest sequence a paged pool's block table can address, within max_ctx.
+int64_t paged_capacity(const kvq_cache_desc* d, const kvq_paged* pg) {
+  return std::min<int64_t>(d->max_ctx, (int64_t)pg->max_pages * pg->page_rows);
+}
+
+Plane pool_plane_of(const kvq_cache_desc* d, const kvq_paged* pg, int which, void* base) {
+  kvq_plane_layout L;
+  fill_layout(which ? d->v_type : d->k_type, d->head_dim, pg->n_pages * d->n_kv_heads, pg->page_rows, &L);
+  Plane p;
+  p.codes = static_cast<uint8_t*>(base);
+  p.scales = reinterpret_cast<__half*>(static_cast<uint8_t*>(base) + L.scale_offset);
+  p.T = L.rows_per_plane;
+  p.code_bytes = (int32_t)L.code_bytes;
+  p.n_scales = (int32_t)L.n_scales;
+  return p;
+}
+
 Plane plane_of(const kvq_cache_desc* d, int32_t batch, int which, void* base) {
   kvq_plane_layout L;
   kvq_cache_layout(d, batch, which, &L);
@@ -235,10 +285,15 @@ Plane plane_of(const kvq_cache_desc* d, int32_t batch, int which, void* base) {
 // kvq_decode_step, and their per-sequence-length forms, where ctx_len is the
 // bound on the lengths); a plain decode appends nothing and writes partials only.
 kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void* v_cache, const void* q,
-                       int32_t batch, int64_t ctx_len, const int32_t* ctx_lens, float softmax_scale,
-                       int32_t n_splits, void* workspace, size_t workspace_bytes, DecodeParams* out) {
+                       int32_t batch, int64_t ctx_len, const int32_t* ctx_lens, const kvq_paged* pg,
+                       float softmax_scale, int32_t n_splits, void* workspace, size_t workspace_bytes,
+                       DecodeParams* out) {
   kvq_status st = kvq_check_desc(d);
   if (st != KVQ_OK) return st;
+  if (pg != nullptr) {
+    if ((st = check_paged(d, pg)) != KVQ_OK) return st;
+    if (ctx_len > paged_capacity(d, pg)) return KVQ_ERR_INVALID;
+  }
   if (!k_cache || !v_cache || !q || !workspace) return KVQ_ERR_INVALID;
   if (batch < 1 || batch > 65535 || ctx_len < 1 || ctx_len > d->max_ctx) return KVQ_ERR_INVALID;
   if (n_splits < 0 || n_splits > kMaxSplits || !std::isfinite(softmax_scale)) return KVQ_ERR_INVALID;
@@ -253,8 +308,14 @@ kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void*
 
   DecodeParams& p = *out;
   p = DecodeParams{};
-  p.k = plane_of(d, batch, 0, const_cast<void*>(k_cache));
-  p.v = plane_of(d, batch, 1, const_cast<void*>(v_cache));
+  p.k = pg ? pool_plane_of(d, pg, 0, const_cast<void*>(k_cache)) : plane_of(d, batch, 0, const_cast<void*>(k_cache));
+  p.v = pg ? pool_plane_of(d, pg, 1, const_cast<void*>(v_cache)) : plane_of(d, batch, 1, const_cast<void*>(v_cache));
+  if (pg) {
+    p.block_table = pg->block_table;
+    p.max_pages = pg->max_pages;
+    p.log2_page = log2_of(pg->page_rows);
+    p.n_pages = pg->n_pages;
+  }
   p.q = static_cast<const __half*>(q);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.ws_m = reinterpret_cast<float*>(ws + w.m_off);
@@ -277,9 +338,11 @@ kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void*
   return KVQ_OK;
 }
 kvq_status append_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
-                       int32_t batch, int64_t pos, const int32_t* lens, int32_t n_tok, void* stream) {
+                       int32_t batch, int64_t pos, const int32_t* lens, const kvq_paged* pg, int32_t n_tok,
+                       void* stream) {
   kvq_status st = kvq_check_desc(d);
   if (st != KVQ_OK) return st;
+  if (pg != nullptr && (st = check_paged(d, pg)) != KVQ_OK) return st;
   if (batch < 1 || batch > 65535 || n_tok < 1 || n_tok > d->max_ctx) return KVQ_ERR_INVALID;
   if (lens == nullptr && (pos < 0 || pos + n_tok > d->max_ctx)) return KVQ_ERR_INVALID;
   if (lens != nullptr && !aligned(lens, 4)) return KVQ_ERR_INVALID;
@@ -298,14 +361,20 @@ kvq_status append_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, co
     AppendParams& p = ap[which];
     p = AppendParams{};
     p.src = static_cast<const __half*>(which ? v_new : k_new);
-    p.dst = plane_of(d, batch, which, cache);
+    p.dst = pg ? pool_plane_of(d, pg, which, cache) : plane_of(d, batch, which, cache);
     p.B = batch;
     p.H = d->n_kv_heads;
     p.D = d->head_dim;
     p.n_tok = n_tok;
     p.pos = lens ? 0 : pos;
     p.lens = lens;
-    p.len_max = d->max_ctx;
+    p.len_max = pg ? paged_capacity(d, pg) : d->max_ctx;
+    if (pg) {
+      p.block_table = pg->block_table;
+      p.max_pages = pg->max_pages;
+      p.log2_page = log2_of(pg->page_rows);
+      p.n_pages = pg->n_pages;
+    }
     p.h_mul = div_multiplier((uint64_t)p.H);
     p.t_mul = div_multiplier((uint64_t)n_tok);
     if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) p.t3 = turbo3_consts(d);
@@ -316,10 +385,11 @@ kvq_status append_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, co
 }
 
 kvq_status decode_impl(const kvq_cache_desc* d, const void* k_cache, const void* v_cache, const void* q,
-                       int32_t batch, int64_t ctx_len, const int32_t* ctx_lens, float softmax_scale,
-                       int32_t n_splits, void* workspace, size_t workspace_bytes, void* stream) {
+                       int32_t batch, int64_t ctx_len, const int32_t* ctx_lens, const kvq_paged* pg,
+                       float softmax_scale, int32_t n_splits, void* workspace, size_t workspace_bytes,
+                       void* stream) {
   DecodeParams p{};
-  const kvq_status st = fill_decode(d, k_cache, v_cache, q, batch, ctx_len, ctx_lens, softmax_scale, n_splits,
+  const kvq_status st = fill_decode(d, k_cache, v_cache, q, batch, ctx_len, ctx_lens, pg, softmax_scale, n_splits,
                                     workspace, workspace_bytes, &p);
   if (st != KVQ_OK) return st;
   const cudaError_t e = launch_decode(d->k_type, d->v_type, p, static_cast<cudaStream_t>(stream));
@@ -329,12 +399,12 @@ kvq_status decode_impl(const kvq_cache_desc* d, const void* k_cache, const void*
 
 kvq_status step_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* q, const void* k_new,
                      const void* v_new, int32_t batch, int64_t ctx_len, const int32_t* ctx_lens,
-                     float softmax_scale, int32_t n_splits, void* workspace, size_t workspace_bytes, float* out,
-                     void* stream) {
+                     const kvq_paged* pg, float softmax_scale, int32_t n_splits, void* workspace,
+                     size_t workspace_bytes, float* out, void* stream) {
   if (!k_new || !v_new || !out) return KVQ_ERR_INVALID;
   if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(out, 16)) return KVQ_ERR_INVALID;
   DecodeParams p{};
-  const kvq_status st = fill_decode(d, k_cache, v_cache, q, batch, ctx_len, ctx_lens, softmax_scale, n_splits,
+  const kvq_status st = fill_decode(d, k_cache, v_cache, q, batch, ctx_len, ctx_lens, pg, softmax_scale, n_splits,
                                     workspace, workspace_bytes, &p);
   if (st != KVQ_OK) return st;
   const WsLayout w = ws_layout(d, batch, p.S);
@@ -350,6 +420,10 @@ kvq_status step_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, cons
     a.pos = p.append_pos;
     a.lens = ctx_lens;
     a.len_max = ctx_len;
+    a.block_table = p.block_table;
+    a.max_pages = p.max_pages;
+    a.log2_page = p.log2_page;
+    a.n_pages = p.n_pages;
     a.h_mul = div_multiplier((uint64_t)a.H);
     a.t_mul = div_multiplier(1);
     if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) a.t3 = turbo3_consts(d);
@@ -412,16 +486,53 @@ kvq_status kvq_cache_layout(const kvq_cache_desc* d, int32_t batch, int32_t whic
   const int32_t type = which ? d->v_type : d->k_type;
   const int64_t T = rows_per_plane(d->max_ctx);
   const int64_t planes = (int64_t)batch * d->n_kv_heads;
-  const int64_t cb = code_bytes_of(type, d->head_dim);
-  const int64_t ns = n_scales_of(type, d->head_dim);
-  const double approx = (double)planes * (double)T * (double)(cb + 2 * ns);
+  const double approx = (double)planes * (double)T * (double)(code_bytes_of(type, d->head_dim) +
+                                                             2 * n_scales_of(type, d->head_dim));
   if (approx > 9.0e18) return KVQ_ERR_INVALID;
-  out->rows_per_plane = T;
-  out->code_bytes = cb;
-  out->n_scales = ns;
-  out->scale_offset = round_up(planes * T * cb, 256);
-  out->total_bytes = out->scale_offset + planes * T * ns * 2;
+  fill_layout(type, d->head_dim, planes, T, out);
   return KVQ_OK;
+}
+
+kvq_status kvq_paged_layout(const kvq_cache_desc* d, int32_t page_rows, int64_t n_pages, int32_t which,
+                            kvq_plane_layout* out) {
+  kvq_status st = kvq_check_desc(d);
+  if (st != KVQ_OK) return st;
+  if (!out || (which != 0 && which != 1)) return KVQ_ERR_INVALID;
+  if ((st = check_pool(d, page_rows, n_pages)) != KVQ_OK) return st;
+  fill_layout(which ? d->v_type : d->k_type, d->head_dim, n_pages * d->n_kv_heads, page_rows, out);
+  return KVQ_OK;
+}
+
+size_t kvq_paged_cache_bytes(const kvq_cache_desc* d, int32_t page_rows, int64_t n_pages, int32_t which) {
+  kvq_plane_layout L;
+  if (kvq_paged_layout(d, page_rows, n_pages, which, &L) != KVQ_OK) return 0;
+  return (size_t)L.total_bytes;
+}
+
+kvq_status kvq_append_quantize_paged(const kvq_cache_desc* d, void* k_pool, void* v_pool, const void* k_new,
+                                     const void* v_new, int32_t batch, const kvq_paged* pages, const int32_t* lens,
+                                     int32_t n_tok, void* stream) {
+  if (!lens || !pages) return KVQ_ERR_INVALID;
+  return append_impl(d, k_pool, v_pool, k_new, v_new, batch, 0, lens, pages, n_tok, stream);
+}
+
+kvq_status kvq_decode_attention_paged(const kvq_cache_desc* d, const void* k_pool, const void* v_pool, const void* q,
+                                      int32_t batch, const kvq_paged* pages, const int32_t* ctx_lens,
+                                      int64_t max_ctx_len, float softmax_scale, int32_t n_splits, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (!ctx_lens || !pages) return KVQ_ERR_INVALID;
+  return decode_impl(d, k_pool, v_pool, q, batch, max_ctx_len, ctx_lens, pages, softmax_scale, n_splits, workspace,
+                     workspace_bytes, stream);
+}
+
+kvq_status kvq_decode_step_paged(const kvq_cache_desc* d, void* k_pool, void* v_pool, const void* q,
+                                 const void* k_new, const void* v_new, int32_t batch, const kvq_paged* pages,
+                                 const int32_t* ctx_lens, int64_t max_ctx_len, float softmax_scale,
+                                 int32_t n_splits, void* workspace, size_t workspace_bytes, float* out,
+                                 void* stream) {
+  if (!ctx_lens || !pages) return KVQ_ERR_INVALID;
+  return step_impl(d, k_pool, v_pool, q, k_new, v_new, batch, max_ctx_len, ctx_lens, pages, softmax_scale,
+                   n_splits, workspace, workspace_bytes, out, stream);
 }
 
 size_t kvq_cache_bytes(const kvq_cache_desc* d, int32_t batch, int32_t which) {
@@ -459,20 +570,20 @@ kvq_status kvq_turbo3_signs(uint64_t seed, int32_t head_dim, float* signs) {
 
 kvq_status kvq_append_quantize(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* k_new,
                                const void* v_new, int32_t batch, int64_t pos, int32_t n_tok, void* stream) {
-  return append_impl(d, k_cache, v_cache, k_new, v_new, batch, pos, nullptr, n_tok, stream);
+  return append_impl(d, k_cache, v_cache, k_new, v_new, batch, pos, nullptr, nullptr, n_tok, stream);
 }
 
 kvq_status kvq_append_quantize_varlen(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* k_new,
                                       const void* v_new, int32_t batch, const int32_t* lens, int32_t n_tok,
                                       void* stream) {
   if (!lens) return KVQ_ERR_INVALID;
-  return append_impl(d, k_cache, v_cache, k_new, v_new, batch, 0, lens, n_tok, stream);
+  return append_impl(d, k_cache, v_cache, k_new, v_new, batch, 0, lens, nullptr, n_tok, stream);
 }
 
 kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* k_cache, const void* v_cache, const void* q,
                                 int32_t batch, int64_t ctx_len, float softmax_scale, int32_t n_splits,
                                 void* workspace, size_t workspace_bytes, void* stream) {
-  return decode_impl(d, k_cache, v_cache, q, batch, ctx_len, nullptr, softmax_scale, n_splits, workspace,
+  return decode_impl(d, k_cache, v_cache, q, batch, ctx_len, nullptr, nullptr, softmax_scale, n_splits, workspace,
                      workspace_bytes, stream);
 }
 
@@ -481,14 +592,14 @@ kvq_status kvq_decode_attention_varlen(const kvq_cache_desc* d, const void* k_ca
                                        float softmax_scale, int32_t n_splits, void* workspace,
                                        size_t workspace_bytes, void* stream) {
   if (!ctx_lens) return KVQ_ERR_INVALID;
-  return decode_impl(d, k_cache, v_cache, q, batch, max_ctx_len, ctx_lens, softmax_scale, n_splits, workspace,
-                     workspace_bytes, stream);
+  return decode_impl(d, k_cache, v_cache, q, batch, max_ctx_len, ctx_lens, nullptr, softmax_scale, n_splits,
+                     workspace, workspace_bytes, stream);
 }
 
 kvq_status kvq_decode_step(const kvq_cache_desc* d, void* k_cache, void* v_cache, const void* q, const void* k_new,
                            const void* v_new, int32_t batch, int64_t ctx_len, float softmax_scale, int32_t n_splits,
                            void* workspace, size_t workspace_bytes, float* out, void* stream) {
-  return step_impl(d, k_cache, v_cache, q, k_new, v_new, batch, ctx_len, nullptr, softmax_scale, n_splits,
+  return step_impl(d, k_cache, v_cache, q, k_new, v_new, batch, ctx_len, nullptr, nullptr, softmax_scale, n_splits,
                    workspace, workspace_bytes, out, stream);
 }
 
@@ -497,8 +608,8 @@ kvq_status kvq_decode_step_varlen(const kvq_cache_desc* d, void* k_cache, void* 
                                   int64_t max_ctx_len, float softmax_scale, int32_t n_splits, void* workspace,
                                   size_t workspace_bytes, float* out, void* stream) {
   if (!ctx_lens) return KVQ_ERR_INVALID;
-  return step_impl(d, k_cache, v_cache, q, k_new, v_new, batch, max_ctx_len, ctx_lens, softmax_scale, n_splits,
-                   workspace, workspace_bytes, out, stream);
+  return step_impl(d, k_cache, v_cache, q, k_new, v_new, batch, max_ctx_len, ctx_lens, nullptr, softmax_scale,
+                   n_splits, workspace, workspace_bytes, out, stream);
 }
 
 kvq_status kvq_combine(const kvq_cache_desc* d, const void* workspace, size_t workspace_bytes, int32_t batch,

@@ -13,7 +13,8 @@ constexpr int kBlock = 32;          // elements per q8_0 / q4_0 block
 constexpr int kMaxHeadDim = 256;
 constexpr int kRowAlign = 16;       // rows per plane are a multiple of this
 constexpr int kMaxSplits = 4096;
-constexpr int kSplitAlign = 16;     // split chunks are a multiple of this many rows
+constexpr int kSplitAlign = 32;     // split chunks are whole 32-row tiles (a tile never
+                                    // crosses a page of a paged pool)
 
 // Device view of one cache tensor (K or V) of one layer.
 struct Plane {
@@ -40,6 +41,13 @@ struct AppendParams {
   // lies outside [n_tok, len_max] is not written.
   const int32_t* lens;
   int64_t len_max;
+  // Paged pool (block_table null: contiguous): logical row r of batch row b is
+  // row r & (2^log2_page - 1) of page block_table[b * max_pages + (r >> log2_page)];
+  // dst then describes the pool (B = pages, T = page rows).  A page id outside
+  // [0, n_pages) is not written.
+  const int32_t* block_table;
+  int32_t max_pages, log2_page;
+  int64_t n_pages;
   // n / H and n / n_tok for 32-bit n as the high half of n * mul (mul = 0: divisor 1)
   uint64_t h_mul, t_mul;
   Turbo3Consts t3;
@@ -62,6 +70,12 @@ struct DecodeParams {
   // rows): batch row b attends rows [0, ctx_lens[b]) in S chunks of its own;
   // ctx is then the bound, and a length outside [1, ctx] attends nothing.
   const int32_t* ctx_lens;
+  // Paged pool (block_table null: contiguous): as in AppendParams; k and v
+  // describe the pools (T = page rows), and the tensor maps span n_pages * n_kv
+  // planes.  A page id outside [0, n_pages) makes the split's partials NaN.
+  const int32_t* block_table;
+  int32_t max_pages, log2_page;
+  int64_t n_pages;
   float qscale;        // softmax_scale * log2(e)
   Turbo3Consts t3;     // V sign bits and codebook (turbo3 values)
   // Fused decode step (kvq_decode_step); a plain decode has append_pos < 0 and

@@ -62,8 +62,8 @@
  *   Queries: fp16 [batch][n_q_heads][head_dim].  Output: fp32
  *   [batch][n_q_heads][head_dim].
  *   Split-KV: with S splits, chunk = ceil(ctx_len / S) rounded up to a multiple
- *   of 16; split s covers rows [s*chunk, min((s+1)*chunk, ctx_len)) and may be
- *   empty.
+ *   of 32 (one tile); split s covers rows [s*chunk, min((s+1)*chunk, ctx_len))
+ *   and may be empty.
  *
  * Ownership, threading, errors
  *   The caller owns every buffer.  No entry point allocates device memory,
@@ -125,6 +125,17 @@ typedef struct {
   int64_t scale_offset;    /* byte offset of the scale plane */
   int64_t total_bytes;     /* bytes to allocate */
 } kvq_plane_layout;
+
+/* A paged cache (see "Paged pools" below): the pool's geometry and the block
+ * table that maps each sequence's pages into it. */
+typedef struct {
+  const int32_t* block_table;  /* device int32 [batch][max_pages], 4-byte aligned:
+                                  page id of sequence b's logical rows
+                                  [j * page_rows, (j + 1) * page_rows) */
+  int32_t max_pages;           /* columns of block_table, >= 1 */
+  int32_t page_rows;           /* rows per page: a power of two, 32 .. 2^20 */
+  int64_t n_pages;             /* pages in the pool, >= 1 (n_pages * n_kv_heads < 2^31) */
+} kvq_paged;
 
 /* Human-readable name of a status.  Never NULL. */
 KVQ_API const char* kvq_status_string(kvq_status s);
@@ -276,7 +287,7 @@ KVQ_API kvq_status kvq_decode_step(const kvq_cache_desc* desc, void* k_cache, vo
  *                 takes ctx_len's place in the split choice (n_splits = 0),
  *                 in kvq_workspace_bytes and in kvq_combine.
  * Batch row b attends rows [0, ctx_lens[b]), cut into n_splits chunks of its
- * own (a multiple of 16 rows each; trailing splits may be empty).  A length
+ * own (a multiple of 32 rows each; trailing splits may be empty).  A length
  * outside [1, max_ctx_len] attends no row: that row reads no cache byte, every
  * split partial is empty (m = -inf, l = 0), and the combined output is NaN.
  * Nothing is read or written out of bounds, whatever the lengths hold.
@@ -309,6 +320,53 @@ KVQ_API kvq_status kvq_decode_step_varlen(const kvq_cache_desc* desc, void* k_ca
 KVQ_API kvq_status kvq_append_quantize_varlen(const kvq_cache_desc* desc, void* k_cache, void* v_cache,
                                               const void* k_new, const void* v_new, int32_t batch,
                                               const int32_t* lens, int32_t n_tok, void* cuda_stream);
+
+/*
+ * Paged pools.  Sequences grow and finish at different times, so a server keeps
+ * their rows in fixed-size pages drawn from one pool instead of one max_ctx
+ * slab per sequence.  A pool tensor (K or V of one layer) has exactly the
+ * layout of a contiguous cache of batch = n_pages and max_ctx = page_rows:
+ *   code plane  [n_pages][n_kv_heads][page_rows][code_bytes]
+ *   scale plane [n_pages][n_kv_heads][page_rows][n_scales] fp16, 256-aligned offset
+ * Logical row r of sequence b is row r mod page_rows of page
+ * block_table[b * max_pages + r / page_rows].  Rows are those of the formats
+ * above, byte for byte.  Sequence lengths are per sequence (as in the _varlen
+ * calls) and at most min(max_ctx, max_pages * page_rows).  A block-table entry
+ * that is read and is not in [0, n_pages) is never dereferenced: the
+ * rows that would go there are not written, and a decode that meets one
+ * makes that sequence's output NaN.
+ */
+KVQ_API kvq_status kvq_paged_layout(const kvq_cache_desc* desc, int32_t page_rows, int64_t n_pages,
+                                    int32_t which, kvq_plane_layout* out);
+
+/* Bytes to allocate for a K (which = 0) or V (which = 1) pool; 0 on error. */
+KVQ_API size_t kvq_paged_cache_bytes(const kvq_cache_desc* desc, int32_t page_rows, int64_t n_pages,
+                                     int32_t which);
+
+/* kvq_append_quantize_varlen into a pool: sequence b's n_tok new rows go to
+ * logical rows lens[b] - n_tok .. lens[b] - 1 (lens: its length after the
+ * append, device int32 [batch]); a sequence whose length lies outside
+ * [n_tok, capacity] is not written. */
+KVQ_API kvq_status kvq_append_quantize_paged(const kvq_cache_desc* desc, void* k_pool, void* v_pool,
+                                             const void* k_new, const void* v_new, int32_t batch,
+                                             const kvq_paged* pages, const int32_t* lens, int32_t n_tok,
+                                             void* cuda_stream);
+
+/* kvq_decode_attention_varlen over a pool (max_ctx_len <= the capacity). */
+KVQ_API kvq_status kvq_decode_attention_paged(const kvq_cache_desc* desc, const void* k_pool,
+                                              const void* v_pool, const void* q, int32_t batch,
+                                              const kvq_paged* pages, const int32_t* ctx_lens,
+                                              int64_t max_ctx_len, float softmax_scale, int32_t n_splits,
+                                              void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* kvq_decode_step_varlen over a pool: sequence b's new row goes to logical row
+ * ctx_lens[b] - 1, through the block table, before it is read back. */
+KVQ_API kvq_status kvq_decode_step_paged(const kvq_cache_desc* desc, void* k_pool, void* v_pool,
+                                         const void* q, const void* k_new, const void* v_new,
+                                         int32_t batch, const kvq_paged* pages, const int32_t* ctx_lens,
+                                         int64_t max_ctx_len, float softmax_scale, int32_t n_splits,
+                                         void* workspace, size_t workspace_bytes, float* out,
+                                         void* cuda_stream);
 
 #ifdef __cplusplus
 }

@@ -226,6 +226,51 @@ def test_varlen_entry_points_reject_before_launch():
     assert _append_varlen(t3k) == kvq.KVQ_ERR_UNSUPPORTED
 
 
+def test_paged_layout_is_the_contiguous_layout_of_pages():
+    """A pool is laid out as a contiguous cache with the pages as batch rows
+    and page_rows rows per plane."""
+    for kt, vt, D in (("q8_0", "q4_0", 128), ("f16", "turbo3", 64), ("q4_0", "q8_0", 256)):
+        for P, n in ((32, 1), (64, 700), (256, 33)):
+            d = kvq.make_desc(32, 8, D, kt, vt, 100000)
+            for which in (0, 1):
+                got = kvq.kvq_paged_layout(d, P, n, which)
+                ref = kvq.kvq_cache_layout(kvq.make_desc(32, 8, D, kt, vt, P), n, which)
+                for f in ("rows_per_plane", "code_bytes", "n_scales", "scale_offset", "total_bytes"):
+                    assert getattr(got, f) == getattr(ref, f), (kt, vt, D, P, n, which, f)
+                assert kvq.kvq_paged_cache_bytes(d, P, n, which) == ref.total_bytes
+
+
+def _pg(table=FAKE, max_pages=4, page_rows=64, n_pages=100):
+    return kvq.kvq_paged(table, max_pages, page_rows, n_pages)
+
+
+def test_paged_entry_points_reject_before_launch():
+    d = kvq.make_desc(32, 8, 128, "q8_0", "q4_0", 8192)
+    dec = lambda pg, lens=FAKE, mx=256: kvq.raw_status("kvq_decode_attention_paged", ctypes.byref(d), FAKE, FAKE,
+                                                        FAKE, 1, ctypes.byref(pg) if pg else None, lens, mx, 0.1,
+                                                        0, FAKE, 1 << 40, None)
+    step = lambda pg, lens=FAKE, mx=256: kvq.raw_status("kvq_decode_step_paged", ctypes.byref(d), FAKE, FAKE, FAKE,
+                                                         FAKE, FAKE, 1, ctypes.byref(pg) if pg else None, lens, mx,
+                                                         0.1, 0, FAKE, 1 << 40, FAKE, None)
+    app = lambda pg, lens=FAKE, n=1: kvq.raw_status("kvq_append_quantize_paged", ctypes.byref(d), FAKE, FAKE, FAKE,
+                                                     FAKE, 1, ctypes.byref(pg) if pg else None, lens, n, None)
+    for call in (dec, step, app):
+        assert call(None) == kvq.KVQ_ERR_INVALID                          # no pool description
+        assert call(_pg(), lens=None) == kvq.KVQ_ERR_INVALID              # no lengths
+        assert call(_pg(table=None)) == kvq.KVQ_ERR_INVALID
+        assert call(_pg(table=FAKE + 2)) == kvq.KVQ_ERR_INVALID           # table not 4-byte aligned
+        assert call(_pg(max_pages=0)) == kvq.KVQ_ERR_INVALID
+        assert call(_pg(n_pages=0)) == kvq.KVQ_ERR_INVALID
+        assert call(_pg(page_rows=16)) == kvq.KVQ_ERR_UNSUPPORTED        # below one 32-row tile
+        assert call(_pg(page_rows=96)) == kvq.KVQ_ERR_UNSUPPORTED        # not a power of two
+        assert call(_pg(n_pages=1 << 28)) == kvq.KVQ_ERR_UNSUPPORTED     # n_pages * n_kv >= 2^31
+    # the host bound on the lengths: within max_ctx and what the block table can address
+    assert dec(_pg(max_pages=4, page_rows=64), mx=257) == kvq.KVQ_ERR_INVALID
+    assert step(_pg(max_pages=4, page_rows=64), mx=257) == kvq.KVQ_ERR_INVALID
+    assert dec(_pg(max_pages=1000, page_rows=64), mx=8193) == kvq.KVQ_ERR_INVALID
+    assert kvq.kvq_paged_cache_bytes(d, 16, 10, 0) == 0
+
+
 def test_workspace_bytes_formula():
     d = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 32768)
     B, S = 4, 9
@@ -250,7 +295,7 @@ def test_auto_splits_bounded_and_nonempty():
             s = kvq.kvq_auto_splits(d, batch, ctx)
             assert 1 <= s <= 4096
             assert kvq.kvq_workspace_bytes(d, batch, s) <= bound
-            # chunks are whole 16-row groups and no automatic split is empty
-            chunk = -(-(-(-ctx // s)) // 16) * 16
+            # chunks are whole 32-row tiles and no automatic split is empty
+            chunk = -(-(-(-ctx // s)) // 32) * 32
             assert (s - 1) * chunk < ctx
     assert kvq.kvq_auto_splits(d, 1, 0) == 0

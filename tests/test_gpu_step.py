@@ -200,7 +200,7 @@ def test_full_size_sampled(name):
 def test_many_splits_and_empty_ones(S):
     """More than 32 splits (the in-kernel combine takes the weights 32 at a
     time) and, at S = 300 over 3000 rows, trailing splits left empty by the
-    16-row chunk rounding (weight 0)."""
+    32-row chunk rounding (weight 0)."""
     B, n_q, n_kv, D, ctx = 1, 8, 2, 128, 3000
     desc, q, k, v = _inputs("q8_0", "turbo3", B, n_q, n_kv, D, ctx, seed=S)
     kc, vc = alloc_cache(desc, B, 0), alloc_cache(desc, B, 1)
