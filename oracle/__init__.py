@@ -17,6 +17,7 @@ Modules:
   blocks      q8_0 / q4_0 / f16 cache rows (quantize, pack, dequantize)
   turbo3      seeded sign vector (splitmix64), Sylvester Hadamard, fast
               Walsh-Hadamard transform, Lloyd-Max codebook, turbo3 rows
+  turbo       the same rows at 2 and 4 bits per value (turbo2, turbo4)
   attention   decode attention (plain softmax definition), split partials
               and their combine
   cache_model bytes per cache row / per cache, the nominal-size model
@@ -27,6 +28,9 @@ Pins (what each function is checked against, in ``tests/test_oracle_*.py``):
   turbo3      published splitmix64 vectors, H*H = d*I, FWHT(e_k) = column k,
               Max (1960) 8-level Gaussian quantizer table, centroid and
               midpoint conditions, round-trip MSE of the Gaussian quantizer
+  turbo       2-level closed form +-sqrt(2/pi), Max (1960) 4- and 16-level
+              tables, hand-packed 2- and 4-bit bytes, the turbo3 oracle at 3
+              bits, round-trip error = the quantizer's distortion
   attention   brute-force full-matrix softmax(Q K^T) V, closed forms
               (ctx=1, identical keys, q=0), rows summing to 1, split/combine
               identity
