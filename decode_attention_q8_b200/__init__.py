@@ -24,15 +24,16 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-KVQ_F16, KVQ_Q8_0, KVQ_Q4_0, KVQ_TURBO3 = 0, 1, 2, 3
-TYPES = {"f16": KVQ_F16, "q8_0": KVQ_Q8_0, "q4_0": KVQ_Q4_0, "turbo3": KVQ_TURBO3}
+KVQ_F16, KVQ_Q8_0, KVQ_Q4_0, KVQ_TURBO3, KVQ_TURBO2, KVQ_TURBO4 = 0, 1, 2, 3, 4, 5
+TYPES = {"f16": KVQ_F16, "q8_0": KVQ_Q8_0, "q4_0": KVQ_Q4_0, "turbo3": KVQ_TURBO3, "turbo2": KVQ_TURBO2,
+         "turbo4": KVQ_TURBO4}
 
 KVQ_OK, KVQ_ERR_INVALID, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA = 0, 1, 2, 3, 4
 
 EXPORTED = (
     "kvq_status_string", "kvq_last_cuda_error", "kvq_row_bytes", "kvq_check_desc",
     "kvq_cache_layout", "kvq_cache_bytes", "kvq_auto_splits", "kvq_workspace_bytes",
-    "kvq_turbo3_codebook", "kvq_turbo3_signs", "kvq_append_quantize",
+    "kvq_turbo3_codebook", "kvq_turbo_codebook", "kvq_turbo3_signs", "kvq_append_quantize",
     "kvq_decode_attention", "kvq_combine", "kvq_decode_attention_noalloc", "kvq_decode_step",
     "kvq_decode_attention_varlen", "kvq_decode_step_varlen", "kvq_append_quantize_varlen",
     "kvq_paged_layout", "kvq_paged_cache_bytes", "kvq_append_quantize_paged", "kvq_decode_attention_paged",
@@ -86,6 +87,7 @@ _sigs = {
     "kvq_workspace_bytes": (ctypes.c_size_t, [_D, ctypes.c_int32, ctypes.c_int32]),
     "kvq_turbo3_codebook": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
     "kvq_turbo3_signs": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]),
+    "kvq_turbo_codebook": (ctypes.c_int, [ctypes.c_int32, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
     "kvq_append_quantize": (ctypes.c_int, [_D, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int64,
                                            ctypes.c_int32, _P]),
     "kvq_decode_attention": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
@@ -195,6 +197,16 @@ def kvq_turbo3_codebook():
     th = (ctypes.c_float * 7)()
     _check(_lib.kvq_turbo3_codebook(lv, th), "kvq_turbo3_codebook")
     return list(lv), list(th)
+
+
+def kvq_turbo_codebook(type_):
+    """(levels[2^b], thresholds[2^b - 1]) of a turbo type ("turbo2", "turbo3", "turbo4")."""
+    t = _type(type_)
+    lv = (ctypes.c_float * 16)()
+    th = (ctypes.c_float * 15)()
+    _check(_lib.kvq_turbo_codebook(t, lv, th), "kvq_turbo_codebook")
+    n = {KVQ_TURBO2: 4, KVQ_TURBO3: 8, KVQ_TURBO4: 16}[t]
+    return list(lv)[:n], list(th)[:n - 1]
 
 
 def kvq_turbo3_signs(seed, head_dim):

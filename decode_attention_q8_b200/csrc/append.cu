@@ -67,20 +67,25 @@ __device__ __forceinline__ void append_blocks(const AppendParams& p, int64_t fir
   }
 }
 
+template <int TYPE>
+__device__ __forceinline__ void append_turbo_part(const AppendParams& p, int64_t first, int64_t stride, int64_t gend) {
+  switch (p.D) {
+    case 32: append_stream<TYPE, 1>(p, first, stride, gend); break;
+    case 64: append_stream<TYPE, 2>(p, first, stride, gend); break;
+    case 128: append_stream<TYPE, 4>(p, first, stride, gend); break;
+    case 256: append_stream<TYPE, 8>(p, first, stride, gend); break;
+  }
+}
+
 __device__ __forceinline__ void append_part(const AppendParams& p, int32_t type, int64_t first, int64_t stride) {
   const int64_t gend = (int64_t)p.B * p.n_tok * p.H * bulk_items(type, p.D);
   switch (type) {
     case KVQ_F16: append_stream<KVQ_F16, 0>(p, first, stride, gend); break;
     case KVQ_Q8_0: append_blocks<KVQ_Q8_0>(p, first, stride, gend); break;
     case KVQ_Q4_0: append_blocks<KVQ_Q4_0>(p, first, stride, gend); break;
-    case KVQ_TURBO3:
-      switch (p.D) {
-        case 32: append_stream<KVQ_TURBO3, 1>(p, first, stride, gend); break;
-        case 64: append_stream<KVQ_TURBO3, 2>(p, first, stride, gend); break;
-        case 128: append_stream<KVQ_TURBO3, 4>(p, first, stride, gend); break;
-        case 256: append_stream<KVQ_TURBO3, 8>(p, first, stride, gend); break;
-      }
-      break;
+    case KVQ_TURBO2: append_turbo_part<KVQ_TURBO2>(p, first, stride, gend); break;
+    case KVQ_TURBO3: append_turbo_part<KVQ_TURBO3>(p, first, stride, gend); break;
+    case KVQ_TURBO4: append_turbo_part<KVQ_TURBO4>(p, first, stride, gend); break;
   }
 }
 

@@ -41,7 +41,7 @@ __device__ __forceinline__ uint4 load_raw(const AppendParams& p, int64_t gtid, i
     r.y = v.y;
   } else if constexpr (TYPE == KVQ_F16) {
     r = __ldg(reinterpret_cast<const uint4*>(p.src + gtid * 8));
-  } else {  // turbo3
+  } else {  // turbo types
     if constexpr (E == 8) {
       r = __ldg(reinterpret_cast<const uint4*>(p.src + gtid * 8));
     } else if constexpr (E == 4) {
@@ -322,9 +322,10 @@ __device__ __forceinline__ void append_f16(const AppendParams& p, int64_t gtid, 
   reinterpret_cast<uint4*>(p.dst.codes + r * p.dst.code_bytes)[c] = raw;
 }
 
-// turbo3: one warp per row, E = D/32 contiguous elements per lane.
-template <int E>
-__device__ __forceinline__ void append_turbo3(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
+// turbo (BITS = 2, 3 or 4 bits per value): one warp per row, E = D/32
+// contiguous elements per lane.
+template <int BITS, int E>
+__device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
   constexpr int D = 32 * E;
   const int64_t row = gtid >> 5;
   const int lane = (int)(gtid & 31);
@@ -334,7 +335,7 @@ __device__ __forceinline__ void append_turbo3(const AppendParams& p, int64_t gti
   for (int e = 0; e < E; ++e) {
     const int i = lane * E + e;
     const float x = raw_elem(raw, e);
-    v[e] = ((p.t3.sign_bits[i >> 5] >> (i & 31)) & 1u) ? -x : x;
+    v[e] = ((p.tq.sign_bits[i >> 5] >> (i & 31)) & 1u) ? -x : x;
   }
   // |v|^2 by the strided pairwise tree a[i] += a[i+h], h = D/2 ... 1
   float a[E];
@@ -380,34 +381,27 @@ __device__ __forceinline__ void append_turbo3(const AppendParams& p, int64_t gti
     const float g = __fmul_rn(v[e], r);
     int c = 0;
 #pragma unroll
-    for (int k = 0; k < 7; ++k) c += (g > p.t3.tau[k]) ? 1 : 0;
-    bits |= (uint32_t)c << (3 * e);
+    for (int k = 0; k < (1 << BITS) - 1; ++k) c += (g > p.tq.tau[k]) ? 1 : 0;
+    bits |= (uint32_t)c << (BITS * e);
   }
-  // 8 consecutive elements -> 3 bytes; a group of 8/E lanes holds them
-  constexpr int L = (E >= 8) ? 1 : 8 / E;
+  // The lane's LB = BITS*E bits start at bit LB*lane of the row; a group of L
+  // lanes (the fewest whose bits make whole bytes, at most 32) is stored by
+  // its first lane.
+  constexpr int LB = BITS * E;
+  constexpr int L = LB % 8 == 0 ? 1 : LB % 4 == 0 ? 2 : LB % 2 == 0 ? 4 : 8;
   uint32_t word = bits;
 #pragma unroll
   for (int j = 1; j < L; ++j) {
     const uint32_t o = __shfl_down_sync(0xffffffffu, bits, j);
-    word |= o << (3 * E * j);
+    word |= o << (LB * j);
   }
   const int64_t r_dst = dst_row(p, row);
   if (r_dst < 0) return;  // after the last shuffle
   uint8_t* codes = p.dst.codes + r_dst * p.dst.code_bytes;
-  if (E >= 8) {
+  if ((lane % L) == 0) {
+    const int byte0 = LB * lane / 8;
 #pragma unroll
-    for (int g8 = 0; g8 < E / 8; ++g8) {
-      const uint32_t w = (bits >> (24 * g8)) & 0xFFFFFFu;  // E == 8: one group
-      const int byte0 = 3 * ((lane * E) / 8 + g8);
-      codes[byte0 + 0] = (uint8_t)(w & 0xFF);
-      codes[byte0 + 1] = (uint8_t)((w >> 8) & 0xFF);
-      codes[byte0 + 2] = (uint8_t)((w >> 16) & 0xFF);
-    }
-  } else if ((lane % L) == 0) {
-    const int byte0 = 3 * ((lane * E) / 8);
-    codes[byte0 + 0] = (uint8_t)(word & 0xFF);
-    codes[byte0 + 1] = (uint8_t)((word >> 8) & 0xFF);
-    codes[byte0 + 2] = (uint8_t)((word >> 16) & 0xFF);
+    for (int i = 0; i < L * LB / 8; ++i) codes[byte0 + i] = (uint8_t)((word >> (8 * i)) & 0xFF);
   }
   if (lane == 0) p.dst.scales[r_dst] = __float2half_rn(fminf(norm, 65504.0f));
 }
@@ -419,7 +413,7 @@ __device__ __forceinline__ void finish(const AppendParams& p, int64_t gtid, int6
   if constexpr (TYPE == KVQ_Q8_0) append_q8_0(p, gtid, gend, raw);
   else if constexpr (TYPE == KVQ_Q4_0) append_q4_0(p, gtid, gend, raw);
   else if constexpr (TYPE == KVQ_F16) append_f16(p, gtid, gend, raw);
-  else append_turbo3<E>(p, gtid, gend, raw);
+  else append_turbo<turbo_bits(TYPE), E>(p, gtid, gend, raw);
 }
 
 template <int TYPE, int E>
@@ -429,25 +423,30 @@ __device__ __forceinline__ void append_one(const AppendParams& p, int64_t gtid, 
 
 // Thread gtid of the flat work of one call's rows of a tensor of `type`;
 // threads at or past gend do no work (but still take part in shuffles).
+template <int TYPE>
+__device__ __forceinline__ void append_turbo_any(const AppendParams& p, int64_t gtid, int64_t gend) {
+  switch (p.D) {
+    case 32: append_one<TYPE, 1>(p, gtid, gend); break;
+    case 64: append_one<TYPE, 2>(p, gtid, gend); break;
+    case 128: append_one<TYPE, 4>(p, gtid, gend); break;
+    case 256: append_one<TYPE, 8>(p, gtid, gend); break;
+  }
+}
+
 __device__ __forceinline__ void append_any(int32_t type, const AppendParams& p, int64_t gtid, int64_t gend) {
   switch (type) {
     case KVQ_F16: append_one<KVQ_F16, 0>(p, gtid, gend); break;
     case KVQ_Q8_0: append_one<KVQ_Q8_0, 0>(p, gtid, gend); break;
     case KVQ_Q4_0: append_one<KVQ_Q4_0, 0>(p, gtid, gend); break;
-    case KVQ_TURBO3:
-      switch (p.D) {
-        case 32: append_one<KVQ_TURBO3, 1>(p, gtid, gend); break;
-        case 64: append_one<KVQ_TURBO3, 2>(p, gtid, gend); break;
-        case 128: append_one<KVQ_TURBO3, 4>(p, gtid, gend); break;
-        case 256: append_one<KVQ_TURBO3, 8>(p, gtid, gend); break;
-      }
-      break;
+    case KVQ_TURBO2: append_turbo_any<KVQ_TURBO2>(p, gtid, gend); break;
+    case KVQ_TURBO3: append_turbo_any<KVQ_TURBO3>(p, gtid, gend); break;
+    case KVQ_TURBO4: append_turbo_any<KVQ_TURBO4>(p, gtid, gend); break;
   }
 }
 
 // Threads one row of a tensor of `type` and head dim d needs.
 __host__ __device__ constexpr int row_threads(int32_t type, int d) {
-  return type == KVQ_F16 ? d / 8 : type == KVQ_TURBO3 ? 32 : (d / kBlock) * 8;
+  return type == KVQ_F16 ? d / 8 : is_turbo(type) ? 32 : (d / kBlock) * 8;
 }
 
 }  // namespace rows

@@ -3,7 +3,7 @@
 //   o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s,   M = max_s m_s,
 // which equals plain softmax attention over the whole context ("llama.cpp für
 // Geschwindigkeit und Speicher optimieren", section "Flash Attention": the
-// tiled form is exact).  For a turbo3 value cache the accumulators live in the
+// tiled form is exact).  For a turbo value cache the accumulators live in the
 // rotated domain (sum_t p_t norm_t c[code_t]); the output is rotated back once:
 // o <- s * H_un * o / d, with H_un the unnormalised Walsh-Hadamard matrix and
 // s the seeded sign vector ("Benchmark TurboQuant en Apple Silicon", section
@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
   extern __shared__ float sm[];
   float* red = sm;              // 8 floats
   float* wts = sm + 8;          // S weights
-  float* xs = wts + p.S;        // D values (turbo3 inverse transform)
+  float* xs = wts + p.S;        // D values (turbo inverse transform)
   const int h = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
   const int64_t base = ((int64_t)b * p.n_q + h) * p.S;
   float M = -INFINITY;
@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
   }
   for (; s < p.S; ++s) num = fmaf(wts[s], acc[(int64_t)s * p.D], num);
   float o = num / den;
-  if (p.turbo3) {
+  if (p.rotated) {
     xs[j] = o;
     for (int hs = 1; hs < p.D; hs <<= 1) {
       __syncthreads();
@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
       }
     }
     __syncthreads();
-    const float sgn = ((p.t3.sign_bits[j >> 5] >> (j & 31)) & 1u) ? -1.f : 1.f;
+    const float sgn = ((p.tq.sign_bits[j >> 5] >> (j & 31)) & 1u) ? -1.f : 1.f;
     o = xs[j] * sgn / (float)p.D;
   }
   p.out[((int64_t)b * p.n_q + h) * p.D + j] = o;

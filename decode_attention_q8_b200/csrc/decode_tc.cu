@@ -86,7 +86,7 @@ bool flat_map(CUtensorMap* m, const void* base, int rb, int64_t T, int64_t plane
 }
 
 bool plane_maps(const Plane& pl, int type, int64_t planes, int64_t ctx, CUtensorMap* codes, CUtensorMap* scales) {
-  const bool ok = type == KVQ_TURBO3 ? flat_map(codes, pl.codes, pl.code_bytes, pl.T, planes, ctx)
+  const bool ok = is_turbo(type) ? flat_map(codes, pl.codes, pl.code_bytes, pl.T, planes, ctx)
                                      : code_map(codes, pl.codes, pl.code_bytes, pl.T, planes, ctx);
   if (!ok) return false;
   if (pl.n_scales == 0) {
@@ -99,7 +99,7 @@ bool plane_maps(const Plane& pl, int type, int64_t planes, int64_t ctx, CUtensor
 }  // namespace
 
 bool decode_supported(int32_t k_type, int32_t v_type, int32_t G, int32_t D) {
-  if (k_type == KVQ_TURBO3 || G < 1 || G > 16) return false;
+  if (is_turbo(k_type) || G < 1 || G > 16) return false;
   if (D != 64 && D != 128 && D != 256) return false;
   if (D == 256 && k_type == KVQ_F16 && v_type == KVQ_F16) return false;  // stage would not fit
   return true;
@@ -112,7 +112,9 @@ int ctas_k(int32_t v_type, int32_t D) {
     case KVQ_F16: return tc::ctas_per_sm_for(KT, KVQ_F16, D);
     case KVQ_Q8_0: return tc::ctas_per_sm_for(KT, KVQ_Q8_0, D);
     case KVQ_Q4_0: return tc::ctas_per_sm_for(KT, KVQ_Q4_0, D);
+    case KVQ_TURBO2: return tc::ctas_per_sm_for(KT, KVQ_TURBO2, D);
     case KVQ_TURBO3: return tc::ctas_per_sm_for(KT, KVQ_TURBO3, D);
+    case KVQ_TURBO4: return tc::ctas_per_sm_for(KT, KVQ_TURBO4, D);
   }
   return 1;
 }
@@ -140,6 +142,14 @@ cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p,
   tc::TcArgs a;
   a.p = p;
   const int nb = p.D / 32, nth = p.G <= 8 ? 1 : 2;
+  if (paged) {
+    switch (k_type) {
+      case KVQ_F16: return tc::launch_kf16_paged(v_type, nb, nth, a, maps, st);
+      case KVQ_Q8_0: return tc::launch_kq8_paged(v_type, nb, nth, a, maps, st);
+      case KVQ_Q4_0: return tc::launch_kq4_paged(v_type, nb, nth, a, maps, st);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (k_type) {
     case KVQ_F16: return tc::launch_kf16(v_type, nb, nth, a, maps, st);
     case KVQ_Q8_0: return tc::launch_kq8(v_type, nb, nth, a, maps, st);

@@ -70,26 +70,31 @@ constexpr int kHalf = 16;    // rows per MMA row block (two per tile)
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 __host__ __device__ constexpr int code_bytes(int t, int d) {
-  return t == KVQ_F16 ? 2 * d : t == KVQ_Q8_0 ? d : t == KVQ_Q4_0 ? d / 2 : 3 * d / 8;
+  return t == KVQ_F16 ? 2 * d : t == KVQ_Q8_0 ? d : t == KVQ_Q4_0 ? d / 2 : turbo_bits(t) * d / 8;
 }
 __host__ __device__ constexpr int n_scales(int t, int d) {
-  return t == KVQ_F16 ? 0 : t == KVQ_TURBO3 ? 1 : d / 32;
+  return t == KVQ_F16 ? 0 : is_turbo(t) ? 1 : d / 32;
 }
 // swizzle of a code plane: 16-byte chunk index XOR ((offset >> 7) & mask)
 __host__ __device__ constexpr int swz_mask(int t, int d) {
-  return t == KVQ_TURBO3 ? 0 : (code_bytes(t, d) >= 128 ? 8 : code_bytes(t, d) / 16) - 1;
+  return is_turbo(t) ? 0 : (code_bytes(t, d) >= 128 ? 8 : code_bytes(t, d) / 16) - 1;
+}
+// Entries of a turbo value type's level table (one copy per lane): the levels
+// of two consecutive dims of a row (2^(2b)) at 2 and 3 bits, single levels at 4.
+__host__ __device__ constexpr int turbo_table_entries(int t) {
+  return !is_turbo(t) ? 0 : turbo_bits(t) <= 3 ? 1 << (2 * turbo_bits(t)) : 1 << turbo_bits(t);
 }
 __host__ __device__ constexpr int round_up_c(int v, int a) { return (v + a - 1) / a * a; }
 __host__ __device__ constexpr int stage_bytes(int kt, int vt, int d) {
   return round_up_c(kSub * code_bytes(kt, d), 1024) +
-         round_up_c(kSub * code_bytes(vt, d), vt == KVQ_TURBO3 ? 128 : 1024) +
+         round_up_c(kSub * code_bytes(vt, d), is_turbo(vt) ? 128 : 1024) +
          round_up_c(kSub * n_scales(kt, d) * 2, 128) + round_up_c(kSub * n_scales(vt, d) * 2, 128);
 }
 // Shared memory of one CTA: the 1024-byte alignment pad, one ring of `stages`
-// stages per warp (rounded to the 1024-byte swizzle atom), the turbo3 pair
+// stages per warp (rounded to the 1024-byte swizzle atom), the turbo level
 // table, the ring barriers and a few bytes of slack.
 __host__ __device__ constexpr int cta_smem(int kt, int vt, int d, int nw, int stages) {
-  return 1024 + nw * round_up_c(stages * stage_bytes(kt, vt, d), 1024) + (vt == KVQ_TURBO3 ? 64 * 32 * 4 : 0) +
+  return 1024 + nw * round_up_c(stages * stage_bytes(kt, vt, d), 1024) + turbo_table_entries(vt) * 32 * 4 +
          nw * stages * 8 + 16;
 }
 // An SM has 228 KB of shared memory and reserves 1 KB per resident CTA; the
@@ -120,12 +125,12 @@ struct Layout {
   static constexpr int RBK = code_bytes(KT, D), RBV = code_bytes(VT, D);
   static constexpr int NSK = n_scales(KT, D), NSV = n_scales(VT, D);
   static constexpr int KC = round_up_c(kSub * RBK, 1024);
-  static constexpr int VC = round_up_c(kSub * RBV, VT == KVQ_TURBO3 ? 128 : 1024);
+  static constexpr int VC = round_up_c(kSub * RBV, is_turbo(VT) ? 128 : 1024);
   static constexpr int KS = round_up_c(kSub * NSK * 2, 128);
   static constexpr int VS = round_up_c(kSub * NSV * 2, 128);
   static constexpr int STAGE = KC + VC + KS + VS;
   static constexpr int WARP = round_up_c(kStages * STAGE, 1024);
-  static constexpr int TABLE = VT == KVQ_TURBO3 ? 64 * 32 * 4 : 0;
+  static constexpr int TABLE = turbo_table_entries(VT) * 32 * 4;
   static constexpr int BARS = NW * kStages * 8;
   static constexpr int TX = kSub * (RBK + 2 * NSK + RBV + 2 * NSV);  // bytes landing per tile
   // CTA-level merge scratch (reuses the stage memory after the main loop)
@@ -406,11 +411,14 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
     fence_barrier_init();
   }
-  if (VT == KVQ_TURBO3) {
-    // table[x * 32 + lane] = half2(c[x & 7], c[x >> 3]) for a 6-bit code pair x; one copy per bank
-    for (int e = threadIdx.x; e < 64 * 32; e += L::NW * 32) {
+  if constexpr (is_turbo(VT)) {
+    // b <= 3: table[x * 32 + lane] = half2(c[x mod 2^b], c[x >> b]), the levels of
+    // a 2b-bit code pair x; b = 4: half2(c[x], c[x]).  One copy per bank.
+    constexpr int TB = turbo_bits(VT), NE = turbo_table_entries(VT);
+    for (int e = threadIdx.x; e < NE * 32; e += L::NW * 32) {
       const int idx = e >> 5;
-      table[e] = pack_half2(p.t3.levels[idx & 7], p.t3.levels[idx >> 3]);
+      table[e] = TB <= 3 ? pack_half2(p.tq.levels[idx & ((1 << TB) - 1)], p.tq.levels[idx >> TB])
+                         : pack_half2(p.tq.levels[idx], p.tq.levels[idx]);
     }
   }
   __syncthreads();
@@ -448,7 +456,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     else
       tma_load_3d(kc_of(st), &tm_kc, 0, r0, tplane, &bars[st], pol);
     if (L::NSK) tma_load_2d(ks_of(st), &tm_ks, r0 * L::NSK / 2, tplane, &bars[st], pol);
-    if (VT == KVQ_TURBO3) {
+    if (is_turbo(VT)) {
       if (kSub * L::RBV / 4 <= 256)
         tma_load_2d(vc_of(st), &tm_vc, r0 * L::RBV / 4, tplane, &bars[st], pol);
       else
@@ -693,17 +701,19 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           mma16816(acc[nt][mt], a[0], a[1], a[2], a[3], b0, b1, acc[nt][mt]);
         }
       }
-    } else if constexpr (VT == KVQ_TURBO3) {
-      // lane g owns dims [g*D/8, (g+1)*D/8): 3*D/8 bits of each row's codes
-      constexpr int BITS = 3 * D / 8;
-      constexpr int BYTE0_STEP = BITS / 8;  // bytes per lane group
-      auto field = [&](int row) -> unsigned long long {
-        const int byte0 = g * BYTE0_STEP;
-        const int w0 = byte0 >> 2;
-        const unsigned char* rp = vc + row * L::RBV;
-        unsigned long long v = *reinterpret_cast<const uint32_t*>(rp + 4 * w0);
-        if (BITS + 8 * (byte0 & 3) > 32)
-          v |= (unsigned long long)(*reinterpret_cast<const uint32_t*>(rp + 4 * w0 + 4)) << 32;
+    } else if constexpr (is_turbo(VT)) {
+      // lane group g owns dims [g*D/8, (g+1)*D/8): GB = b*D/8 bits of each row's
+      // codes, read as one or two 64-bit windows (HB bits, MTH m-tiles each)
+      constexpr int TB = turbo_bits(VT);
+      constexpr int GB = TB * D / 8;
+      constexpr int HALVES = GB > 64 ? 2 : 1;
+      constexpr int HB = GB / HALVES;
+      constexpr int MTH = NMT / HALVES;
+      auto field = [&](int row, int h) -> unsigned long long {  // bits [g*GB + h*HB, +HB) of a row
+        const int byte0 = (g * GB + h * HB) >> 3;
+        const unsigned char* rp = vc + row * L::RBV + (byte0 & ~3);
+        unsigned long long v = *reinterpret_cast<const uint32_t*>(rp);
+        if (HB + 8 * (byte0 & 3) > 32) v |= (unsigned long long)(*reinterpret_cast<const uint32_t*>(rp + 4)) << 32;
         return v >> (8 * (byte0 & 3));
       };
       // norms of rows (2c, 2c+1) and (2c+8, 2c+9) are adjacent fp16 pairs
@@ -719,18 +729,34 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           pbw[nt][1] &= pmask_hi;
         }
       }
-      // table[x * 32 + lane] = half2(c[x & 7], c[x >> 3]): the levels of one
-      // row's two consecutive dims; a byte permute pairs rows 2c and 2c+1
+      // b <= 3: table[x * 32 + lane] = half2(c[x mod 2^b], c[x >> b]), the levels
+      // of one row's two consecutive dims; b = 4: half2(c[x], c[x]), two
+      // lookups per dim pair.  A byte permute then pairs rows 2c and 2c+1.
       const uint32_t* tl = table + lane;
-      if (D <= 128) {
-        const unsigned long long fA = field(2 * c), fB = field(2 * c + 1);
-        const unsigned long long fC = field(2 * c + 8), fD = field(2 * c + 9);
 #pragma unroll
-        for (int mt = 0; mt < NMT; ++mt) {
-          const uint32_t tA = tl[((uint32_t)(fA >> (6 * mt)) & 63u) << 5];
-          const uint32_t tB = tl[((uint32_t)(fB >> (6 * mt)) & 63u) << 5];
-          const uint32_t tC = tl[((uint32_t)(fC >> (6 * mt)) & 63u) << 5];
-          const uint32_t tD = tl[((uint32_t)(fD >> (6 * mt)) & 63u) << 5];
+      for (int h = 0; h < HALVES; ++h) {
+        const unsigned long long fA = field(2 * c, h), fB = field(2 * c + 1, h);
+        const unsigned long long fC = field(2 * c + 8, h), fD = field(2 * c + 9, h);
+#pragma unroll
+        for (int k = 0; k < MTH; ++k) {
+          const int mt = h * MTH + k;
+          uint32_t tA, tB, tC, tD;  // half2(level of dim 2mt, of dim 2mt+1) of each row
+          if constexpr (TB <= 3) {
+            constexpr uint32_t PM = (1u << (2 * TB)) - 1;
+            tA = tl[((uint32_t)(fA >> (2 * TB * k)) & PM) << 5];
+            tB = tl[((uint32_t)(fB >> (2 * TB * k)) & PM) << 5];
+            tC = tl[((uint32_t)(fC >> (2 * TB * k)) & PM) << 5];
+            tD = tl[((uint32_t)(fD >> (2 * TB * k)) & PM) << 5];
+          } else {
+            auto pair = [&](unsigned long long f) {
+              return prmt(tl[((uint32_t)(f >> (8 * k)) & 15u) << 5], tl[((uint32_t)(f >> (8 * k + 4)) & 15u) << 5],
+                          0x5410);
+            };
+            tA = pair(fA);
+            tB = pair(fB);
+            tC = pair(fC);
+            tD = pair(fD);
+          }
           uint32_t a[4];
           a[0] = prmt(tA, tB, 0x5410);  // dim 2mt:   rows 2c, 2c+1
           a[1] = prmt(tA, tB, 0x7632);  // dim 2mt+1
@@ -739,36 +765,6 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 #pragma unroll
           for (int nt = 0; nt < NTH; ++nt)
             mma16816(acc[nt][mt], a[0], a[1], a[2], a[3], pbw[nt][0], pbw[nt][1], acc[nt][mt]);
-        }
-      } else {
-        // D = 256: 96 bits per lane group, read as two 48-bit halves
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          auto field48 = [&](int row) -> unsigned long long {
-            const unsigned char* rp = vc + row * L::RBV + g * 12 + half * 6;
-            const unsigned long long lo = *reinterpret_cast<const uint16_t*>(rp);
-            const unsigned long long mid = *reinterpret_cast<const uint16_t*>(rp + 2);
-            const unsigned long long hi = *reinterpret_cast<const uint16_t*>(rp + 4);
-            return lo | (mid << 16) | (hi << 32);
-          };
-          const unsigned long long fA = field48(2 * c), fB = field48(2 * c + 1);
-          const unsigned long long fC = field48(2 * c + 8), fD = field48(2 * c + 9);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int mt = half * 8 + k;
-            const uint32_t tA = tl[((uint32_t)(fA >> (6 * k)) & 63u) << 5];
-            const uint32_t tB = tl[((uint32_t)(fB >> (6 * k)) & 63u) << 5];
-            const uint32_t tC = tl[((uint32_t)(fC >> (6 * k)) & 63u) << 5];
-            const uint32_t tD = tl[((uint32_t)(fD >> (6 * k)) & 63u) << 5];
-            uint32_t a[4];
-            a[0] = prmt(tA, tB, 0x5410);
-            a[1] = prmt(tA, tB, 0x7632);
-            a[2] = prmt(tC, tD, 0x5410);
-            a[3] = prmt(tC, tD, 0x7632);
-#pragma unroll
-            for (int nt = 0; nt < NTH; ++nt)
-              mma16816(acc[nt][mt], a[0], a[1], a[2], a[3], pbw[nt][0], pbw[nt][1], acc[nt][mt]);
-          }
         }
       }
     } else {
@@ -1044,7 +1040,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   float* mrg = reinterpret_cast<float*>(smem);
   auto dim_of = [&](int mt, int row) -> int {  // PV m-tile row -> head dim
     if (VT == KVQ_F16) return 16 * mt + row;                       // row in 0..15
-    if (VT == KVQ_TURBO3) return (row & 7) * (D / 8) + 2 * mt + (row >> 3);
+    if (is_turbo(VT)) return (row & 7) * (D / 8) + 2 * mt + (row >> 3);
     return 32 * (mt >> 1) + 16 * (mt & 1) + 2 * (row & 7) + (row >> 3);  // q8_0, q4_0
   };
   const bool failed = cta_failed != 0;
@@ -1276,7 +1272,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         float o_v[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) o_v[e] = comb_failed ? __int_as_float(0x7fc00000) : num[hi][e] / den[hi];
-        if (VT == KVQ_TURBO3) {
+        if (is_turbo(VT)) {
           // o <- s * H_un * o / D: butterflies of strides 1 .. E/2 in registers,
           // E .. D/2 across lanes
 #pragma unroll
@@ -1301,7 +1297,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 #pragma unroll
           for (int e = 0; e < E; ++e) {
             const int d = lane * E + e;
-            const float sgn = ((p.t3.sign_bits[d >> 5] >> (d & 31)) & 1u) ? -1.f : 1.f;
+            const float sgn = ((p.tq.sign_bits[d >> 5] >> (d & 31)) & 1u) ? -1.f : 1.f;
             o_v[e] = o_v[e] * sgn / (float)D;
           }
         }
@@ -1339,40 +1335,44 @@ cudaError_t launch_one(const TcArgs& a, const TcMaps& m, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int KT, int VT, int NB>
+template <int KT, int VT, int NB, bool PAGED>
 cudaError_t launch_nb(int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st) {
-  if (a.p.block_table != nullptr)
-    return nth == 1 ? launch_one<KT, VT, NB, 1, true>(a, m, st) : launch_one<KT, VT, NB, 2, true>(a, m, st);
-  return nth == 1 ? launch_one<KT, VT, NB, 1, false>(a, m, st) : launch_one<KT, VT, NB, 2, false>(a, m, st);
+  return nth == 1 ? launch_one<KT, VT, NB, 1, PAGED>(a, m, st) : launch_one<KT, VT, NB, 2, PAGED>(a, m, st);
 }
 
-template <int KT, int VT>
+template <int KT, int VT, bool PAGED>
 cudaError_t launch_v(int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st) {
   switch (nb) {
-    case 2: return launch_nb<KT, VT, 2>(nth, a, m, st);
-    case 4: return launch_nb<KT, VT, 4>(nth, a, m, st);
+    case 2: return launch_nb<KT, VT, 2, PAGED>(nth, a, m, st);
+    case 4: return launch_nb<KT, VT, 4, PAGED>(nth, a, m, st);
     case 8:
       if constexpr (KT == KVQ_F16 && VT == KVQ_F16) return cudaErrorInvalidValue;
-      else return launch_nb<KT, VT, 8>(nth, a, m, st);
+      else return launch_nb<KT, VT, 8, PAGED>(nth, a, m, st);
   }
   return cudaErrorInvalidValue;
 }
 
-template <int KT>
+template <int KT, bool PAGED>
 cudaError_t launch_k(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st) {
   switch (vt) {
-    case KVQ_F16: return launch_v<KT, KVQ_F16>(nb, nth, a, m, st);
-    case KVQ_Q8_0: return launch_v<KT, KVQ_Q8_0>(nb, nth, a, m, st);
-    case KVQ_Q4_0: return launch_v<KT, KVQ_Q4_0>(nb, nth, a, m, st);
-    case KVQ_TURBO3: return launch_v<KT, KVQ_TURBO3>(nb, nth, a, m, st);
+    case KVQ_F16: return launch_v<KT, KVQ_F16, PAGED>(nb, nth, a, m, st);
+    case KVQ_Q8_0: return launch_v<KT, KVQ_Q8_0, PAGED>(nb, nth, a, m, st);
+    case KVQ_Q4_0: return launch_v<KT, KVQ_Q4_0, PAGED>(nb, nth, a, m, st);
+    case KVQ_TURBO2: return launch_v<KT, KVQ_TURBO2, PAGED>(nb, nth, a, m, st);
+    case KVQ_TURBO3: return launch_v<KT, KVQ_TURBO3, PAGED>(nb, nth, a, m, st);
+    case KVQ_TURBO4: return launch_v<KT, KVQ_TURBO4, PAGED>(nb, nth, a, m, st);
   }
   return cudaErrorInvalidValue;
 }
 
-// one per key type, each in its own translation unit
+// one per key type and cache kind (contiguous, paged pool), each in its own
+// translation unit so they compile in parallel
 cudaError_t launch_kf16(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq8(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq4(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kf16_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kq8_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kq4_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 
 }  // namespace tc
 }  // namespace kvq

@@ -6,7 +6,7 @@ namespace kvq {
 namespace tc {
 
 cudaError_t launch_kf16(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st) {
-  return launch_k<KVQ_F16>(vt, nb, nth, a, m, st);
+  return launch_k<KVQ_F16, false>(vt, nb, nth, a, m, st);
 }
 
 }  // namespace tc

@@ -6,7 +6,7 @@ namespace kvq {
 namespace tc {
 
 cudaError_t launch_kq4(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st) {
-  return launch_k<KVQ_Q4_0>(vt, nb, nth, a, m, st);
+  return launch_k<KVQ_Q4_0, false>(vt, nb, nth, a, m, st);
 }
 
 }  // namespace tc

@@ -23,7 +23,9 @@ int32_t code_bytes_of(int32_t type, int32_t d) {
     case KVQ_F16: return 2 * d;
     case KVQ_Q8_0: return d;
     case KVQ_Q4_0: return d / 2;
-    case KVQ_TURBO3: return 3 * d / 8;
+    case KVQ_TURBO2:
+    case KVQ_TURBO3:
+    case KVQ_TURBO4: return turbo_bits(type) * d / 8;
   }
   return 0;
 }
@@ -33,7 +35,9 @@ int32_t n_scales_of(int32_t type, int32_t d) {
     case KVQ_F16: return 0;
     case KVQ_Q8_0:
     case KVQ_Q4_0: return d / kBlock;
-    case KVQ_TURBO3: return 1;
+    case KVQ_TURBO2:
+    case KVQ_TURBO3:
+    case KVQ_TURBO4: return 1;
   }
   return 0;
 }
@@ -45,7 +49,7 @@ thread_local std::string g_last_cuda_error;
 constexpr int64_t kMaxCtx = (int64_t)1 << 31;
 constexpr int64_t kMinChunk = 256;  // fewest rows per split the heuristic plans
 
-bool known_type(int32_t t) { return t >= KVQ_F16 && t <= KVQ_TURBO3; }
+bool known_type(int32_t t) { return t >= KVQ_F16 && t <= KVQ_TURBO4; }
 bool pow2(int32_t v) { return v > 0 && (v & (v - 1)) == 0; }
 bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
 int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
@@ -74,55 +78,66 @@ void sign_bits(uint64_t seed, int32_t d, uint32_t out[kMaxHeadDim / 32]) {
     if (splitmix64_next(st) >> 63) out[i >> 5] |= 1u << (i & 31);
 }
 
-// 8-level Lloyd-Max quantizer of N(0,1) by Lloyd's iteration in double:
-// thresholds are midpoints of neighbouring levels, each level is the mean of
-// N(0,1) on its cell, (phi(a) - phi(b)) / (Q(a) - Q(b)) with Q the upper tail.
-// Symmetric: the positive half is iterated with the middle threshold at 0.
+// n-level Lloyd-Max quantizer of N(0,1) (n = 4, 8, 16) by Lloyd's iteration in
+// double: thresholds are midpoints of neighbouring levels, each level is the
+// mean of N(0,1) on its cell, (phi(a) - phi(b)) / (Q(a) - Q(b)) with Q the
+// upper tail.  Symmetric: the positive half is iterated with the middle
+// threshold at 0.
 struct Codebook {
-  float levels[8];
-  float tau[7];
+  int n;
+  float levels[16];
+  float tau[15];
 };
 
 double npdf(double x) { return std::exp(-0.5 * x * x) * 0.39894228040143267794; }
 double upper_tail(double x) { return 0.5 * std::erfc(x * 0.70710678118654752440); }
 
-Codebook compute_codebook() {
-  double c[4] = {0.3, 0.8, 1.4, 2.2};
-  for (int it = 0; it < 100000; ++it) {
-    double t[5] = {0.0, 0.5 * (c[0] + c[1]), 0.5 * (c[1] + c[2]), 0.5 * (c[2] + c[3]), INFINITY};
-    double next[4];
+Codebook compute_codebook(int n) {
+  const int m = n / 2;
+  double c[8];
+  for (int k = 0; k < m; ++k) c[k] = 2.5 * (k + 0.5) / m;  // start spread over [0, 2.5]
+  for (int it = 0; it < 400000; ++it) {
+    double t[9];
+    t[0] = 0.0;
+    for (int k = 1; k < m; ++k) t[k] = 0.5 * (c[k - 1] + c[k]);
+    t[m] = INFINITY;
+    double next[8];
     double change = 0.0;
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < m; ++k) {
       const double pa = npdf(t[k]), qa = upper_tail(t[k]);
       const double pb = std::isinf(t[k + 1]) ? 0.0 : npdf(t[k + 1]);
       const double qb = std::isinf(t[k + 1]) ? 0.0 : upper_tail(t[k + 1]);
       next[k] = (pa - pb) / (qa - qb);
       change = std::fmax(change, std::fabs(next[k] - c[k]));
     }
-    std::memcpy(c, next, sizeof(c));
+    std::memcpy(c, next, sizeof(double) * m);
     if (change < 1e-15) break;
   }
-  double lv[8];
-  for (int k = 0; k < 4; ++k) {
-    lv[4 + k] = c[k];
-    lv[3 - k] = -c[k];
+  double lv[16];
+  for (int k = 0; k < m; ++k) {
+    lv[m + k] = c[k];
+    lv[m - 1 - k] = -c[k];
   }
-  Codebook cb;
-  for (int k = 0; k < 8; ++k) cb.levels[k] = (float)lv[k];
-  for (int k = 0; k < 7; ++k) cb.tau[k] = (float)(0.5 * (lv[k] + lv[k + 1]));
+  Codebook cb{};
+  cb.n = n;
+  for (int k = 0; k < n; ++k) cb.levels[k] = (float)lv[k];
+  for (int k = 0; k + 1 < n; ++k) cb.tau[k] = (float)(0.5 * (lv[k] + lv[k + 1]));
   return cb;
 }
 
-const Codebook& codebook() {
+// The codebook of turbo type t, computed once per width.
+const Codebook& codebook(int32_t t) {
   static std::once_flag once;
-  static Codebook cb;
-  std::call_once(once, [] { cb = compute_codebook(); });
-  return cb;
+  static Codebook cb[3];
+  std::call_once(once, [] {
+    for (int b = 2; b <= 4; ++b) cb[b - 2] = compute_codebook(1 << b);
+  });
+  return cb[turbo_bits(t) - 2];
 }
 
-Turbo3Consts turbo3_consts(const kvq_cache_desc* d) {
-  Turbo3Consts t{};
-  const Codebook& cb = codebook();
+TurboConsts turbo_consts(const kvq_cache_desc* d, int32_t type) {
+  TurboConsts t{};
+  const Codebook& cb = codebook(type);
   std::memcpy(t.levels, cb.levels, sizeof(t.levels));
   std::memcpy(t.tau, cb.tau, sizeof(t.tau));
   sign_bits(d->turbo_seed, d->head_dim, t.sign_bits);
@@ -331,7 +346,7 @@ kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void*
   p.chunk = chunk_rows(ctx_len, S);
   p.ctx_lens = ctx_lens;
   p.qscale = softmax_scale * 1.4426950408889634f;
-  if (d->v_type == KVQ_TURBO3) p.t3 = turbo3_consts(d);
+  if (is_turbo(d->v_type)) p.tq = turbo_consts(d, d->v_type);
   p.append_pos = -1;
   p.out = nullptr;
   p.counters = nullptr;
@@ -377,7 +392,8 @@ kvq_status append_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, co
     }
     p.h_mul = div_multiplier((uint64_t)p.H);
     p.t_mul = div_multiplier((uint64_t)n_tok);
-    if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) p.t3 = turbo3_consts(d);
+    const int32_t type = which ? d->v_type : d->k_type;
+    if (is_turbo(type)) p.tq = turbo_consts(d, type);
   }
   const cudaError_t e = launch_append(do_k ? &ap[0] : nullptr, d->k_type, do_v ? &ap[1] : nullptr, d->v_type, s);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -426,7 +442,8 @@ kvq_status step_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, cons
     a.n_pages = p.n_pages;
     a.h_mul = div_multiplier((uint64_t)a.H);
     a.t_mul = div_multiplier(1);
-    if ((which ? d->v_type : d->k_type) == KVQ_TURBO3) a.t3 = turbo3_consts(d);
+    const int32_t type = which ? d->v_type : d->k_type;
+    if (is_turbo(type)) a.tq = turbo_consts(d, type);
   }
   p.out = out;
   p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + w.cnt_off);
@@ -462,7 +479,7 @@ const char* kvq_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
 
 size_t kvq_row_bytes(int32_t type, int32_t head_dim) {
   if (!known_type(type) || head_dim <= 0 || head_dim % kBlock || head_dim > kMaxHeadDim) return 0;
-  if (type == KVQ_TURBO3 && !pow2(head_dim)) return 0;
+  if (is_turbo(type) && !pow2(head_dim)) return 0;
   return (size_t)code_bytes_of(type, head_dim) + 2 * (size_t)n_scales_of(type, head_dim);
 }
 
@@ -473,8 +490,8 @@ kvq_status kvq_check_desc(const kvq_cache_desc* d) {
   if (d->max_ctx < 1 || d->max_ctx > kMaxCtx) return KVQ_ERR_INVALID;
   if (!known_type(d->k_type) || !known_type(d->v_type)) return KVQ_ERR_INVALID;
   if (d->head_dim % kBlock || d->head_dim > kMaxHeadDim) return KVQ_ERR_UNSUPPORTED;
-  if (d->k_type == KVQ_TURBO3) return KVQ_ERR_UNSUPPORTED;  // turbo3 is a value format
-  if (d->v_type == KVQ_TURBO3 && !pow2(d->head_dim)) return KVQ_ERR_UNSUPPORTED;
+  if (is_turbo(d->k_type)) return KVQ_ERR_UNSUPPORTED;  // the turbo formats are value formats
+  if (is_turbo(d->v_type) && !pow2(d->head_dim)) return KVQ_ERR_UNSUPPORTED;
   if (d->n_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }
@@ -553,10 +570,14 @@ size_t kvq_workspace_bytes(const kvq_cache_desc* d, int32_t batch, int32_t n_spl
 }
 
 kvq_status kvq_turbo3_codebook(float levels[8], float thresholds[7]) {
-  if (!levels || !thresholds) return KVQ_ERR_INVALID;
-  const Codebook& cb = codebook();
-  std::memcpy(levels, cb.levels, sizeof(cb.levels));
-  std::memcpy(thresholds, cb.tau, sizeof(cb.tau));
+  return kvq_turbo_codebook(KVQ_TURBO3, levels, thresholds);
+}
+
+kvq_status kvq_turbo_codebook(int32_t type, float* levels, float* thresholds) {
+  if (!levels || !thresholds || !is_turbo(type)) return KVQ_ERR_INVALID;
+  const Codebook& cb = codebook(type);
+  std::memcpy(levels, cb.levels, sizeof(float) * cb.n);
+  std::memcpy(thresholds, cb.tau, sizeof(float) * (cb.n - 1));
   return KVQ_OK;
 }
 
@@ -633,8 +654,8 @@ kvq_status kvq_combine(const kvq_cache_desc* d, const void* workspace, size_t wo
   p.n_q = d->n_q_heads;
   p.D = d->head_dim;
   p.S = S;
-  p.turbo3 = d->v_type == KVQ_TURBO3;
-  if (p.turbo3) p.t3 = turbo3_consts(d);
+  p.rotated = is_turbo(d->v_type);
+  if (p.rotated) p.tq = turbo_consts(d, d->v_type);
   const cudaError_t e = launch_combine(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return KVQ_OK;

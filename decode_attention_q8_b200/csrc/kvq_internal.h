@@ -25,9 +25,16 @@ struct Plane {
   int32_t n_scales;
 };
 
-struct Turbo3Consts {
-  float levels[8];
-  float tau[7];
+// Turbo value formats: 2, 3 or 4 bits per value, else 0.
+__host__ __device__ constexpr int turbo_bits(int32_t t) {
+  return t == KVQ_TURBO2 ? 2 : t == KVQ_TURBO3 ? 3 : t == KVQ_TURBO4 ? 4 : 0;
+}
+__host__ __device__ constexpr bool is_turbo(int32_t t) { return turbo_bits(t) != 0; }
+
+// A turbo type's codebook (2^b levels, 2^b - 1 thresholds) and sign bits.
+struct TurboConsts {
+  float levels[16];
+  float tau[15];
   uint32_t sign_bits[kMaxHeadDim / 32];  // bit i set -> s_i = -1
 };
 
@@ -50,7 +57,7 @@ struct AppendParams {
   int64_t n_pages;
   // n / H and n / n_tok for 32-bit n as the high half of n * mul (mul = 0: divisor 1)
   uint64_t h_mul, t_mul;
-  Turbo3Consts t3;
+  TurboConsts tq;
 };
 
 // Multiplier for exact division of any 32-bit n by d (d >= 1): n / d equals the
@@ -77,7 +84,7 @@ struct DecodeParams {
   int32_t max_pages, log2_page;
   int64_t n_pages;
   float qscale;        // softmax_scale * log2(e)
-  Turbo3Consts t3;     // V sign bits and codebook (turbo3 values)
+  TurboConsts tq;      // V sign bits and codebook (turbo values)
   // Fused decode step (kvq_decode_step); a plain decode has append_pos < 0 and
   // out == null.
   int64_t append_pos;    // row the new K/V rows are written to first (< 0: none;
@@ -96,8 +103,8 @@ struct CombineParams {
   const float* ws_acc;
   float* out;          // [B][n_q][D]
   int32_t B, n_q, D, S;
-  int32_t turbo3;      // apply s * H_un * (.) / D
-  Turbo3Consts t3;
+  int32_t rotated;     // turbo values: apply s * H_un * (.) / D
+  TurboConsts tq;
 };
 
 // Host-side helpers (kvq_api.cu).

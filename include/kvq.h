@@ -42,6 +42,11 @@
  *              codes packed 3 bits each, little-endian (code i in bits
  *              3i..3i+2); stored norm fp16(min(norm, 65504)).  3d/8 + 2 bytes.
  *              Decoded value: x_hat = (norm/d) * s * H_un * c[code].
+ *   KVQ_TURBO2, KVQ_TURBO4 (values only) the same row at 2 and 4 bits per value:
+ *              the 4- and 16-level Lloyd-Max quantizers of N(0,1) (3 and 15
+ *              midpoints), code i in bits b*i .. b*i+b-1.  The TurboQuant page's
+ *              FAQ ("¿Qué formato TurboQuant debería usar?") puts values at 2 to 3
+ *              bits; 4 bits is the next width.  d/4 + 2 and d/2 + 2 bytes.
  *
  * Memory layout of one cache tensor (K or V) of one layer, in device memory
  * owned by the caller:
@@ -94,7 +99,9 @@ typedef enum {
   KVQ_F16 = 0,
   KVQ_Q8_0 = 1,
   KVQ_Q4_0 = 2,
-  KVQ_TURBO3 = 3
+  KVQ_TURBO3 = 3,
+  KVQ_TURBO2 = 4,
+  KVQ_TURBO4 = 5
 } kvq_type;
 
 typedef enum {
@@ -173,7 +180,13 @@ KVQ_API size_t kvq_workspace_bytes(const kvq_cache_desc* desc, int32_t batch, in
  * the 7 binary32 thresholds between them.  Host only; no device needed. */
 KVQ_API kvq_status kvq_turbo3_codebook(float levels[8], float thresholds[7]);
 
-/* The turbo3 sign vector (+1.f / -1.f) for `seed`, head_dim entries.  Host only. */
+/* The codebook of a turbo type (KVQ_TURBO2, KVQ_TURBO3, KVQ_TURBO4): its 2^b
+ * binary32 levels (ascending) into levels[] and the 2^b - 1 binary32
+ * thresholds into thresholds[] (room for 16 and 15).  Host only. */
+KVQ_API kvq_status kvq_turbo_codebook(int32_t type, float* levels, float* thresholds);
+
+/* The turbo3 sign vector (+1.f / -1.f) for `seed`, head_dim entries (every
+ * turbo type uses it).  Host only. */
 KVQ_API kvq_status kvq_turbo3_signs(uint64_t seed, int32_t head_dim, float* signs);
 
 /*

@@ -7,7 +7,7 @@ import numpy as np
 import torch
 
 import decode_attention_q8_b200 as kvq
-from oracle import attention, blocks, turbo3
+from oracle import attention, blocks, turbo, turbo3
 
 SENTINEL = 0xA5
 
@@ -51,6 +51,9 @@ def oracle_rows(kind, x_f16, seed=0):
     if kind == "turbo3":
         nrm, codes = turbo3.quantize_turbo3(x, seed)
         return codes, nrm.reshape(n, 1)
+    if kind in ("turbo2", "turbo4"):
+        nrm, codes = turbo.quantize(x, seed, turbo.BITS[kind])
+        return codes, nrm.reshape(n, 1)
     raise ValueError(kind)
 
 
@@ -64,6 +67,8 @@ def oracle_dequant(kind, codes, scales, D, seed=0):
         return blocks.dequantize_q4_0(scales, codes)
     if kind == "turbo3":
         return turbo3.dequantize_turbo3(scales[:, 0], codes, seed, D)
+    if kind in ("turbo2", "turbo4"):
+        return turbo.dequantize(scales[:, 0], codes, seed, D, turbo.BITS[kind])
     raise ValueError(kind)
 
 

@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 
 import decode_attention_q8_b200 as kvq
-from oracle import cache_model, turbo3
+from oracle import cache_model, turbo, turbo3
 from conftest import ROOT, read_golden
 
 HEADER = os.path.join(ROOT, "include", "kvq.h")
@@ -46,10 +46,12 @@ def test_row_bytes_match_oracle_model():
         for d in (32, 64, 128, 256):
             assert kvq.kvq_row_bytes(t, d) == cache_model.row_bytes(t, d)
     for d in (32, 64, 128, 256):
-        assert kvq.kvq_row_bytes("turbo3", d) == cache_model.row_bytes("turbo3", d)
+        for t in ("turbo2", "turbo3", "turbo4"):
+            assert kvq.kvq_row_bytes(t, d) == cache_model.row_bytes(t, d)
     assert kvq.kvq_row_bytes("q8_0", 48) == 0
     assert kvq.kvq_row_bytes("turbo3", 96) == 0
     assert kvq.kvq_row_bytes(7, 128) == 0
+    assert kvq.kvq_row_bytes("turbo2", 96) == 0
 
 
 def test_cache_bytes_reproduce_pages():
@@ -84,6 +86,14 @@ def test_turbo3_codebook_equals_oracle():
     np.testing.assert_array_equal(np.array(th, np.float32), oth)
 
 
+@pytest.mark.parametrize("kind", ["turbo2", "turbo3", "turbo4"])
+def test_turbo_codebooks_equal_oracle(kind):
+    lv, th = kvq.kvq_turbo_codebook(kind)
+    olv, oth = turbo.codebook_f32(turbo.BITS[kind])
+    np.testing.assert_array_equal(np.array(lv, np.float32), olv)
+    np.testing.assert_array_equal(np.array(th, np.float32), oth)
+
+
 @pytest.mark.parametrize("seed", [0, 1, 1234567, 0x7475726233, 2**64 - 1])
 def test_turbo3_signs_equal_oracle(seed):
     for d in (32, 128, 256):
@@ -103,6 +113,10 @@ def test_check_desc():
         (kvq.make_desc(64, 8, 512, "q8_0", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),  # head_dim > 256
         (kvq.make_desc(64, 8, 128, "turbo3", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),  # turbo3 K
         (kvq.make_desc(64, 8, 96, "q8_0", "turbo3", 16), kvq.KVQ_ERR_UNSUPPORTED),   # WHT needs 2^k
+        (kvq.make_desc(64, 8, 128, "turbo2", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),  # value formats only
+        (kvq.make_desc(64, 8, 128, "turbo4", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),
+        (kvq.make_desc(64, 8, 96, "q8_0", "turbo4", 16), kvq.KVQ_ERR_UNSUPPORTED),
+        (kvq.make_desc(64, 8, 128, 6, "q4_0", 16), kvq.KVQ_ERR_INVALID),           # past the last type
     ]
     for desc, st in bad:
         assert kvq.kvq_check_desc(desc) == st
