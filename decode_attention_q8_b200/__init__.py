@@ -37,7 +37,7 @@ EXPORTED = (
     "kvq_decode_attention", "kvq_combine", "kvq_decode_attention_noalloc", "kvq_decode_step",
     "kvq_decode_attention_varlen", "kvq_decode_step_varlen", "kvq_append_quantize_varlen",
     "kvq_paged_layout", "kvq_paged_cache_bytes", "kvq_append_quantize_paged", "kvq_decode_attention_paged",
-    "kvq_decode_step_paged",
+    "kvq_decode_step_paged", "kvq_partials_region", "kvq_combine_ranks",
 )
 
 
@@ -112,6 +112,9 @@ _sigs = {
                                                   ctypes.c_float, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "kvq_decode_step_paged": (ctypes.c_int, [_D, _P, _P, _P, _P, _P, ctypes.c_int32, _PG, _P, ctypes.c_int64,
                                              ctypes.c_float, ctypes.c_int32, _P, ctypes.c_size_t, _P, _P]),
+    "kvq_partials_region": (ctypes.c_int, [_D, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t),
+                                           ctypes.POINTER(ctypes.c_size_t)]),
+    "kvq_combine_ranks": (ctypes.c_int, [_D, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P]),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -343,6 +346,48 @@ def kvq_decode_step_paged(desc, k_pool, v_pool, q, k_new, v_new, batch, pages, c
                                              softmax_scale, n_splits, _ptr(workspace), workspace_bytes, _ptr(out),
                                              _stream(stream)),
                   "kvq_decode_step_paged")
+
+
+def kvq_partials_region(desc, batch, n_splits):
+    """(byte offset, bytes) of the split partials inside a workspace."""
+    off, n = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.kvq_partials_region(ctypes.byref(desc), batch, n_splits, ctypes.byref(off), ctypes.byref(n)),
+           "kvq_partials_region")
+    return off.value, n.value
+
+
+def kvq_combine_ranks(desc, partials, n_ranks, batch, n_splits, out, stream=None):
+    """Merge n_ranks ranks' gathered partial regions (rank after rank) into ``out``."""
+    return _check(_lib.kvq_combine_ranks(ctypes.byref(desc), _ptr(partials), n_ranks, batch, n_splits, _ptr(out),
+                                         _stream(stream)),
+                  "kvq_combine_ranks")
+
+
+def gather_partials(region, group=None):
+    """All-gather every rank's partial region (a 1-D uint8 tensor) into one
+    buffer, rank after rank: the exchange step of a context split across GPUs."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    out = torch.empty(world * region.numel(), dtype=region.dtype, device=region.device)
+    if dist.get_backend(group) == "nccl":
+        dist.all_gather_into_tensor(out, region, group=group)
+    else:
+        dist.all_gather(list(out.chunk(world)), region, group=group)
+    return out
+
+
+def decode_context_parallel(desc, k_cache, v_cache, q, batch, ctx_len, softmax_scale, n_splits, workspace, out,
+                            group=None):
+    """Context split across GPUs: this rank decodes its own ctx_len rows
+    (kvq_decode_attention), the ranks' partials are all-gathered, and every
+    rank combines all of them into ``out`` (kvq_combine_ranks).  Everything
+    runs on torch's current stream, which the collective also orders on."""
+    import torch.distributed as dist
+    kvq_decode_attention(desc, k_cache, v_cache, q, batch, ctx_len, softmax_scale, n_splits, workspace)
+    off, n = kvq_partials_region(desc, batch, n_splits)
+    gathered = gather_partials(workspace[off:off + n], group)
+    return kvq_combine_ranks(desc, gathered, dist.get_world_size(group), batch, n_splits, out)
 
 
 def raw_status(name, *args):

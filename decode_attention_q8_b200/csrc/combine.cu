@@ -37,34 +37,42 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) 
 // is L2-resident behind the decode kernel).
 __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
   extern __shared__ float sm[];
+  const int SS = p.S * p.n_ranks;  // splits of all ranks
   float* red = sm;              // 8 floats
-  float* wts = sm + 8;          // S weights
-  float* xs = wts + p.S;        // D values (turbo inverse transform)
+  float* wts = sm + 8;          // SS weights
+  float* xs = wts + SS;         // D values (turbo inverse transform)
   const int h = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
   const int64_t base = ((int64_t)b * p.n_q + h) * p.S;
+  // split k = r * S + s: rank r's split s
+  auto at = [&](int k) -> int64_t { return (int64_t)(k / p.S) * p.rank_stride + base + k % p.S; };
   float M = -INFINITY;
-  for (int s = j; s < p.S; s += blockDim.x) M = fmaxf(M, p.ws_m[base + s]);
+  for (int s = j; s < SS; s += blockDim.x) M = fmaxf(M, p.ws_m[at(s)]);
   M = block_reduce(M, true, red);
   float den = 0.f;
-  for (int s = j; s < p.S; s += blockDim.x) {
-    const float ms = p.ws_m[base + s];
+  for (int s = j; s < SS; s += blockDim.x) {
+    const float ms = p.ws_m[at(s)];
     const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);  // empty split: weight 0
     wts[s] = w;
-    den += w * p.ws_l[base + s];
+    den += w * p.ws_l[at(s)];
   }
   den = block_reduce(den, false, red);  // its barriers also publish wts[]
-  const float* acc = p.ws_acc + base * p.D + j;
   float num = 0.f;
   int s = 0;
   constexpr int kU = 16;  // independent loads per round: the partials may come from HBM
-  for (; s + kU <= p.S; s += kU) {
-    float a[kU];
+  if (p.n_ranks == 1) {
+    const float* acc = p.ws_acc + base * p.D + j;
+    for (; s + kU <= SS; s += kU) {
+      float a[kU];
 #pragma unroll
-    for (int u = 0; u < kU; ++u) a[u] = acc[(int64_t)(s + u) * p.D];
+      for (int u = 0; u < kU; ++u) a[u] = acc[(int64_t)(s + u) * p.D];
 #pragma unroll
-    for (int u = 0; u < kU; ++u) num = fmaf(wts[s + u], a[u], num);
+      for (int u = 0; u < kU; ++u) num = fmaf(wts[s + u], a[u], num);
+    }
   }
-  for (; s < p.S; ++s) num = fmaf(wts[s], acc[(int64_t)s * p.D], num);
+  for (; s < SS; ++s) {
+    const int64_t k = (int64_t)(s / p.S) * p.rank_stride + (base + s % p.S) * p.D + j;
+    num = fmaf(wts[s], p.ws_acc[k], num);
+  }
   float o = num / den;
   if (p.rotated) {
     xs[j] = o;
@@ -87,7 +95,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st) {
   const dim3 grid(p.n_q, p.B);
-  const size_t smem = (8 + (size_t)p.S + (size_t)p.D) * sizeof(float);
+  const size_t smem = (8 + (size_t)p.S * p.n_ranks + (size_t)p.D) * sizeof(float);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
   combine_kernel<<<grid, p.D, smem, st>>>(p);
   return cudaGetLastError();

@@ -654,6 +654,48 @@ kvq_status kvq_combine(const kvq_cache_desc* d, const void* workspace, size_t wo
   p.n_q = d->n_q_heads;
   p.D = d->head_dim;
   p.S = S;
+  p.n_ranks = 1;
+  p.rank_stride = 0;
+  p.rotated = is_turbo(d->v_type);
+  if (p.rotated) p.tq = turbo_consts(d, d->v_type);
+  const cudaError_t e = launch_combine(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KVQ_OK;
+}
+
+kvq_status kvq_partials_region(const kvq_cache_desc* d, int32_t batch, int32_t n_splits, size_t* offset,
+                               size_t* bytes) {
+  kvq_status st = kvq_check_desc(d);
+  if (st != KVQ_OK) return st;
+  if (!offset || !bytes || batch < 1 || batch > 65535 || n_splits < 1 || n_splits > kMaxSplits)
+    return KVQ_ERR_INVALID;
+  const WsLayout w = ws_layout(d, batch, n_splits);
+  *offset = (size_t)w.m_off;
+  *bytes = (size_t)(w.total - w.m_off);
+  return KVQ_OK;
+}
+
+kvq_status kvq_combine_ranks(const kvq_cache_desc* d, const void* partials, int32_t n_ranks, int32_t batch,
+                             int32_t n_splits, float* out, void* stream) {
+  kvq_status st = kvq_check_desc(d);
+  if (st != KVQ_OK) return st;
+  if (!partials || !out || n_ranks < 1 || n_ranks > 4096) return KVQ_ERR_INVALID;
+  if (batch < 1 || batch > 65535 || n_splits < 1 || n_splits > kMaxSplits) return KVQ_ERR_INVALID;
+  if ((int64_t)n_ranks * n_splits > 8192) return KVQ_ERR_UNSUPPORTED;  // the combine's weight array
+  if (!aligned(partials, 16) || !aligned(out, 16)) return KVQ_ERR_INVALID;
+  const WsLayout w = ws_layout(d, batch, n_splits);
+  const uint8_t* base = static_cast<const uint8_t*>(partials);
+  CombineParams p{};
+  p.ws_m = reinterpret_cast<const float*>(base);
+  p.ws_l = reinterpret_cast<const float*>(base + (w.l_off - w.m_off));
+  p.ws_acc = reinterpret_cast<const float*>(base + (w.acc_off - w.m_off));
+  p.out = out;
+  p.B = batch;
+  p.n_q = d->n_q_heads;
+  p.D = d->head_dim;
+  p.S = n_splits;
+  p.n_ranks = n_ranks;
+  p.rank_stride = (w.total - w.m_off) / 4;
   p.rotated = is_turbo(d->v_type);
   if (p.rotated) p.tq = turbo_consts(d, d->v_type);
   const cudaError_t e = launch_combine(p, static_cast<cudaStream_t>(stream));

@@ -103,6 +103,11 @@ struct CombineParams {
   const float* ws_acc;
   float* out;          // [B][n_q][D]
   int32_t B, n_q, D, S;
+  // Partials of several ranks (context split across GPUs), rank after rank:
+  // rank r's m, l and acc start rank_stride floats after rank r-1's; the
+  // n_ranks * S partials of a query head are merged as one set of splits.
+  int32_t n_ranks;     // 1: one workspace
+  int64_t rank_stride;
   int32_t rotated;     // turbo values: apply s * H_un * (.) / D
   TurboConsts tq;
 };

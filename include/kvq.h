@@ -234,6 +234,27 @@ KVQ_API kvq_status kvq_combine(const kvq_cache_desc* desc, const void* workspace
                        int32_t n_splits, float* out, void* cuda_stream);
 
 /*
+ * Context split across GPUs.  The sequences' rows are spread over n_ranks GPUs
+ * (any partition, a rank may hold none of a sequence's rows).  Each rank runs
+ * kvq_decode_attention (or _varlen) over its own rows with the same explicit
+ * n_splits.  The ranks' partial regions (m, l, acc; kvq_partials_region) are
+ * then gathered rank after rank into one buffer, and kvq_combine_ranks merges
+ * all n_ranks * n_splits partials.  Partials merge exactly, so the output is
+ * that of one decode over all the rows, up to fp32 rounding order (section
+ * "Flash Attention" of "llama.cpp für Geschwindigkeit und Speicher optimieren":
+ * the tiled softmax is exact).
+ *   kvq_partials_region: byte offset and size of the partials inside a
+ *     workspace for (batch, n_splits); host only.
+ *   partials: device, n_ranks regions of that size back to back, 16-byte
+ *     aligned (an all-gather of each rank's region).
+ *   n_ranks * n_splits <= 8192.
+ */
+KVQ_API kvq_status kvq_partials_region(const kvq_cache_desc* desc, int32_t batch, int32_t n_splits,
+                                       size_t* offset, size_t* bytes);
+KVQ_API kvq_status kvq_combine_ranks(const kvq_cache_desc* desc, const void* partials, int32_t n_ranks,
+                                     int32_t batch, int32_t n_splits, float* out, void* cuda_stream);
+
+/*
  * Allocation-free decode: kvq_decode_attention followed by kvq_combine, with the
  * split partials kept in scratch memory that the library itself owns, so the
  * caller passes only inputs and the output.  The pages have no counterpart; it

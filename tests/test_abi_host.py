@@ -285,6 +285,27 @@ def test_paged_entry_points_reject_before_launch():
     assert kvq.kvq_paged_cache_bytes(d, 16, 10, 0) == 0
 
 
+def test_partials_region_is_the_workspace_tail():
+    """The partials (m, l, acc) follow the counters and epoch words and run to
+    the end of the workspace."""
+    d = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 32768)
+    r256 = lambda v: (v + 255) // 256 * 256
+    for B, S in ((1, 37), (4, 9), (16, 3)):
+        off, n = kvq.kvq_partials_region(d, B, S)
+        assert off == r256(B * 8 * 8)
+        assert off + n == kvq.kvq_workspace_bytes(d, B, S)
+    for bad in ((0, 4), (1, 0), (1, 5000)):
+        with pytest.raises(kvq.KvqError):
+            kvq.kvq_partials_region(d, *bad)
+    rank = lambda **kw: kvq.raw_status("kvq_combine_ranks", ctypes.byref(d), kw.get("parts", FAKE), kw.get("r", 2),
+                                        1, kw.get("s", 4), kw.get("out", FAKE), None)
+    assert rank(parts=None) == kvq.KVQ_ERR_INVALID
+    assert rank(r=0) == kvq.KVQ_ERR_INVALID
+    assert rank(s=0) == kvq.KVQ_ERR_INVALID
+    assert rank(parts=FAKE + 4) == kvq.KVQ_ERR_INVALID
+    assert rank(r=4096, s=4) == kvq.KVQ_ERR_UNSUPPORTED  # more weights than the combine holds
+
+
 def test_workspace_bytes_formula():
     d = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 32768)
     B, S = 4, 9

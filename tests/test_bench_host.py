@@ -122,6 +122,37 @@ def test_max_over_ranks_on_two_gloo_ranks():
         assert gbs == pytest.approx(2 * 2e9 * 4 / 11e-3 / 1e9)
 
 
+def _gather_main(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import decode_attention_q8_b200 as kvq
+        region = torch.arange(10, dtype=torch.uint8) + 100 * rank  # this rank's partials, as bytes
+        q.put((rank, kvq.gather_partials(region).tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_partials_gather_is_rank_major_on_two_gloo_ranks():
+    """The exchange step of a context split: every rank ends with all ranks'
+    partial regions back to back, rank 0 first."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    expect = list(range(10)) + [100 + i for i in range(10)]
+    assert sorted(got) == [(0, expect), (1, expect)]
+
+
 def test_reference_arm_runs_on_rank_zero_only():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
