@@ -1135,12 +1135,14 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       const unsigned int e0 = p.comb_ctas > 1 ? *reinterpret_cast<volatile unsigned int*>(p.epochs + plane) : 0u;
       if (p.comb_ctas > 1) __threadfence();
       const unsigned int ticket = atomicInc(p.counters + plane, (unsigned)(p.S - 1));
+      // a counter left outside [0, S) by a caller (it must start at 0) gives a
+      // ticket above S - 1: a huge rank, so that CTA only arrives
       const unsigned int rank = (unsigned)(p.S - 1) - ticket;
       int failed = 0;
       if (rank == 0) {
         __threadfence();
         if (p.comb_ctas > 1) atomicAdd(p.epochs + plane, 1u);
-      } else if ((int)rank < p.comb_ctas) {
+      } else if (rank < (unsigned)p.comb_ctas) {
         const unsigned long long w0 = global_ns();
         while (*reinterpret_cast<volatile unsigned int*>(p.epochs + plane) == e0) {
           if (global_ns() - w0 > kWaitLimitNs) {
@@ -1155,8 +1157,8 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       comb_wait_failed = failed;
     }
     __syncthreads();
-    const int rank = (int)comb_rank;
-    if (rank < p.comb_ctas) {
+    if (comb_rank < (unsigned)p.comb_ctas) {
+      const int rank = (int)comb_rank;
       __threadfence();
       // the partials were written through the generic proxy by other CTAs and
       // are read here by bulk copies (the async proxy)

@@ -235,3 +235,39 @@ def test_combine_shared_by_the_last_arrivals(B, n_q, n_kv):
             out = _step(desc, kc, vc, q, k, v, B, ctx, scale, S, ws)
             _check_out(desc, q, k, v, out, ctx, scale, f"B{B} G{n_q // n_kv} S={S} call {call}", groups=groups)
             assert not ws[:4 * B * n_kv].cpu().numpy().any()
+
+
+def test_missing_arrival_times_out_to_nan():
+    """Failure detection without a fault: group 0's arrival counter is left
+    outside [0, S) (the contract asks for 0), so no CTA of that group becomes
+    its last arrival.  The CTAs that would share its combine wait for an epoch
+    bump that never comes; each wait gives up after its bound (about 2 s) and
+    writes NaN for its heads.  The other groups are unaffected, and the GPU
+    context stays usable: the next call on a zeroed workspace is correct."""
+    import time
+    B, n_q, n_kv, D, ctx, S = 1, 64, 8, 128, 16384, 40   # 8 heads x 40 splits: several CTAs combine
+    desc, q, k, v = _inputs("q8_0", "q4_0", B, n_q, n_kv, D, ctx, seed=17)
+    kc, vc = alloc_cache(desc, B, 0), alloc_cache(desc, B, 1)
+    kvq.kvq_append_quantize(desc, kc, vc, k[:, :ctx - 1].contiguous(), v[:, :ctx - 1].contiguous(), B, 0, ctx - 1)
+    scale = 1 / math.sqrt(D)
+    good = _step(desc, kc, vc, q, k, v, B, ctx, scale, S, _workspace(desc, B, S))
+    ws = _workspace(desc, B, S)
+    ws.view(torch.int32)[0] = -1                      # group (0, 0): counter 0xffffffff
+    out = torch.full((B, n_q, D), 12345.0, dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.time()
+    kvq.kvq_decode_step(desc, kc, vc, q, k[:, ctx - 1].contiguous(), v[:, ctx - 1].contiguous(), B, ctx, scale, S,
+                        ws, out)
+    torch.cuda.synchronize()
+    waited = time.time() - t0
+    G = n_q // n_kv
+    o = out.cpu().numpy()
+    g0 = o[0, :G]
+    nan_heads = [h for h in range(G) if np.isnan(g0[h]).all()]
+    untouched = [h for h in range(G) if (g0[h] == 12345.0).all()]
+    assert nan_heads and sorted(nan_heads + untouched) == list(range(G)), (nan_heads, untouched)
+    assert waited > 1.0, waited
+    assert torch.equal(out[:, G:], good[:, G:])       # the other groups
+    # the context is usable: a fresh workspace gives the right output again
+    again = _step(desc, kc, vc, q, k, v, B, ctx, scale, S, _workspace(desc, B, S))
+    assert torch.equal(again, good)
