@@ -1,4 +1,4 @@
-"""Oracle for the 32-element block cache formats q8_0 and q4_0, and the f16 row.
+"""Oracle for the 32-element block cache formats q8_0, q4_0 and q5_0, and the f16 row.
 
 Test infrastructure only (see ``oracle/__init__.py``).
 
@@ -16,6 +16,12 @@ library implements; the pages print none of it:
   q4_0: m = the signed x_j of largest magnitude; d = m / -8;
         q_j = min(15, trunc(x_j * (1/d) + 8.5)); element j goes to the low
         nibble of byte j and element j+16 to its high nibble; store d as fp16.
+  q5_0: q4_0 widened by one bit: d = m / -16; q_j = min(31, trunc(x_j * (1/d)
+        + 16.5)); the low four bits of q_j are packed as q4_0's nibbles and bit 4
+        of q_j is bit j of a little-endian 32-bit word qh; store d as fp16.  (A
+        comment in the llama.cpp issue reports q5_0/q5_0 caches as a usable
+        middle ground between q8_0 and q4_0; no page prints q5_0's arithmetic,
+        so this widening of q4_0 is a reading.)
 
 Readings taken where the definition is silent:
   * the fp32 d, not its fp16 image, is used to compute q_j;
@@ -131,6 +137,57 @@ def quantize_q4_0(x_f16):
 def dequantize_q4_0(d_f16, qs):
     """x_hat_j = double(d_h) * (q_j - 8), in float64."""
     codes = unpack_q4_0(qs).astype(np.float64) - 8.0
+    d = np.asarray(d_f16, dtype=np.float16).astype(np.float64)
+    n = codes.shape[-1]
+    return (codes.reshape(*codes.shape[:-1], n // QK, QK) * d[..., None]).reshape(codes.shape)
+
+
+def quantize_q5_0_codes(x_f16):
+    """Quantize rows to q5_0; returns ``(d, codes)``: ``d`` float16 ``[..., n/32]``,
+    ``codes`` uint8 in 0..31 ``[..., n]`` (the q4_0 steps with -16, 16.5, 31)."""
+    lead = np.asarray(x_f16).shape[:-1]
+    n = np.asarray(x_f16).shape[-1]
+    x = _blocks_f32(x_f16)
+    j = np.argmax(np.abs(x), axis=1)               # first (lowest) index on ties
+    m = x[np.arange(x.shape[0]), j]
+    d = m / F32(-16.0)
+    inv = np.zeros_like(d)
+    nz = d != 0
+    inv[nz] = F32(1.0) / d[nz]
+    t = (x * inv[:, None]) + F32(16.5)             # two binary32 roundings
+    q = np.minimum(31, t.astype(np.int32))         # truncation; t >= 0.5
+    return (d.astype(np.float16).reshape(*lead, n // QK),
+            q.astype(np.uint8).reshape(*lead, n))
+
+
+def pack_q5_0(codes):
+    """(qs, qh): the low four bits as q4_0's nibbles ``[..., n/2]`` and bit 4 of
+    element j as bit j of a uint32 per block ``[..., n/32]``."""
+    c = np.asarray(codes, dtype=np.uint8)
+    n = c.shape[-1]
+    qs = pack_q4_0(c & 0x0F)
+    b = (c.reshape(*c.shape[:-1], n // QK, QK) >> 4).astype(np.uint64) & 1
+    qh = np.sum(b << np.arange(QK, dtype=np.uint64), axis=-1).astype(np.uint32)
+    return qs, qh
+
+
+def unpack_q5_0(qs, qh):
+    low = unpack_q4_0(qs)
+    h = np.asarray(qh, dtype=np.uint32)
+    bits = ((h[..., None] >> np.arange(QK, dtype=np.uint32)) & 1).astype(np.uint8)
+    return low | (bits.reshape(low.shape) << 4)
+
+
+def quantize_q5_0(x_f16):
+    """Quantize rows to q5_0; returns ``(d, qs, qh)``."""
+    d, codes = quantize_q5_0_codes(x_f16)
+    qs, qh = pack_q5_0(codes)
+    return d, qs, qh
+
+
+def dequantize_q5_0(d_f16, qs, qh):
+    """x_hat_j = double(d_h) * (q_j - 16), in float64."""
+    codes = unpack_q5_0(qs, qh).astype(np.float64) - 16.0
     d = np.asarray(d_f16, dtype=np.float16).astype(np.float64)
     n = codes.shape[-1]
     return (codes.reshape(*codes.shape[:-1], n // QK, QK) * d[..., None]).reshape(codes.shape)

@@ -3,7 +3,8 @@
 Test infrastructure only (see ``oracle/__init__.py``).
 
 Per 32 elements: f16 64 bytes, q8_0 34 bytes (fp16 scale + 32 int8),
-q4_0 18 bytes (fp16 scale + 16 bytes of nibbles).  turbo2 / turbo3 / turbo4
+q4_0 18 bytes (fp16 scale + 16 bytes of nibbles), q5_0 22 bytes (fp16 scale, 16 bytes of
+nibbles, a 32-bit word of fifth bits).  turbo2 / turbo3 / turbo4
 per row of d elements: 2d/8, 3d/8, 4d/8 bytes of codes + an fp16 norm.  Nominal costs are on
 ``llama.cpp für Geschwindigkeit und Speicher optimieren``, section
 "KV-Cache-Präzision" (2 / 1 / 0.5 bytes per element); the exact block sizes
@@ -11,7 +12,7 @@ are pinned by the cache sizes the KVSplit page and the llama.cpp issue print
 (see ``tests/golden/kv_cache_bytes.txt``).
 """
 
-BYTES_PER_32 = {"f16": 64, "q8_0": 34, "q4_0": 18}
+BYTES_PER_32 = {"f16": 64, "q8_0": 34, "q4_0": 18, "q5_0": 22}
 
 
 def row_bytes(kind, d):

@@ -135,6 +135,72 @@ def test_q4_0_pack_roundtrip_and_order():
     assert packed[0, 16 + 5] >> 4 == codes[0, 32 + 21]
 
 
+def test_q5_0_codes_and_bounds():
+    """Every unclamped element at the nearest point of the grid -16..15 (times
+    d = m / -16), the largest-magnitude element at code 0, the opposite extreme
+    clamped to 31, and the qualified round-trip bound with the stored fp16 d."""
+    rng = np.random.default_rng(5)
+    x16 = np.concatenate([_rand_blocks(rng, 4000), _adversarial_blocks(rng)])
+    d_h, codes = blocks.quantize_q5_0_codes(x16)
+    x = x16.astype(np.float64)
+    assert codes.max() <= 31
+    j = np.argmax(np.abs(x), axis=1)
+    m = x[np.arange(len(x)), j]
+    nz = m != 0
+    assert np.all(codes[np.arange(len(x)), j][nz] == 0)
+    assert np.all(codes[~nz] == 16)
+    d = m[nz] / -16.0
+    r = x[nz] / d[:, None]                      # in [-16, 16]
+    c = codes[nz].astype(np.float64) - 16.0
+    unclamped = r < 15.5 - 1e-5
+    assert np.all(np.abs(r - c)[unclamped] <= 0.5 + 1e-5)
+    assert np.all(c[r > 15.5 + 1e-5] == 15)
+    dh = d_h[:, 0].astype(np.float64)[nz]
+    err = np.abs(x[nz] - dh[:, None] * c)
+    bound_un = np.abs(d)[:, None] / 2 * (1 + 1e-5) + 32 * np.abs(d - dh)[:, None]
+    bound_cl = np.abs(d)[:, None] * (1 + 1e-5) + 32 * np.abs(d - dh)[:, None]
+    assert np.all(np.where(unclamped, err <= bound_un + 1e-12, err <= bound_cl + 1e-12))
+
+
+def test_q5_0_closed_form_block():
+    """x_j = j - 16: m = -16 (index 0), d = 1, q_j = j; the fifth bits are
+    those of j >= 16, each byte holds (j, j + 16 mod 16) = j | j << 4, and
+    the block dequantizes to x exactly."""
+    x = (np.arange(32) - 16).astype(np.float16)[None]
+    d, qs, qh = blocks.quantize_q5_0(x)
+    assert float(d[0, 0]) == 1.0
+    assert int(qh[0, 0]) == 0xFFFF0000
+    assert qs[0].tolist() == [j | (j << 4) for j in range(16)]
+    np.testing.assert_array_equal(blocks.dequantize_q5_0(d, qs, qh)[0], np.arange(32) - 16.0)
+    # and the same block negated: m = +16 at index 0... index 0 holds -16 -> +16, d = -1
+    d2, qs2, qh2 = blocks.quantize_q5_0(-x)
+    assert float(d2[0, 0]) == -1.0
+    np.testing.assert_array_equal(blocks.dequantize_q5_0(d2, qs2, qh2)[0], -(np.arange(32) - 16.0))
+
+
+def test_q5_0_is_q4_0_widened():
+    """q5_0's grid step (|m|/16) is half of q4_0's (|m|/8), so over many blocks
+    its largest error per block is about half of q4_0's."""
+    rng = np.random.default_rng(6)
+    x16 = _rand_blocks(rng, 2000)
+    d4, c4 = blocks.quantize_q4_0_codes(x16)
+    d5, c5 = blocks.quantize_q5_0_codes(x16)
+    x = x16.astype(np.float64)
+    e4 = np.abs(x - d4.astype(np.float64) * (c4.astype(np.float64) - 8)).max(axis=1)
+    e5 = np.abs(x - d5.astype(np.float64) * (c5.astype(np.float64) - 16)).max(axis=1)
+    assert 0.4 < np.mean(e5) / np.mean(e4) < 0.6
+
+
+def test_q5_0_pack_roundtrip_and_order():
+    rng = np.random.default_rng(7)
+    codes = rng.integers(0, 32, size=(5, 128)).astype(np.uint8)
+    qs, qh = blocks.pack_q5_0(codes)
+    assert qs.shape == (5, 64) and qh.shape == (5, 4) and qh.dtype == np.uint32
+    np.testing.assert_array_equal(blocks.unpack_q5_0(qs, qh), codes)
+    assert (int(qh[0, 1]) >> 7) & 1 == codes[0, 32 + 7] >> 4
+    assert qs[0, 16 + 5] & 0xF == codes[0, 32 + 5] & 0xF
+
+
 def test_f16_identity():
     x = np.array([[1.5, -2.0, 65504.0, 2.0 ** -24]], np.float16)
     np.testing.assert_array_equal(blocks.dequantize_f16(x), x.astype(np.float64))
