@@ -24,9 +24,9 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-KVQ_F16, KVQ_Q8_0, KVQ_Q4_0, KVQ_TURBO3, KVQ_TURBO2, KVQ_TURBO4 = 0, 1, 2, 3, 4, 5
+KVQ_F16, KVQ_Q8_0, KVQ_Q4_0, KVQ_TURBO3, KVQ_TURBO2, KVQ_TURBO4, KVQ_Q5_0 = 0, 1, 2, 3, 4, 5, 6
 TYPES = {"f16": KVQ_F16, "q8_0": KVQ_Q8_0, "q4_0": KVQ_Q4_0, "turbo3": KVQ_TURBO3, "turbo2": KVQ_TURBO2,
-         "turbo4": KVQ_TURBO4}
+         "turbo4": KVQ_TURBO4, "q5_0": KVQ_Q5_0}
 
 KVQ_OK, KVQ_ERR_INVALID, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA = 0, 1, 2, 3, 4
 

@@ -15,7 +15,7 @@ constexpr int kBlockRound = 1;   // q8_0 / q4_0 blocks per thread and round (a b
 // Work items of one row in this kernel: a 32-element block for q8_0 / q4_0,
 // otherwise the row bodies' threads.
 __host__ __device__ constexpr int bulk_items(int32_t type, int d) {
-  return type == KVQ_Q8_0 || type == KVQ_Q4_0 ? d / kBlock : rows::row_threads(type, d);
+  return type == KVQ_Q8_0 || type == KVQ_Q4_0 || type == KVQ_Q5_0 ? d / kBlock : rows::row_threads(type, d);
 }
 
 // K and V rows of one append call in one launch.  Every CTA takes its share of
@@ -61,7 +61,8 @@ __device__ __forceinline__ void append_blocks(const AppendParams& p, int64_t fir
       const int64_t g = base + u * stride;
       if (g < nblk) {
         if constexpr (TYPE == KVQ_Q8_0) rows::q8_0_block(p, g, raw[u]);
-        else rows::q4_0_block(p, g, raw[u]);
+        else if constexpr (TYPE == KVQ_Q4_0) rows::q4_0_block(p, g, raw[u]);
+        else rows::q5_0_block(p, g, raw[u]);
       }
     }
   }
@@ -83,6 +84,7 @@ __device__ __forceinline__ void append_part(const AppendParams& p, int32_t type,
     case KVQ_F16: append_stream<KVQ_F16, 0>(p, first, stride, gend); break;
     case KVQ_Q8_0: append_blocks<KVQ_Q8_0>(p, first, stride, gend); break;
     case KVQ_Q4_0: append_blocks<KVQ_Q4_0>(p, first, stride, gend); break;
+    case KVQ_Q5_0: append_blocks<KVQ_Q5_0>(p, first, stride, gend); break;
     case KVQ_TURBO2: append_turbo_part<KVQ_TURBO2>(p, first, stride, gend); break;
     case KVQ_TURBO3: append_turbo_part<KVQ_TURBO3>(p, first, stride, gend); break;
     case KVQ_TURBO4: append_turbo_part<KVQ_TURBO4>(p, first, stride, gend); break;

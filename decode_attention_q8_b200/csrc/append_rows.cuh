@@ -35,7 +35,7 @@ template <int TYPE, int E>
 __device__ __forceinline__ uint4 load_raw(const AppendParams& p, int64_t gtid, int64_t gend) {
   uint4 r = make_uint4(0u, 0u, 0u, 0u);
   if (gtid >= gend) return r;
-  if constexpr (TYPE == KVQ_Q8_0 || TYPE == KVQ_Q4_0) {
+  if constexpr (TYPE == KVQ_Q8_0 || TYPE == KVQ_Q4_0 || TYPE == KVQ_Q5_0) {
     const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.src + gtid * 4));
     r.x = v.x;
     r.y = v.y;
@@ -183,6 +183,58 @@ __device__ __forceinline__ void append_q4_0(const AppendParams& p, int64_t gtid,
   if (sub == 0) p.dst.scales[r * p.dst.n_scales + blk] = __float2half_rn(d);
 }
 
+// q5_0: q4_0 widened by one bit: d = m / -16; q = min(31, trunc(fl(fl(x * fl(1/d))
+// + 16.5))); the low nibbles as q4_0's, bit 4 of element j in bit j of qh, which
+// sits in the scale plane after the row's block scales (two fp16 slots).
+__device__ __forceinline__ void append_q5_0(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
+  const int nb = p.D / kBlock;
+  const int64_t gblk = gtid >> 3;
+  const int sub = (int)(gtid & 7);
+  const bool active = gtid < gend;
+  float x[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) x[i] = raw_elem(raw, i);  // zeros past gend
+  float bm = x[0];
+  int bi = sub * 4;
+#pragma unroll
+  for (int i = 1; i < 4; ++i)
+    if (fabsf(x[i]) > fabsf(bm)) { bm = x[i]; bi = sub * 4 + i; }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, bm, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    const float a = fabsf(bm), b = fabsf(om);
+    if (b > a || (b == a && oi < bi)) { bm = om; bi = oi; }
+  }
+  const float d = __fdiv_rn(bm, -16.0f);
+  const float id = (d != 0.0f) ? __frcp_rn(d) : 0.0f;
+  uint32_t nib = 0, h = 0;  // 4 low nibbles, one per byte; their fifth bits
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float t = __fadd_rn(__fmul_rn(x[i], id), 16.5f);
+    const int q = min(31, __float2int_rz(t));
+    nib |= (uint32_t)(q & 15) << (8 * i);
+    h |= (uint32_t)(q >> 4) << i;
+  }
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, nib, 4);
+  uint32_t qh = h << (4 * sub);  // elements 4 sub .. 4 sub + 3
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) qh |= __shfl_xor_sync(0xffffffffu, qh, o);
+  if (!active || sub >= 4) return;
+  const uint32_t bytes = nib | (hi << 4);
+  const int64_t row = gblk >> log2_blocks(p);
+  const int blk = (int)(gblk & (nb - 1));
+  const int64_t r = dst_row(p, row);
+  if (r < 0) return;
+  *reinterpret_cast<uint32_t*>(p.dst.codes + r * p.dst.code_bytes + blk * 16 + sub * 4) = bytes;
+  if (sub == 0) {
+    __half* sc = p.dst.scales + r * p.dst.n_scales;
+    sc[blk] = __float2half_rn(d);
+    sc[nb + 2 * blk] = __ushort_as_half((unsigned short)(qh & 0xFFFF));
+    sc[nb + 2 * blk + 1] = __ushort_as_half((unsigned short)(qh >> 16));
+  }
+}
+
 // ---- Bulk mapping for q8_0 / q4_0: one thread per 32-element block ----------
 // The 8-lane bodies above keep the latency of one row low (the fused decode
 // step appends one row per KV head).  Many rows at once are bound by
@@ -310,6 +362,44 @@ __device__ __forceinline__ void q4_0_block(const AppendParams& p, int64_t gblk, 
   p.dst.scales[r * p.dst.n_scales + blk] = __float2half_rn(d);
 }
 
+// q5_0 of one block (same definition as append_q5_0).
+__device__ __forceinline__ void q5_0_block(const AppendParams& p, int64_t gblk, const BlockRaw& raw) {
+  float bm = block_elem(raw, 0);
+#pragma unroll
+  for (int i = 1; i < kBlock; ++i) {
+    const float x = block_elem(raw, i);
+    if (fabsf(x) > fabsf(bm)) bm = x;  // strictly larger: the first index wins ties
+  }
+  const float d = __fdiv_rn(bm, -16.0f);
+  const float id = d != 0.0f ? __frcp_rn(d) : 0.0f;
+  uint32_t q[kBlock];
+  uint32_t qh = 0;
+#pragma unroll
+  for (int i = 0; i < kBlock; ++i) {
+    q[i] = (uint32_t)min(31, __float2int_rz(__fadd_rn(__fmul_rn(block_elem(raw, i), id), 16.5f)));
+    qh |= (q[i] >> 4) << i;
+  }
+  uint32_t word[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {  // byte j = low nibbles of q_j and q_{j+16}
+    uint32_t b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) b[i] = (q[4 * w + i] & 15) | ((q[4 * w + i + 16] & 15) << 4);
+    word[w] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+  }
+  int64_t r;
+  int blk;
+  block_dst(p, gblk, r, blk);
+  if (r < 0) return;
+  *reinterpret_cast<uint4*>(p.dst.codes + r * p.dst.code_bytes + blk * (kBlock / 2)) =
+      make_uint4(word[0], word[1], word[2], word[3]);
+  const int nb = p.D / kBlock;
+  __half* sc = p.dst.scales + r * p.dst.n_scales;
+  sc[blk] = __float2half_rn(d);
+  sc[nb + 2 * blk] = __ushort_as_half((unsigned short)(qh & 0xFFFF));
+  sc[nb + 2 * blk + 1] = __ushort_as_half((unsigned short)(qh >> 16));
+}
+
 // f16: copy rows, 16 bytes per thread.
 __device__ __forceinline__ void append_f16(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
   const int per_row = p.D / 8;  // 16-byte chunks per row (a power of two)
@@ -412,6 +502,7 @@ template <int TYPE, int E>
 __device__ __forceinline__ void finish(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
   if constexpr (TYPE == KVQ_Q8_0) append_q8_0(p, gtid, gend, raw);
   else if constexpr (TYPE == KVQ_Q4_0) append_q4_0(p, gtid, gend, raw);
+  else if constexpr (TYPE == KVQ_Q5_0) append_q5_0(p, gtid, gend, raw);
   else if constexpr (TYPE == KVQ_F16) append_f16(p, gtid, gend, raw);
   else append_turbo<turbo_bits(TYPE), E>(p, gtid, gend, raw);
 }
@@ -438,6 +529,7 @@ __device__ __forceinline__ void append_any(int32_t type, const AppendParams& p, 
     case KVQ_F16: append_one<KVQ_F16, 0>(p, gtid, gend); break;
     case KVQ_Q8_0: append_one<KVQ_Q8_0, 0>(p, gtid, gend); break;
     case KVQ_Q4_0: append_one<KVQ_Q4_0, 0>(p, gtid, gend); break;
+    case KVQ_Q5_0: append_one<KVQ_Q5_0, 0>(p, gtid, gend); break;
     case KVQ_TURBO2: append_turbo_any<KVQ_TURBO2>(p, gtid, gend); break;
     case KVQ_TURBO3: append_turbo_any<KVQ_TURBO3>(p, gtid, gend); break;
     case KVQ_TURBO4: append_turbo_any<KVQ_TURBO4>(p, gtid, gend); break;

@@ -112,6 +112,7 @@ int ctas_k(int32_t v_type, int32_t D) {
     case KVQ_F16: return tc::ctas_per_sm_for(KT, KVQ_F16, D);
     case KVQ_Q8_0: return tc::ctas_per_sm_for(KT, KVQ_Q8_0, D);
     case KVQ_Q4_0: return tc::ctas_per_sm_for(KT, KVQ_Q4_0, D);
+    case KVQ_Q5_0: return tc::ctas_per_sm_for(KT, KVQ_Q5_0, D);
     case KVQ_TURBO2: return tc::ctas_per_sm_for(KT, KVQ_TURBO2, D);
     case KVQ_TURBO3: return tc::ctas_per_sm_for(KT, KVQ_TURBO3, D);
     case KVQ_TURBO4: return tc::ctas_per_sm_for(KT, KVQ_TURBO4, D);
@@ -125,6 +126,7 @@ int decode_ctas_per_sm(int32_t k_type, int32_t v_type, int32_t D) {
     case KVQ_F16: return ctas_k<KVQ_F16>(v_type, D);
     case KVQ_Q8_0: return ctas_k<KVQ_Q8_0>(v_type, D);
     case KVQ_Q4_0: return ctas_k<KVQ_Q4_0>(v_type, D);
+    case KVQ_Q5_0: return ctas_k<KVQ_Q5_0>(v_type, D);
   }
   return 1;
 }
@@ -147,6 +149,7 @@ cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p,
       case KVQ_F16: return tc::launch_kf16_paged(v_type, nb, nth, a, maps, st);
       case KVQ_Q8_0: return tc::launch_kq8_paged(v_type, nb, nth, a, maps, st);
       case KVQ_Q4_0: return tc::launch_kq4_paged(v_type, nb, nth, a, maps, st);
+      case KVQ_Q5_0: return tc::launch_kq5_paged(v_type, nb, nth, a, maps, st);
     }
     return cudaErrorInvalidValue;
   }
@@ -154,6 +157,7 @@ cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p,
     case KVQ_F16: return tc::launch_kf16(v_type, nb, nth, a, maps, st);
     case KVQ_Q8_0: return tc::launch_kq8(v_type, nb, nth, a, maps, st);
     case KVQ_Q4_0: return tc::launch_kq4(v_type, nb, nth, a, maps, st);
+    case KVQ_Q5_0: return tc::launch_kq5(v_type, nb, nth, a, maps, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -70,10 +70,10 @@ constexpr int kHalf = 16;    // rows per MMA row block (two per tile)
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 __host__ __device__ constexpr int code_bytes(int t, int d) {
-  return t == KVQ_F16 ? 2 * d : t == KVQ_Q8_0 ? d : t == KVQ_Q4_0 ? d / 2 : turbo_bits(t) * d / 8;
+  return t == KVQ_F16 ? 2 * d : t == KVQ_Q8_0 ? d : (t == KVQ_Q4_0 || t == KVQ_Q5_0) ? d / 2 : turbo_bits(t) * d / 8;
 }
 __host__ __device__ constexpr int n_scales(int t, int d) {
-  return t == KVQ_F16 ? 0 : is_turbo(t) ? 1 : d / 32;
+  return t == KVQ_F16 ? 0 : is_turbo(t) ? 1 : t == KVQ_Q5_0 ? 3 * d / 32 : d / 32;
 }
 // swizzle of a code plane: 16-byte chunk index XOR ((offset >> 7) & mask)
 __host__ __device__ constexpr int swz_mask(int t, int d) {
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   constexpr int S = L::kStages;
   constexpr int KMASK = swz_mask(KT, D), VMASK = swz_mask(VT, D);
   constexpr int NMT = D / 16;  // PV m-tiles
-  constexpr bool kVQ = VT == KVQ_Q8_0 || VT == KVQ_Q4_0;  // block-scaled integer values
+  constexpr bool kVQ = VT == KVQ_Q8_0 || VT == KVQ_Q4_0 || VT == KVQ_Q5_0;  // block-scaled integer values
   const DecodeParams& p = args.p;
 
   extern __shared__ unsigned char smem_raw[];
@@ -455,7 +455,12 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       tma_load_4d(kc_of(st), &tm_kc, 0, 0, r0, tplane, &bars[st], pol);
     else
       tma_load_3d(kc_of(st), &tm_kc, 0, r0, tplane, &bars[st], pol);
-    if (L::NSK) tma_load_2d(ks_of(st), &tm_ks, r0 * L::NSK / 2, tplane, &bars[st], pol);
+    if (L::NSK) {  // flat words while a tile is at most 256 of them, else row-wise
+      if (kSub * L::NSK / 2 <= 256)
+        tma_load_2d(ks_of(st), &tm_ks, r0 * L::NSK / 2, tplane, &bars[st], pol);
+      else
+        tma_load_3d(ks_of(st), &tm_ks, 0, r0, tplane, &bars[st], pol);
+    }
     if (is_turbo(VT)) {
       if (kSub * L::RBV / 4 <= 256)
         tma_load_2d(vc_of(st), &tm_vc, r0 * L::RBV / 4, tplane, &bars[st], pol);
@@ -466,7 +471,12 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     } else {
       tma_load_3d(vc_of(st), &tm_vc, 0, r0, tplane, &bars[st], pol);
     }
-    if (L::NSV) tma_load_2d(vs_of(st), &tm_vs, r0 * L::NSV / 2, tplane, &bars[st], pol);
+    if (L::NSV) {
+      if (kSub * L::NSV / 2 <= 256)
+        tma_load_2d(vs_of(st), &tm_vs, r0 * L::NSV / 2, tplane, &bars[st], pol);
+      else
+        tma_load_3d(vs_of(st), &tm_vs, 0, r0, tplane, &bars[st], pol);
+    }
   };
   // Fused decode step: the new row (row append_pos) lies in tile jt of warp wt
   // of the CTA whose split holds it.  That warp issues its other first tiles,
@@ -512,14 +522,14 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   //      -8 * sum(q), in the same 2^-24 units.
   uint32_t qb[NTH][NB][2][2];
   float cq[NTH][NB][4];
-  constexpr float kBiasK = KT == KVQ_Q8_0 ? 128.f : KT == KVQ_Q4_0 ? 8.f : 0.f;
+  constexpr float kBiasK = KT == KVQ_Q8_0 ? 128.f : KT == KVQ_Q4_0 ? 8.f : KT == KVQ_Q5_0 ? 16.f : 0.f;
 #pragma unroll
   for (int nt = 0; nt < NTH; ++nt) {
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk) {
       const uint32_t* r = qraw[nt][blk];
       uint32_t w0 = r[0], w1 = r[1], w2 = r[2], w3 = r[3];
-      if (KT == KVQ_Q4_0) {
+      if (KT == KVQ_Q4_0 || KT == KVQ_Q5_0) {
         w0 = prmt(r[0], r[1], 0x5410);  // (4c, 4c+2)
         w1 = prmt(r[0], r[1], 0x7632);  // (4c+1, 4c+3)
         w2 = prmt(r[2], r[3], 0x5410);
@@ -538,7 +548,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       // lane (g', c') needs the sums of heads 2c', 2c'+1 (held by groups 2c', 2c'+1)
       const float s0 = __shfl_sync(0xffffffffu, part, (2 * c) * 4);
       const float s1 = __shfl_sync(0xffffffffu, part, (2 * c + 1) * 4);
-      if (KT == KVQ_Q4_0) {
+      if (KT == KVQ_Q4_0 || KT == KVQ_Q5_0) {
         w2 = hmul2_u32(w2, kHalfSixteenth);
         w3 = hmul2_u32(w3, kHalfSixteenth);
       }
@@ -630,7 +640,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         a[1][2] = prmt(u2, 0u, 0x4342);
         a[1][1] = prmt(u3, 0u, 0x4140);
         a[1][3] = prmt(u3, 0u, 0x4342);
-      } else if constexpr (KT == KVQ_Q4_0) {
+      } else if constexpr (KT == KVQ_Q4_0 || KT == KVQ_Q5_0) {
         // one x4 load covers blocks blk (regs 0, 1) and blk + 1 (regs 2, 3):
         // reg = bytes 4c..4c+3 of the block in row g (even regs) or g+8 (odd)
         if ((blk & 1) == 0) ldmatrix_x4(kr, kbase ^ blk_xor(KT, L::RBK, blk));
@@ -644,6 +654,21 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         a[0][3] = wbs & 0x000F000Fu;
         a[1][1] = wb & 0x00F000F0u;
         a[1][3] = wbs & 0x00F000F0u;
+        if constexpr (KT == KVQ_Q5_0) {
+          // fifth bits of rows g and g+8 (bit j of the block's qh word: dim j):
+          // bit 4 of a low-nibble half, bit 8 of a high-nibble half
+          const int hw = NB + 2 * blk;  // the block's qh word, in fp16 slots
+          const uint32_t xa = *reinterpret_cast<const uint32_t*>(ksc + g * L::NSK + hw) >> (4 * c);
+          const uint32_t xb = *reinterpret_cast<const uint32_t*>(ksc + (g + 8) * L::NSK + hw) >> (4 * c);
+          a[0][0] |= ((xa << 4) & 0x10u) | ((xa << 18) & 0x100000u);    // dims 4c, 4c+2
+          a[0][2] |= ((xa << 3) & 0x10u) | ((xa << 17) & 0x100000u);    // dims 4c+1, 4c+3
+          a[1][0] |= ((xa >> 8) & 0x100u) | ((xa << 6) & 0x1000000u);   // dims 4c+16, 4c+18
+          a[1][2] |= ((xa >> 9) & 0x100u) | ((xa << 5) & 0x1000000u);   // dims 4c+17, 4c+19
+          a[0][1] |= ((xb << 4) & 0x10u) | ((xb << 18) & 0x100000u);
+          a[0][3] |= ((xb << 3) & 0x10u) | ((xb << 17) & 0x100000u);
+          a[1][1] |= ((xb >> 8) & 0x100u) | ((xb << 6) & 0x1000000u);
+          a[1][3] |= ((xb >> 9) & 0x100u) | ((xb << 5) & 0x1000000u);
+        }
       } else {  // f16
 #pragma unroll
         for (int s2 = 0; s2 < 2; ++s2) {
@@ -774,8 +799,18 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       // (128 or 8) times sum_t d[t][blk] p[t] comes from one more MMA per half
       // tile whose A operand is the block-scale matrix (m = block, k = row).
       // Scales of rows (2c, 2c+1) and (2c+8, 2c+9) are adjacent.
-      uint32_t sAB[L::NSV], sCD[L::NSV];  // words: row 2c blocks | row 2c+1 blocks
-      if (L::NSV == 2) {
+      constexpr int NSD = VT == KVQ_Q5_0 ? NB : L::NSV;  // block scales per row
+      uint32_t sAB[NSD], sCD[NSD];  // words: row 2c blocks | row 2c+1 blocks
+      if constexpr (VT == KVQ_Q5_0) {
+        // a q5_0 row's qh words follow its scales: the two rows are read apart
+#pragma unroll
+        for (int i = 0; i < NB / 2; ++i) {
+          sAB[i] = *reinterpret_cast<const uint32_t*>(vsc + 2 * c * L::NSV + 2 * i);
+          sAB[NB / 2 + i] = *reinterpret_cast<const uint32_t*>(vsc + (2 * c + 1) * L::NSV + 2 * i);
+          sCD[i] = *reinterpret_cast<const uint32_t*>(vsc + (2 * c + 8) * L::NSV + 2 * i);
+          sCD[NB / 2 + i] = *reinterpret_cast<const uint32_t*>(vsc + (2 * c + 9) * L::NSV + 2 * i);
+        }
+      } else if (L::NSV == 2) {
         const uint2 x = *reinterpret_cast<const uint2*>(vsc + 2 * c * L::NSV);
         const uint2 y = *reinterpret_cast<const uint2*>(vsc + (2 * c + 8) * L::NSV);
         sAB[0] = x.x; sAB[1] = x.y; sCD[0] = y.x; sCD[1] = y.y;
@@ -788,16 +823,16 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           sCD[4 * i] = y.x; sCD[4 * i + 1] = y.y; sCD[4 * i + 2] = y.z; sCD[4 * i + 3] = y.w;
         }
       }
-      // row 2c's scales are words 0 .. NSV/2-1, row 2c+1's are NSV/2 ..
+      // row 2c's scales are words 0 .. NSD/2-1, row 2c+1's are NSD/2 ..
       {
-        uint32_t xa = sAB[0], xb = sAB[L::NSV / 2], xc = sCD[0], xd = sCD[L::NSV / 2];
+        uint32_t xa = sAB[0], xb = sAB[NSD / 2], xc = sCD[0], xd = sCD[NSD / 2];
 #pragma unroll
-        for (int i = 1; i < L::NSV / 2; ++i) {
+        for (int i = 1; i < NSD / 2; ++i) {
           const bool hit = (g >> 1) == i;
           xa = hit ? sAB[i] : xa;
-          xb = hit ? sAB[L::NSV / 2 + i] : xb;
+          xb = hit ? sAB[NSD / 2 + i] : xb;
           xc = hit ? sCD[i] : xc;
-          xd = hit ? sCD[L::NSV / 2 + i] : xd;
+          xd = hit ? sCD[NSD / 2 + i] : xd;
         }
         const uint32_t oa0 = prmt(xa, xb, osel) & omask, oa2 = prmt(xc, xd, osel) & omask;
 #pragma unroll
@@ -815,8 +850,8 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
         const uint32_t sel = (blk & 1) ? 0x7632u : 0x5410u;
-        const uint32_t dAB = prmt(sAB[blk >> 1], sAB[L::NSV / 2 + (blk >> 1)], sel);
-        const uint32_t dCD = prmt(sCD[blk >> 1], sCD[L::NSV / 2 + (blk >> 1)], sel);
+        const uint32_t dAB = prmt(sAB[blk >> 1], sAB[NSD / 2 + (blk >> 1)], sel);
+        const uint32_t dCD = prmt(sCD[blk >> 1], sCD[NSD / 2 + (blk >> 1)], sel);
         uint32_t pbw[NTH][2];
 #pragma unroll
         for (int nt = 0; nt < NTH; ++nt) {
@@ -828,7 +863,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           }
         }
         uint32_t a0[4], a1[4];  // m-tiles (blk, 0) and (blk, 1)
-        if (VT == KVQ_Q4_0) {
+        if (VT == KVQ_Q4_0 || VT == KVQ_Q5_0) {
           // trans load: reg = [row 2c: bytes 2g, 2g+1 | row 2c+1: bytes 2g, 2g+1]
           // of the block -> dims 2g, 2g+1 (low nibbles), 2g+16, 2g+17 (high)
           if ((blk & 1) == 0) ldmatrix_x4_trans(vr, vbase ^ blk_xor(VT, L::RBV, blk));
@@ -842,6 +877,23 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           a1[1] = w1s & 0x00F000F0u;
           a1[2] = w2 & 0x00F000F0u;
           a1[3] = w2s & 0x00F000F0u;
+          if constexpr (VT == KVQ_Q5_0) {
+            // fifth bits (bit j of a row's qh word: dim j): 16 more in the code,
+            // bit 4 of a low-nibble half, bit 8 of a high-nibble half
+            const int hw = NB + 2 * blk;  // the block's qh word, in fp16 slots
+            const uint32_t xA = *reinterpret_cast<const uint32_t*>(vsc + 2 * c * L::NSV + hw) >> (2 * g);
+            const uint32_t xB = *reinterpret_cast<const uint32_t*>(vsc + (2 * c + 1) * L::NSV + hw) >> (2 * g);
+            const uint32_t xC = *reinterpret_cast<const uint32_t*>(vsc + (2 * c + 8) * L::NSV + hw) >> (2 * g);
+            const uint32_t xD = *reinterpret_cast<const uint32_t*>(vsc + (2 * c + 9) * L::NSV + hw) >> (2 * g);
+            a0[0] |= ((xA << 4) & 0x10u) | ((xB << 20) & 0x100000u);  // dim 2g
+            a0[1] |= ((xA << 3) & 0x10u) | ((xB << 19) & 0x100000u);  // dim 2g+1
+            a0[2] |= ((xC << 4) & 0x10u) | ((xD << 20) & 0x100000u);
+            a0[3] |= ((xC << 3) & 0x10u) | ((xD << 19) & 0x100000u);
+            a1[0] |= ((xA >> 8) & 0x100u) | ((xB << 8) & 0x1000000u);  // dim 2g+16
+            a1[1] |= ((xA >> 9) & 0x100u) | ((xB << 7) & 0x1000000u);  // dim 2g+17
+            a1[2] |= ((xC >> 8) & 0x100u) | ((xD << 8) & 0x1000000u);
+            a1[3] |= ((xC >> 9) & 0x100u) | ((xD << 7) & 0x1000000u);
+          }
         } else {
           // q8_0 trans load of segments 2blk (regs 0, 1) and 2blk+1 (regs 2, 3):
           // reg = [row 2c: bytes 2g, 2g+1 | row 2c+1: bytes 2g, 2g+1]
@@ -1009,7 +1061,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   // ---- q8_0 / q4_0 values: take the 2^24 (2^20) out and subtract the code
   //      offset times sum_t d[t][blk] p[t] (held by lane 4 * blk + c)
   if constexpr (kVQ) {
-    constexpr float vb = VT == KVQ_Q8_0 ? 128.f : 8.f;
+    constexpr float vb = VT == KVQ_Q8_0 ? 128.f : VT == KVQ_Q5_0 ? 16.f : 8.f;
 #pragma unroll
     for (int nt = 0; nt < NTH; ++nt) {
 #pragma unroll
@@ -1019,7 +1071,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int mt = 2 * blk + h;
-          const float f = (VT == KVQ_Q4_0 && h == 1) ? kTwo20 : kTwo24;
+          const float f = ((VT == KVQ_Q4_0 || VT == KVQ_Q5_0) && h == 1) ? kTwo20 : kTwo24;
           acc[nt][mt][0] = fmaf(acc[nt][mt][0], f, o0);
           acc[nt][mt][1] = fmaf(acc[nt][mt][1], f, o1);
           acc[nt][mt][2] = fmaf(acc[nt][mt][2], f, o0);
@@ -1360,6 +1412,7 @@ cudaError_t launch_k(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, 
     case KVQ_F16: return launch_v<KT, KVQ_F16, PAGED>(nb, nth, a, m, st);
     case KVQ_Q8_0: return launch_v<KT, KVQ_Q8_0, PAGED>(nb, nth, a, m, st);
     case KVQ_Q4_0: return launch_v<KT, KVQ_Q4_0, PAGED>(nb, nth, a, m, st);
+    case KVQ_Q5_0: return launch_v<KT, KVQ_Q5_0, PAGED>(nb, nth, a, m, st);
     case KVQ_TURBO2: return launch_v<KT, KVQ_TURBO2, PAGED>(nb, nth, a, m, st);
     case KVQ_TURBO3: return launch_v<KT, KVQ_TURBO3, PAGED>(nb, nth, a, m, st);
     case KVQ_TURBO4: return launch_v<KT, KVQ_TURBO4, PAGED>(nb, nth, a, m, st);
@@ -1372,9 +1425,11 @@ cudaError_t launch_k(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, 
 cudaError_t launch_kf16(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq8(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq4(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kq5(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kf16_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq8_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq4_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kq5_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 
 }  // namespace tc
 }  // namespace kvq

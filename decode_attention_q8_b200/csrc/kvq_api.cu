@@ -22,7 +22,8 @@ int32_t code_bytes_of(int32_t type, int32_t d) {
   switch (type) {
     case KVQ_F16: return 2 * d;
     case KVQ_Q8_0: return d;
-    case KVQ_Q4_0: return d / 2;
+    case KVQ_Q4_0:
+    case KVQ_Q5_0: return d / 2;
     case KVQ_TURBO2:
     case KVQ_TURBO3:
     case KVQ_TURBO4: return turbo_bits(type) * d / 8;
@@ -35,6 +36,7 @@ int32_t n_scales_of(int32_t type, int32_t d) {
     case KVQ_F16: return 0;
     case KVQ_Q8_0:
     case KVQ_Q4_0: return d / kBlock;
+    case KVQ_Q5_0: return 3 * d / kBlock;
     case KVQ_TURBO2:
     case KVQ_TURBO3:
     case KVQ_TURBO4: return 1;
@@ -49,7 +51,7 @@ thread_local std::string g_last_cuda_error;
 constexpr int64_t kMaxCtx = (int64_t)1 << 31;
 constexpr int64_t kMinChunk = 256;  // fewest rows per split the heuristic plans
 
-bool known_type(int32_t t) { return t >= KVQ_F16 && t <= KVQ_TURBO4; }
+bool known_type(int32_t t) { return t >= KVQ_F16 && t <= KVQ_Q5_0; }
 bool pow2(int32_t v) { return v > 0 && (v & (v - 1)) == 0; }
 bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
 int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }

@@ -31,6 +31,12 @@
  *              d = m / -8, q_j = min(15, trunc(fl(fl(x_j * fl(1/d)) + 8.5))),
  *              element j in the low nibble of byte j, element j+16 in the high
  *              nibble; d == 0 gives nibble 8.  18 bytes.
+ *   KVQ_Q5_0   q4_0 widened by one bit: d = m / -16, q_j = min(31, trunc(fl(fl(
+ *              x_j * fl(1/d)) + 16.5))); the low four bits of q_j are packed as
+ *              q4_0's nibbles and bit 4 of q_j is bit j of a 32-bit word qh;
+ *              d == 0 gives q_j = 16.  22 bytes.  (A comment in the llama.cpp
+ *              issue reports q5_0/q5_0 caches as a usable middle ground; no page
+ *              prints its arithmetic.)
  *   KVQ_TURBO3 (values only; head_dim a power of two) one row of head_dim
  *              elements: signs s_i = -1 when output i of splitmix64(turbo_seed)
  *              has its top bit set; v = s*x; norm = sqrtf(tree sum of v_i^2,
@@ -54,7 +60,9 @@
  *   code plane  at byte 0:           [batch][n_kv_heads][T][code_bytes]
  *   scale plane at byte scale_offset: [batch][n_kv_heads][T][n_scales] fp16
  *   with code_bytes = 2d (f16), d (q8_0), d/2 (q4_0), 3d/8 (turbo3);
- *   n_scales = 0 (f16), d/32 (q8_0, q4_0), 1 (turbo3, the norm);
+ *   n_scales = 0 (f16), d/32 (q8_0, q4_0), 3d/32 (q5_0: the d/32 block scales,
+ *   then the d/32 qh words, each as two fp16 slots, little-endian), 1 (turbo
+ *   types, the norm);
  *   scale_offset = code plane bytes rounded up to a multiple of 256.
  *   Within a row, q8_0 codes and q4_0 bytes are in block order, exactly as the
  *   block formats above; scale n of a row belongs to block n.
@@ -101,7 +109,8 @@ typedef enum {
   KVQ_Q4_0 = 2,
   KVQ_TURBO3 = 3,
   KVQ_TURBO2 = 4,
-  KVQ_TURBO4 = 5
+  KVQ_TURBO4 = 5,
+  KVQ_Q5_0 = 6
 } kvq_type;
 
 typedef enum {

@@ -48,6 +48,9 @@ def oracle_rows(kind, x_f16, seed=0):
     if kind == "q4_0":
         d, qs = blocks.quantize_q4_0(x)
         return qs, d
+    if kind == "q5_0":  # scale plane row: block scales, then each qh word as two fp16 slots
+        d, qs, qh = blocks.quantize_q5_0(x)
+        return qs, np.concatenate([d, np.ascontiguousarray(qh).view(np.float16)], axis=1)
     if kind == "turbo3":
         nrm, codes = turbo3.quantize_turbo3(x, seed)
         return codes, nrm.reshape(n, 1)
@@ -65,6 +68,10 @@ def oracle_dequant(kind, codes, scales, D, seed=0):
         return blocks.dequantize_q8_0(scales, np.ascontiguousarray(codes).view(np.int8))
     if kind == "q4_0":
         return blocks.dequantize_q4_0(scales, codes)
+    if kind == "q5_0":
+        nb = D // 32
+        qh = np.ascontiguousarray(scales[:, nb:]).view(np.uint32)
+        return blocks.dequantize_q5_0(scales[:, :nb], codes, qh)
     if kind == "turbo3":
         return turbo3.dequantize_turbo3(scales[:, 0], codes, seed, D)
     if kind in ("turbo2", "turbo4"):

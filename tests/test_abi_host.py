@@ -42,7 +42,7 @@ def test_status_strings():
 
 
 def test_row_bytes_match_oracle_model():
-    for t in ("f16", "q8_0", "q4_0"):
+    for t in ("f16", "q8_0", "q4_0", "q5_0"):
         for d in (32, 64, 128, 256):
             assert kvq.kvq_row_bytes(t, d) == cache_model.row_bytes(t, d)
     for d in (32, 64, 128, 256):
@@ -65,6 +65,17 @@ def test_cache_bytes_reproduce_pages():
         v = L * kvq.kvq_cache_bytes(desc, 1, 1)
         got = {"K": k, "V": v, "KV": k + v}[which] / mib
         assert got == exp, row
+
+
+def test_q5_0_layout():
+    """q5_0: d/2 code bytes (q4_0's nibbles) and 3d/32 fp16 slots per row in the
+    scale plane (block scales, then the qh words)."""
+    desc = kvq.make_desc(32, 8, 128, "q5_0", "q5_0", 1000)
+    L = kvq.kvq_cache_layout(desc, 2, 0)
+    assert L.code_bytes == 64 and L.n_scales == 12
+    assert L.total_bytes == L.scale_offset + 2 * 8 * 1008 * 12 * 2
+    assert kvq.kvq_row_bytes("q5_0", 128) == 88 == cache_model.row_bytes("q5_0", 128)
+    assert kvq.kvq_check_desc(desc) == kvq.KVQ_OK
 
 
 def test_layout_formula():
@@ -116,7 +127,7 @@ def test_check_desc():
         (kvq.make_desc(64, 8, 128, "turbo2", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),  # value formats only
         (kvq.make_desc(64, 8, 128, "turbo4", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),
         (kvq.make_desc(64, 8, 96, "q8_0", "turbo4", 16), kvq.KVQ_ERR_UNSUPPORTED),
-        (kvq.make_desc(64, 8, 128, 6, "q4_0", 16), kvq.KVQ_ERR_INVALID),           # past the last type
+        (kvq.make_desc(64, 8, 128, 7, "q4_0", 16), kvq.KVQ_ERR_INVALID),           # past the last type
     ]
     for desc, st in bad:
         assert kvq.kvq_check_desc(desc) == st

@@ -70,14 +70,14 @@ def _check_append(k_type, v_type, D, B, H, max_ctx, pos, n_tok, seed, adversaria
 
 @pytest.mark.parametrize("k_type,v_type", [("q8_0", "q4_0"), ("q4_0", "q8_0"), ("f16", "turbo3"),
                                            ("q8_0", "turbo3"), ("f16", "f16"), ("q8_0", "turbo2"),
-                                           ("q4_0", "turbo4")])
+                                           ("q4_0", "turbo4"), ("q5_0", "q5_0"), ("q8_0", "q5_0")])
 @pytest.mark.parametrize("D", [32, 64, 128, 256])
 def test_append_bit_exact(k_type, v_type, D):
     _check_append(k_type, v_type, D, B=2, H=3, max_ctx=100, pos=37, n_tok=21, seed=D)
 
 
 @pytest.mark.parametrize("k_type,v_type", [("q8_0", "q4_0"), ("q4_0", "turbo3"), ("q8_0", "turbo2"),
-                                           ("f16", "turbo4")])
+                                           ("f16", "turbo4"), ("q5_0", "q5_0")])
 def test_append_adversarial_blocks(k_type, v_type):
     _check_append(k_type, v_type, 128, B=1, H=2, max_ctx=64, pos=0, n_tok=64, seed=3, adversarial=True)
 

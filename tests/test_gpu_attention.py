@@ -33,7 +33,7 @@ def _setup(k_type, v_type, B, n_q, n_kv, D, ctx, seed, max_ctx=None, outliers=(3
 def _oracle_out(desc, q, k, v, b, g, ctx, scale):
     """Oracle outputs [G, D] of the query heads of KV head g in batch row b."""
     G = desc.n_q_heads // desc.n_kv_heads
-    names = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4"}
+    names = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4", 6: "q5_0"}
     kt, vt = names[desc.k_type], names[desc.v_type]
     kx = k[b, :ctx, g, :].cpu().numpy()
     vx = v[b, :ctx, g, :].cpu().numpy()
@@ -63,8 +63,8 @@ def test_tiny_workload():
     _check_all(desc, q, k, v, out, w.ctx, w.scale, "tiny")
 
 
-@pytest.mark.parametrize("k_type", ["f16", "q8_0", "q4_0"])
-@pytest.mark.parametrize("v_type", ["f16", "q8_0", "q4_0", "turbo3", "turbo2", "turbo4"])
+@pytest.mark.parametrize("k_type", ["f16", "q8_0", "q4_0", "q5_0"])
+@pytest.mark.parametrize("v_type", ["f16", "q8_0", "q4_0", "turbo3", "turbo2", "turbo4", "q5_0"])
 def test_type_matrix(k_type, v_type):
     B, n_q, n_kv, D, ctx = 2, 16, 4, 128, 1000
     desc, q, k, v, kc, vc = _setup(k_type, v_type, B, n_q, n_kv, D, ctx, seed=41, max_ctx=1100)
@@ -80,6 +80,19 @@ def test_ragged_context_lengths(ctx):
     for S in (0, 1, 5):
         out = decode(desc, kc, vc, q, 1, ctx, 0.09, S)
         _check_all(desc, q, k, v, out, ctx, 0.09, f"ctx={ctx} S={S}")
+
+
+@pytest.mark.parametrize("k_type,v_type", [("q5_0", "q5_0"), ("q5_0", "q8_0"), ("q8_0", "q5_0")])
+@pytest.mark.parametrize("G", [1, 8])
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_q5_0_head_dims_and_groups(k_type, v_type, G, D):
+    """q5_0 keys and values (the fifth bit spliced into the subnormal codes)
+    at every head dim: the scale-plane rows (scales + qh words) are 12, 24 and
+    48 bytes, the last loaded row-wise."""
+    n_kv = 2
+    desc, q, k, v, kc, vc = _setup(k_type, v_type, 2, n_kv * G, n_kv, D, 300, seed=G * 7 + D)
+    out = decode(desc, kc, vc, q, 2, 300, 1 / math.sqrt(D))
+    _check_all(desc, q, k, v, out, 300, 1 / math.sqrt(D), f"{k_type}/{v_type} G={G} D={D}")
 
 
 @pytest.mark.parametrize("v_type", ["turbo2", "turbo4"])
@@ -103,8 +116,8 @@ def test_group_sizes_and_head_dims(G, D):
     _check_all(desc, q, k, v, out, 300, 1 / math.sqrt(D), f"G={G} D={D}")
 
 
-@pytest.mark.parametrize("k_type", ["f16", "q8_0", "q4_0"])
-@pytest.mark.parametrize("v_type", ["f16", "q8_0", "q4_0", "turbo3", "turbo2", "turbo4"])
+@pytest.mark.parametrize("k_type", ["f16", "q8_0", "q4_0", "q5_0"])
+@pytest.mark.parametrize("v_type", ["f16", "q8_0", "q4_0", "turbo3", "turbo2", "turbo4", "q5_0"])
 def test_type_matrix_head_dim_256(k_type, v_type):
     B, n_q, n_kv, D, ctx = 1, 8, 2, 256, 333
     desc, q, k, v, kc, vc = _setup(k_type, v_type, B, n_q, n_kv, D, ctx, seed=77)

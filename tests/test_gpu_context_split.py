@@ -17,7 +17,7 @@ from kvq_testlib import alloc_cache, assert_attention_close, decode, oracle_atte
 
 pytestmark = pytest.mark.gpu
 
-NAMES = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4"}
+NAMES = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4", 6: "q5_0"}
 
 
 def _inputs(k_type, v_type, B, n_q, n_kv, D, ctx, seed):

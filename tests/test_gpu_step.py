@@ -16,7 +16,7 @@ from kvq_testlib import (alloc_cache, assert_attention_close, decode, oracle_att
 
 pytestmark = pytest.mark.gpu
 
-NAMES = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4"}
+NAMES = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4", 6: "q5_0"}
 
 
 def _inputs(k_type, v_type, B, n_q, n_kv, D, ctx, seed, max_ctx=None, turbo_seed=None):
@@ -71,8 +71,8 @@ def _check_row_bytes(desc, kc, vc, k, v, B, row, what):
                                               err_msg=f"{what} {kind} scales b{b} g{g}")
 
 
-@pytest.mark.parametrize("k_type", ["f16", "q8_0", "q4_0"])
-@pytest.mark.parametrize("v_type", ["f16", "q8_0", "q4_0", "turbo3", "turbo2", "turbo4"])
+@pytest.mark.parametrize("k_type", ["f16", "q8_0", "q4_0", "q5_0"])
+@pytest.mark.parametrize("v_type", ["f16", "q8_0", "q4_0", "turbo3", "turbo2", "turbo4", "q5_0"])
 def test_type_matrix(k_type, v_type):
     """Rows 0 .. ctx-2 prefilled by kvq_append_quantize; the step writes row
     ctx-1 (over sentinel bytes) and attends over all ctx rows."""
