@@ -99,7 +99,9 @@ bool plane_maps(const Plane& pl, int type, int64_t planes, int64_t ctx, CUtensor
 }  // namespace
 
 bool decode_supported(int32_t k_type, int32_t v_type, int32_t G, int32_t D) {
-  if (is_turbo(k_type) || G < 1 || G > 16) return false;
+  if (G < 1 || G > 16) return false;
+  // turbo keys: with q8_0, q4_0 or the same turbo type as values
+  if (is_turbo(k_type) && v_type != KVQ_Q8_0 && v_type != KVQ_Q4_0 && v_type != k_type) return false;
   if (D != 64 && D != 128 && D != 256) return false;
   if (D == 256 && k_type == KVQ_F16 && v_type == KVQ_F16) return false;  // stage would not fit
   return true;
@@ -127,6 +129,9 @@ int decode_ctas_per_sm(int32_t k_type, int32_t v_type, int32_t D) {
     case KVQ_Q8_0: return ctas_k<KVQ_Q8_0>(v_type, D);
     case KVQ_Q4_0: return ctas_k<KVQ_Q4_0>(v_type, D);
     case KVQ_Q5_0: return ctas_k<KVQ_Q5_0>(v_type, D);
+    case KVQ_TURBO2: return ctas_k<KVQ_TURBO2>(v_type, D);
+    case KVQ_TURBO3: return ctas_k<KVQ_TURBO3>(v_type, D);
+    case KVQ_TURBO4: return ctas_k<KVQ_TURBO4>(v_type, D);
   }
   return 1;
 }
@@ -150,6 +155,9 @@ cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p,
       case KVQ_Q8_0: return tc::launch_kq8_paged(v_type, nb, nth, a, maps, st);
       case KVQ_Q4_0: return tc::launch_kq4_paged(v_type, nb, nth, a, maps, st);
       case KVQ_Q5_0: return tc::launch_kq5_paged(v_type, nb, nth, a, maps, st);
+      case KVQ_TURBO2: return tc::launch_kt2_paged(v_type, nb, nth, a, maps, st);
+      case KVQ_TURBO3: return tc::launch_kt3_paged(v_type, nb, nth, a, maps, st);
+      case KVQ_TURBO4: return tc::launch_kt4_paged(v_type, nb, nth, a, maps, st);
     }
     return cudaErrorInvalidValue;
   }
@@ -158,6 +166,9 @@ cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p,
     case KVQ_Q8_0: return tc::launch_kq8(v_type, nb, nth, a, maps, st);
     case KVQ_Q4_0: return tc::launch_kq4(v_type, nb, nth, a, maps, st);
     case KVQ_Q5_0: return tc::launch_kq5(v_type, nb, nth, a, maps, st);
+    case KVQ_TURBO2: return tc::launch_kt2(v_type, nb, nth, a, maps, st);
+    case KVQ_TURBO3: return tc::launch_kt3(v_type, nb, nth, a, maps, st);
+    case KVQ_TURBO4: return tc::launch_kt4(v_type, nb, nth, a, maps, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -86,16 +86,23 @@ __host__ __device__ constexpr int turbo_table_entries(int t) {
 }
 __host__ __device__ constexpr int round_up_c(int v, int a) { return (v + a - 1) / a * a; }
 __host__ __device__ constexpr int stage_bytes(int kt, int vt, int d) {
-  return round_up_c(kSub * code_bytes(kt, d), 1024) +
+  return round_up_c(kSub * code_bytes(kt, d), is_turbo(kt) ? 128 : 1024) +
          round_up_c(kSub * code_bytes(vt, d), is_turbo(vt) ? 128 : 1024) +
          round_up_c(kSub * n_scales(kt, d) * 2, 128) + round_up_c(kSub * n_scales(vt, d) * 2, 128);
 }
 // Shared memory of one CTA: the 1024-byte alignment pad, one ring of `stages`
 // stages per warp (rounded to the 1024-byte swizzle atom), the turbo level
-// table, the ring barriers and a few bytes of slack.
+// tables (values, then keys) and, for turbo keys, the rotated queries of up to 16
+// heads, the ring barriers and a few bytes of slack.
+// Turbo keys: one entry per level, half2(c_hi, c_lo) with c = c_hi + c_lo to
+// ~2^-22 (the scores enter an exponential, so fp16 levels alone are too coarse).
+__host__ __device__ constexpr int key_table_entries(int t) { return is_turbo(t) ? 1 << turbo_bits(t) : 0; }
+__host__ __device__ constexpr int table_bytes(int kt, int vt, int d) {
+  return (turbo_table_entries(vt) + key_table_entries(kt)) * 32 * 4 + (is_turbo(kt) ? 16 * d * 4 : 0);
+}
 __host__ __device__ constexpr int cta_smem(int kt, int vt, int d, int nw, int stages) {
-  return 1024 + nw * round_up_c(stages * stage_bytes(kt, vt, d), 1024) + turbo_table_entries(vt) * 32 * 4 +
-         nw * stages * 8 + 16;
+  return 1024 + nw * round_up_c(stages * stage_bytes(kt, vt, d), 1024) + table_bytes(kt, vt, d) + nw * stages * 8 +
+         16;
 }
 // An SM has 228 KB of shared memory and reserves 1 KB per resident CTA; the
 // kernel's static shared variables take a few bytes more.
@@ -124,13 +131,13 @@ struct Layout {
   static constexpr int kStages = stages_for(KT, VT, D);
   static constexpr int RBK = code_bytes(KT, D), RBV = code_bytes(VT, D);
   static constexpr int NSK = n_scales(KT, D), NSV = n_scales(VT, D);
-  static constexpr int KC = round_up_c(kSub * RBK, 1024);
+  static constexpr int KC = round_up_c(kSub * RBK, is_turbo(KT) ? 128 : 1024);
   static constexpr int VC = round_up_c(kSub * RBV, is_turbo(VT) ? 128 : 1024);
   static constexpr int KS = round_up_c(kSub * NSK * 2, 128);
   static constexpr int VS = round_up_c(kSub * NSV * 2, 128);
   static constexpr int STAGE = KC + VC + KS + VS;
   static constexpr int WARP = round_up_c(kStages * STAGE, 1024);
-  static constexpr int TABLE = turbo_table_entries(VT) * 32 * 4;
+  static constexpr int TABLE = table_bytes(KT, VT, D);
   static constexpr int BARS = NW * kStages * 8;
   static constexpr int TX = kSub * (RBK + 2 * NSK + RBV + 2 * NSV);  // bytes landing per tile
   // CTA-level merge scratch (reuses the stage memory after the main loop)
@@ -421,6 +428,19 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
                          : pack_half2(p.tq.levels[idx], p.tq.levels[idx]);
     }
   }
+  // turbo keys: their level table after the value table, ktable[x * 32 + lane]
+  // = half2(c_hi[x], c_lo[x]); then the rotated queries as fp16 hi and lo parts
+  uint32_t* ktable = table + turbo_table_entries(VT) * 32;
+  __half* qhi = reinterpret_cast<__half*>(ktable + key_table_entries(KT) * 32);  // [16][D]
+  __half* qlo = qhi + 16 * D;                                                        // [16][D]
+  if constexpr (is_turbo(KT)) {
+    constexpr int NE = key_table_entries(KT);
+    for (int e = threadIdx.x; e < NE * 32; e += L::NW * 32) {
+      const float cl = p.tqk.levels[e >> 5];
+      const float hi = __half2float(__float2half_rn(cl));
+      ktable[e] = pack_half2(hi, cl - hi);
+    }
+  }
   __syncthreads();
 
   auto kc_of = [&](int st) { return wbase + st * L::KC; };
@@ -451,10 +471,16 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       tplane = pg * p.n_kv + kvh;
     }
     mbar_expect_tx(&bars[st], L::TX);
-    if (L::RBK > 128)
+    if (is_turbo(KT)) {
+      if (kSub * L::RBK / 4 <= 256)
+        tma_load_2d(kc_of(st), &tm_kc, r0 * L::RBK / 4, tplane, &bars[st], pol);
+      else
+        tma_load_3d(kc_of(st), &tm_kc, 0, r0, tplane, &bars[st], pol);
+    } else if (L::RBK > 128) {
       tma_load_4d(kc_of(st), &tm_kc, 0, 0, r0, tplane, &bars[st], pol);
-    else
+    } else {
       tma_load_3d(kc_of(st), &tm_kc, 0, r0, tplane, &bars[st], pol);
+    }
     if (L::NSK) {  // flat words while a tile is at most 256 of them, else row-wise
       if (kSub * L::NSK / 2 <= 256)
         tma_load_2d(ks_of(st), &tm_ks, r0 * L::NSK / 2, tplane, &bars[st], pol);
@@ -506,6 +532,54 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     if (lane == 0 && jt < S && jt < my_tiles) issue(jt, jt, pgt);
   }
 
+  // ---- turbo keys: score = (norm/D) * <H_un (s * q), c[code]>, so each query
+  //      is rotated once: one warp per head, D/32 consecutive dims per lane,
+  //      unnormalised Walsh-Hadamard butterflies in fp32 (in registers below
+  //      stride D/32, shuffles above), stored as fp16 hi + lo parts for every
+  //      warp (the heads past G of the last n-tile as zeros).
+  if constexpr (is_turbo(KT)) {
+    constexpr int E = D / 32;
+    for (int h = p.G + warp; h < 8 * NTH; h += L::NW)
+#pragma unroll
+      for (int e = 0; e < E; ++e) qhi[h * D + lane * E + e] = qlo[h * D + lane * E + e] = __float2half_rn(0.f);
+    for (int h = warp; h < p.G; h += L::NW) {
+      const __half* qrow = p.q + ((int64_t)b * p.n_q + (int64_t)kvh * p.G + h) * D + lane * E;
+      float v[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int i = lane * E + e;
+        const float x = __half2float(qrow[e]);
+        v[e] = ((p.tqk.sign_bits[i >> 5] >> (i & 31)) & 1u) ? -x : x;
+      }
+#pragma unroll
+      for (int hs = 1; hs < E; hs <<= 1)
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          if ((e & hs) == 0) {
+            const float a0 = v[e], a1 = v[e + hs];
+            v[e] = a0 + a1;
+            v[e + hs] = a0 - a1;
+          }
+#pragma unroll
+      for (int hs = E; hs < D; hs <<= 1) {
+        const int lm = hs / E;
+        const bool upper = (lane & lm) != 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const float o = __shfl_xor_sync(0xffffffffu, v[e], lm);
+          v[e] = upper ? o - v[e] : v[e] + o;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const __half hi = __float2half_rn(v[e]);
+        qhi[h * D + lane * E + e] = hi;
+        qlo[h * D + lane * E + e] = __float2half_rn(v[e] - __half2float(hi));
+      }
+    }
+    __syncthreads();
+  }
+
   // ---- queries: B fragments of Q^T per (block, k-step) and, for quantized
   //      keys, the MMA C input -bias * sum(q) * 2^-24 of heads 2c, 2c+1 of each
   //      n-tile.  The dim order inside a block follows the A-operand loads
@@ -523,6 +597,24 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   uint32_t qb[NTH][NB][2][2];
   float cq[NTH][NB][4];
   constexpr float kBiasK = KT == KVQ_Q8_0 ? 128.f : KT == KVQ_Q4_0 ? 8.f : KT == KVQ_Q5_0 ? 16.f : 0.f;
+  if constexpr (is_turbo(KT)) {
+    // rotated queries (hi parts) in the natural dim order (k-step s of block
+    // blk covers dims 32 blk + 16 s .. +15), no code bias
+#pragma unroll
+    for (int nt = 0; nt < NTH; ++nt) {
+      const __half* qr = qhi + (nt * 8 + g) * D;
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk) {
+#pragma unroll
+        for (int s2 = 0; s2 < 2; ++s2) {
+          const int d0 = 32 * blk + 16 * s2 + 2 * c;
+          qb[nt][blk][s2][0] = *reinterpret_cast<const uint32_t*>(qr + d0);
+          qb[nt][blk][s2][1] = *reinterpret_cast<const uint32_t*>(qr + d0 + 8);
+        }
+        cq[nt][blk][0] = cq[nt][blk][1] = cq[nt][blk][2] = cq[nt][blk][3] = 0.f;
+      }
+    }
+  } else {
 #pragma unroll
   for (int nt = 0; nt < NTH; ++nt) {
 #pragma unroll
@@ -563,7 +655,8 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       cq[nt][blk][3] = c1;
     }
   }
-  const float qs = KT == KVQ_F16 ? p.qscale : p.qscale * kTwo24;
+  }
+  const float qs = (KT == KVQ_F16 || is_turbo(KT)) ? p.qscale : p.qscale * kTwo24;
 
   // ---- running state
   float m_run[NTH][2], l_run[NTH][2];
@@ -592,11 +685,66 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   int failed_at = -1;  // tile whose wait timed out (warp-uniform), -1 if none
 
   // QK of one 16-row tile: scaled scores S[row][head] of rows g, g+8 (heads 2c, 2c+1)
-  auto qk_tile = [&](uint32_t kc, const __half* ksc, float (&sc)[NTH][4]) {
+  auto qk_tile = [&](uint32_t kc, const unsigned char* kcp, const __half* ksc, float (&sc)[NTH][4]) {
 #pragma unroll
     for (int nt = 0; nt < NTH; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    if constexpr (is_turbo(KT)) {
+      // turbo keys: per 16-dim k-step one 64-bit window of each row's codes
+      // (16 b bits); the pair table gives half2(level of dim 2c, of dim 2c+1)
+      // of a row, exactly an A-operand register in the natural dim order
+      constexpr int TB = turbo_bits(KT);
+      const uint32_t* ktl = ktable + lane;
+      auto window = [&](int row, int kstep) -> unsigned long long {
+        const int byte0 = TB * kstep * 2;  // TB * 16 * kstep / 8
+        const unsigned char* rp = kcp + row * L::RBK + (byte0 & ~3);
+        unsigned long long v = *reinterpret_cast<const uint32_t*>(rp);
+        if (16 * TB + 8 * (byte0 & 3) > 32) v |= (unsigned long long)(*reinterpret_cast<const uint32_t*>(rp + 4)) << 32;
+        return v >> (8 * (byte0 & 3));
+      };
+      // dims j, j+1 of the window: (hi pair, lo pair) from two level lookups
+      auto pair = [&](unsigned long long f, int j, uint32_t& hi, uint32_t& lo) {
+        constexpr uint32_t M = (1u << TB) - 1;
+        const uint32_t e0 = ktl[((uint32_t)(f >> (TB * j)) & M) << 5];
+        const uint32_t e1 = ktl[((uint32_t)(f >> (TB * j + TB)) & M) << 5];
+        hi = prmt(e0, e1, 0x5410);
+        lo = prmt(e0, e1, 0x7632);
+      };
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk) {
+#pragma unroll
+        for (int s2 = 0; s2 < 2; ++s2) {
+          const unsigned long long fa = window(g, 2 * blk + s2), fb = window(g + 8, 2 * blk + s2);
+          uint32_t h[4], l[4];  // A operand: rows g, g+8 x dims (2c, 2c+1), (2c+8, 2c+9)
+          pair(fa, 2 * c, h[0], l[0]);
+          pair(fb, 2 * c, h[1], l[1]);
+          pair(fa, 2 * c + 8, h[2], l[2]);
+          pair(fb, 2 * c + 8, h[3], l[3]);
+          const int d0 = 32 * blk + 16 * s2 + 2 * c;
+#pragma unroll
+          for (int nt = 0; nt < NTH; ++nt) {
+            const __half* ql = qlo + (nt * 8 + g) * D + d0;
+            const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(ql);
+            const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(ql + 8);
+            // k_hi q_hi + k_hi q_lo + k_lo q_hi (k_lo q_lo is below 2^-22 relative)
+            mma16816(sc[nt], h[0], h[1], h[2], h[3], qb[nt][blk][s2][0], qb[nt][blk][s2][1], sc[nt]);
+            mma16816(sc[nt], h[0], h[1], h[2], h[3], bl0, bl1, sc[nt]);
+            mma16816(sc[nt], l[0], l[1], l[2], l[3], qb[nt][blk][s2][0], qb[nt][blk][s2][1], sc[nt]);
+          }
+        }
+      }
+      // the rows' norms / D
+      const float nA = __half2float(ksc[g]) * (1.0f / D), nB = __half2float(ksc[g + 8]) * (1.0f / D);
+#pragma unroll
+      for (int nt = 0; nt < NTH; ++nt) {
+        sc[nt][0] *= qs * nA;
+        sc[nt][1] *= qs * nA;
+        sc[nt][2] *= qs * nB;
+        sc[nt][3] *= qs * nB;
+      }
+      return;
+    }
     float dA[NB], dB[NB];  // block scales of rows g and g+8
-    if (L::NSK) {
+    if constexpr (L::NSK > 0 && !is_turbo(KT)) {
       uint32_t sa[NB / 2], sb[NB / 2];
       if (NB == 2) {
         sa[0] = *reinterpret_cast<const uint32_t*>(ksc + g * L::NSK);
@@ -943,9 +1091,9 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     const __half* vs0 = reinterpret_cast<const __half*>(vs_of(st));
 
     float sc0[NTH][4], sc1[NTH][4];
-    qk_tile(kc0, ks0, sc0);
+    qk_tile(kc0, kc_of(st), ks0, sc0);
     if (two) {
-      qk_tile(kc0 + kHalf * L::RBK, ks0 + kHalf * L::NSK, sc1);
+      qk_tile(kc0 + kHalf * L::RBK, kc_of(st) + kHalf * L::RBK, ks0 + kHalf * L::NSK, sc1);
     } else {
 #pragma unroll
       for (int nt = 0; nt < NTH; ++nt) sc1[nt][0] = sc1[nt][1] = sc1[nt][2] = sc1[nt][3] = -INFINITY;
@@ -1408,16 +1556,23 @@ cudaError_t launch_v(int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStre
 
 template <int KT, bool PAGED>
 cudaError_t launch_k(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st) {
-  switch (vt) {
-    case KVQ_F16: return launch_v<KT, KVQ_F16, PAGED>(nb, nth, a, m, st);
-    case KVQ_Q8_0: return launch_v<KT, KVQ_Q8_0, PAGED>(nb, nth, a, m, st);
-    case KVQ_Q4_0: return launch_v<KT, KVQ_Q4_0, PAGED>(nb, nth, a, m, st);
-    case KVQ_Q5_0: return launch_v<KT, KVQ_Q5_0, PAGED>(nb, nth, a, m, st);
-    case KVQ_TURBO2: return launch_v<KT, KVQ_TURBO2, PAGED>(nb, nth, a, m, st);
-    case KVQ_TURBO3: return launch_v<KT, KVQ_TURBO3, PAGED>(nb, nth, a, m, st);
-    case KVQ_TURBO4: return launch_v<KT, KVQ_TURBO4, PAGED>(nb, nth, a, m, st);
+  if constexpr (is_turbo(KT)) {  // turbo keys: q8_0, q4_0 or the same turbo type as values
+    if (vt == KVQ_Q8_0) return launch_v<KT, KVQ_Q8_0, PAGED>(nb, nth, a, m, st);
+    if (vt == KVQ_Q4_0) return launch_v<KT, KVQ_Q4_0, PAGED>(nb, nth, a, m, st);
+    if (vt == KT) return launch_v<KT, KT, PAGED>(nb, nth, a, m, st);
+    return cudaErrorInvalidValue;
+  } else {
+    switch (vt) {
+      case KVQ_F16: return launch_v<KT, KVQ_F16, PAGED>(nb, nth, a, m, st);
+      case KVQ_Q8_0: return launch_v<KT, KVQ_Q8_0, PAGED>(nb, nth, a, m, st);
+      case KVQ_Q4_0: return launch_v<KT, KVQ_Q4_0, PAGED>(nb, nth, a, m, st);
+      case KVQ_Q5_0: return launch_v<KT, KVQ_Q5_0, PAGED>(nb, nth, a, m, st);
+      case KVQ_TURBO2: return launch_v<KT, KVQ_TURBO2, PAGED>(nb, nth, a, m, st);
+      case KVQ_TURBO3: return launch_v<KT, KVQ_TURBO3, PAGED>(nb, nth, a, m, st);
+      case KVQ_TURBO4: return launch_v<KT, KVQ_TURBO4, PAGED>(nb, nth, a, m, st);
+    }
+    return cudaErrorInvalidValue;
   }
-  return cudaErrorInvalidValue;
 }
 
 // one per key type and cache kind (contiguous, paged pool), each in its own
@@ -1426,10 +1581,16 @@ cudaError_t launch_kf16(int vt, int nb, int nth, const TcArgs& a, const TcMaps& 
 cudaError_t launch_kq8(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq4(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq5(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kt2(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kt3(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kt4(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kf16_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq8_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq4_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq5_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kt2_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kt3_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kt4_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 
 }  // namespace tc
 }  // namespace kvq

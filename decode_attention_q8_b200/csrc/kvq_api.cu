@@ -349,6 +349,7 @@ kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void*
   p.ctx_lens = ctx_lens;
   p.qscale = softmax_scale * 1.4426950408889634f;
   if (is_turbo(d->v_type)) p.tq = turbo_consts(d, d->v_type);
+  if (is_turbo(d->k_type)) p.tqk = turbo_consts(d, d->k_type);
   p.append_pos = -1;
   p.out = nullptr;
   p.counters = nullptr;
@@ -492,8 +493,7 @@ kvq_status kvq_check_desc(const kvq_cache_desc* d) {
   if (d->max_ctx < 1 || d->max_ctx > kMaxCtx) return KVQ_ERR_INVALID;
   if (!known_type(d->k_type) || !known_type(d->v_type)) return KVQ_ERR_INVALID;
   if (d->head_dim % kBlock || d->head_dim > kMaxHeadDim) return KVQ_ERR_UNSUPPORTED;
-  if (is_turbo(d->k_type)) return KVQ_ERR_UNSUPPORTED;  // the turbo formats are value formats
-  if (is_turbo(d->v_type) && !pow2(d->head_dim)) return KVQ_ERR_UNSUPPORTED;
+  if ((is_turbo(d->k_type) || is_turbo(d->v_type)) && !pow2(d->head_dim)) return KVQ_ERR_UNSUPPORTED;
   if (d->n_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }

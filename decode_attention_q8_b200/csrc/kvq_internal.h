@@ -85,6 +85,7 @@ struct DecodeParams {
   int64_t n_pages;
   float qscale;        // softmax_scale * log2(e)
   TurboConsts tq;      // V sign bits and codebook (turbo values)
+  TurboConsts tqk;     // K sign bits and codebook (turbo keys)
   // Fused decode step (kvq_decode_step); a plain decode has append_pos < 0 and
   // out == null.
   int64_t append_pos;    // row the new K/V rows are written to first (< 0: none;

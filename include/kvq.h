@@ -37,7 +37,7 @@
  *              d == 0 gives q_j = 16.  22 bytes.  (A comment in the llama.cpp
  *              issue reports q5_0/q5_0 caches as a usable middle ground; no page
  *              prints its arithmetic.)
- *   KVQ_TURBO3 (values only; head_dim a power of two) one row of head_dim
+ *   KVQ_TURBO3 (head_dim a power of two) one row of head_dim
  *              elements: signs s_i = -1 when output i of splitmix64(turbo_seed)
  *              has its top bit set; v = s*x; norm = sqrtf(tree sum of v_i^2,
  *              pairs at stride d/2, d/4, ..., 1); w = unnormalised fast
@@ -48,11 +48,16 @@
  *              codes packed 3 bits each, little-endian (code i in bits
  *              3i..3i+2); stored norm fp16(min(norm, 65504)).  3d/8 + 2 bytes.
  *              Decoded value: x_hat = (norm/d) * s * H_un * c[code].
- *   KVQ_TURBO2, KVQ_TURBO4 (values only) the same row at 2 and 4 bits per value:
+ *   KVQ_TURBO2, KVQ_TURBO4 the same row at 2 and 4 bits per value:
  *              the 4- and 16-level Lloyd-Max quantizers of N(0,1) (3 and 15
  *              midpoints), code i in bits b*i .. b*i+b-1.  The TurboQuant page's
  *              FAQ ("¿Qué formato TurboQuant debería usar?") puts values at 2 to 3
  *              bits; 4 bits is the next width.  d/4 + 2 and d/2 + 2 bytes.
+ *   Turbo keys: a key row x_hat gives the score <q, x_hat> = (norm/d) *
+ *   <H_un (s * q), c[code]>, so the decode rotates each query once.  The same
+ *   page's FAQ finds keys more sensitive to compression than values.  Turbo keys
+ *   decode with q8_0, q4_0 or the same turbo type as values (other pairings are
+ *   KVQ_ERR_UNSUPPORTED at decode; append takes any pairing).
  *
  * Memory layout of one cache tensor (K or V) of one layer, in device memory
  * owned by the caller:

@@ -122,15 +122,17 @@ def test_check_desc():
         (kvq.make_desc(64, 8, 128, 9, "q4_0", 16), kvq.KVQ_ERR_INVALID),           # unknown type
         (kvq.make_desc(64, 8, 80, "q8_0", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),   # head_dim % 32
         (kvq.make_desc(64, 8, 512, "q8_0", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),  # head_dim > 256
-        (kvq.make_desc(64, 8, 128, "turbo3", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),  # turbo3 K
+        (kvq.make_desc(64, 8, 96, "turbo3", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),   # turbo K needs 2^k too
         (kvq.make_desc(64, 8, 96, "q8_0", "turbo3", 16), kvq.KVQ_ERR_UNSUPPORTED),   # WHT needs 2^k
-        (kvq.make_desc(64, 8, 128, "turbo2", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),  # value formats only
-        (kvq.make_desc(64, 8, 128, "turbo4", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),
+        (kvq.make_desc(64, 8, 96, "turbo2", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),
         (kvq.make_desc(64, 8, 96, "q8_0", "turbo4", 16), kvq.KVQ_ERR_UNSUPPORTED),
         (kvq.make_desc(64, 8, 128, 7, "q4_0", 16), kvq.KVQ_ERR_INVALID),           # past the last type
     ]
     for desc, st in bad:
         assert kvq.kvq_check_desc(desc) == st
+    # turbo keys are a valid description (the decode pairs them with q8_0, q4_0 or the same type)
+    for kt in ("turbo2", "turbo3", "turbo4"):
+        assert kvq.kvq_check_desc(kvq.make_desc(64, 8, 128, kt, "q4_0", 16)) == kvq.KVQ_OK
     d = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 16)
     d.reserved = 1
     assert kvq.kvq_check_desc(d) == kvq.KVQ_ERR_INVALID
@@ -170,7 +172,7 @@ def test_append_rejects_before_launch():
     assert _append(d, k_cache=None, k_new=None, v_cache=None, v_new=None) == kvq.KVQ_ERR_INVALID
     assert _append(d, k_cache=FAKE + 16) == kvq.KVQ_ERR_INVALID     # cache not 256-aligned
     assert _append(d, v_new=FAKE + 2) == kvq.KVQ_ERR_INVALID        # rows not 16-aligned
-    assert _append(kvq.make_desc(8, 2, 64, "turbo3", "q4_0", 256)) == kvq.KVQ_ERR_UNSUPPORTED
+    assert _append(kvq.make_desc(8, 2, 96, "turbo3", "q4_0", 256)) == kvq.KVQ_ERR_UNSUPPORTED
 
 
 def test_decode_and_combine_reject_before_launch():
@@ -188,7 +190,8 @@ def test_decode_and_combine_reject_before_launch():
     assert _combine(d, S=4, ws_bytes=need - 1) == kvq.KVQ_ERR_WORKSPACE
     assert _combine(d, out=None) == kvq.KVQ_ERR_INVALID
     assert _combine(d, ctx=0) == kvq.KVQ_ERR_INVALID
-    assert _decode(kvq.make_desc(32, 8, 128, "turbo3", "q4_0", 64)) == kvq.KVQ_ERR_UNSUPPORTED
+    assert _decode(kvq.make_desc(32, 8, 128, "turbo3", "f16", 64)) == kvq.KVQ_ERR_UNSUPPORTED   # pairing
+    assert _decode(kvq.make_desc(32, 8, 128, "turbo3", "turbo2", 64)) == kvq.KVQ_ERR_UNSUPPORTED
 
 
 def test_decode_step_rejects_before_launch():
@@ -203,7 +206,7 @@ def test_decode_step_rejects_before_launch():
     assert _step(d, k=FAKE + 16) == kvq.KVQ_ERR_INVALID
     need = kvq.kvq_workspace_bytes(d, 1, 4)
     assert _step(d, S=4, ws_bytes=need - 1) == kvq.KVQ_ERR_WORKSPACE  # the counters are part of it
-    assert _step(kvq.make_desc(32, 8, 128, "turbo3", "q4_0", 64)) == kvq.KVQ_ERR_UNSUPPORTED
+    assert _step(kvq.make_desc(32, 8, 128, "turbo3", "f16", 64)) == kvq.KVQ_ERR_UNSUPPORTED
 
 
 def _decode_varlen(desc, lens=FAKE, max_ctx=16, q=FAKE, S=0, ws=FAKE, ws_bytes=1 << 40):
@@ -246,9 +249,9 @@ def test_varlen_entry_points_reject_before_launch():
     assert _append_varlen(d, n_tok=8193) == kvq.KVQ_ERR_INVALID     # no sequence can hold them
     assert _append_varlen(d, batch=0) == kvq.KVQ_ERR_INVALID
     assert _append_varlen(d, k_new=FAKE + 8) == kvq.KVQ_ERR_INVALID
-    t3k = kvq.make_desc(32, 8, 128, "turbo3", "q4_0", 64)
+    t3k = kvq.make_desc(32, 8, 128, "turbo3", "q5_0", 64)     # a pairing the decode does not take
     assert _decode_varlen(t3k) == kvq.KVQ_ERR_UNSUPPORTED
-    assert _append_varlen(t3k) == kvq.KVQ_ERR_UNSUPPORTED
+    assert _append_varlen(kvq.make_desc(32, 8, 96, "turbo3", "q4_0", 64)) == kvq.KVQ_ERR_UNSUPPORTED
 
 
 def test_paged_layout_is_the_contiguous_layout_of_pages():

@@ -70,7 +70,8 @@ def _check_append(k_type, v_type, D, B, H, max_ctx, pos, n_tok, seed, adversaria
 
 @pytest.mark.parametrize("k_type,v_type", [("q8_0", "q4_0"), ("q4_0", "q8_0"), ("f16", "turbo3"),
                                            ("q8_0", "turbo3"), ("f16", "f16"), ("q8_0", "turbo2"),
-                                           ("q4_0", "turbo4"), ("q5_0", "q5_0"), ("q8_0", "q5_0")])
+                                           ("q4_0", "turbo4"), ("q5_0", "q5_0"), ("q8_0", "q5_0"),
+                                           ("turbo3", "turbo3"), ("turbo2", "q8_0"), ("turbo4", "turbo4")])
 @pytest.mark.parametrize("D", [32, 64, 128, 256])
 def test_append_bit_exact(k_type, v_type, D):
     _check_append(k_type, v_type, D, B=2, H=3, max_ctx=100, pos=37, n_tok=21, seed=D)

@@ -37,7 +37,7 @@ def _oracle_out(desc, q, k, v, b, g, ctx, scale):
     kt, vt = names[desc.k_type], names[desc.v_type]
     kx = k[b, :ctx, g, :].cpu().numpy()
     vx = v[b, :ctx, g, :].cpu().numpy()
-    kh = oracle_dequant(kt, *oracle_rows(kt, kx), desc.head_dim)
+    kh = oracle_dequant(kt, *oracle_rows(kt, kx, desc.turbo_seed), desc.head_dim, desc.turbo_seed)
     vh = oracle_dequant(vt, *oracle_rows(vt, vx, desc.turbo_seed), desc.head_dim, desc.turbo_seed)
     return oracle_attention_rows(q[b, g * G:(g + 1) * G].cpu().numpy(), kh, vh, scale)
 
@@ -80,6 +80,20 @@ def test_ragged_context_lengths(ctx):
     for S in (0, 1, 5):
         out = decode(desc, kc, vc, q, 1, ctx, 0.09, S)
         _check_all(desc, q, k, v, out, ctx, 0.09, f"ctx={ctx} S={S}")
+
+
+@pytest.mark.parametrize("k_type,v_type", [("turbo3", "turbo3"), ("turbo2", "turbo2"), ("turbo4", "turbo4"),
+                                           ("turbo3", "q8_0"), ("turbo2", "q4_0")])
+@pytest.mark.parametrize("G", [1, 8, 16])
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_turbo_keys(k_type, v_type, G, D):
+    """Turbo keys: each query is rotated once in the kernel (H_un (s * q)) and
+    scored against the level table, scaled by norm / D per row."""
+    n_kv = 2
+    desc, q, k, v, kc, vc = _setup(k_type, v_type, 2, n_kv * G, n_kv, D, 400, seed=G * 3 + D + 5)
+    for S in (0, 3):
+        out = decode(desc, kc, vc, q, 2, 400, 1 / math.sqrt(D), S)
+        _check_all(desc, q, k, v, out, 400, 1 / math.sqrt(D), f"{k_type}/{v_type} G={G} D={D} S={S}")
 
 
 @pytest.mark.parametrize("k_type,v_type", [("q5_0", "q5_0"), ("q5_0", "q8_0"), ("q8_0", "q5_0")])

@@ -51,7 +51,8 @@ def _rank_partials(desc, q, k, v, B, bounds, S, scale, lens=None):
 def _oracle(desc, q, k, v, b, g, n, scale):
     G = desc.n_q_heads // desc.n_kv_heads
     kt, vt = NAMES[desc.k_type], NAMES[desc.v_type]
-    kh = oracle_dequant(kt, *oracle_rows(kt, k[b, :n, g].cpu().numpy()), desc.head_dim)
+    kh = oracle_dequant(kt, *oracle_rows(kt, k[b, :n, g].cpu().numpy(), desc.turbo_seed), desc.head_dim,
+                        desc.turbo_seed)
     vh = oracle_dequant(vt, *oracle_rows(vt, v[b, :n, g].cpu().numpy(), desc.turbo_seed), desc.head_dim,
                         desc.turbo_seed)
     return oracle_attention_rows(q[b, g * G:(g + 1) * G].cpu().numpy(), kh, vh, scale)

@@ -44,7 +44,8 @@ def _step(desc, kc, vc, q, k, v, B, ctx, scale, S, ws):
 def _oracle(desc, q, k, v, b, g, ctx, scale):
     G = desc.n_q_heads // desc.n_kv_heads
     kt, vt = NAMES[desc.k_type], NAMES[desc.v_type]
-    kh = oracle_dequant(kt, *oracle_rows(kt, k[b, :ctx, g, :].cpu().numpy()), desc.head_dim)
+    kh = oracle_dequant(kt, *oracle_rows(kt, k[b, :ctx, g, :].cpu().numpy(), desc.turbo_seed), desc.head_dim,
+                        desc.turbo_seed)
     vh = oracle_dequant(vt, *oracle_rows(vt, v[b, :ctx, g, :].cpu().numpy(), desc.turbo_seed), desc.head_dim,
                         desc.turbo_seed)
     return oracle_attention_rows(q[b, g * G:(g + 1) * G].cpu().numpy(), kh, vh, scale)
@@ -71,8 +72,14 @@ def _check_row_bytes(desc, kc, vc, k, v, B, row, what):
                                               err_msg=f"{what} {kind} scales b{b} g{g}")
 
 
-@pytest.mark.parametrize("k_type", ["f16", "q8_0", "q4_0", "q5_0"])
-@pytest.mark.parametrize("v_type", ["f16", "q8_0", "q4_0", "turbo3", "turbo2", "turbo4", "q5_0"])
+def _pairs():
+    plain = [(k, v) for k in ("f16", "q8_0", "q4_0", "q5_0")
+             for v in ("f16", "q8_0", "q4_0", "turbo3", "turbo2", "turbo4", "q5_0")]
+    turbo_keys = [(k, v) for k in ("turbo2", "turbo3", "turbo4") for v in ("q8_0", "q4_0", k)]
+    return plain + turbo_keys
+
+
+@pytest.mark.parametrize("k_type,v_type", _pairs())
 def test_type_matrix(k_type, v_type):
     """Rows 0 .. ctx-2 prefilled by kvq_append_quantize; the step writes row
     ctx-1 (over sentinel bytes) and attends over all ctx rows."""

@@ -32,7 +32,8 @@ def _oracle(desc, q, k, v, b, g, n):
     """Oracle output of group (b, g) over rows 0 .. n-1 of the fp16 inputs k, v."""
     G = desc.n_q_heads // desc.n_kv_heads
     kt, vt = NAMES[desc.k_type], NAMES[desc.v_type]
-    kh = oracle_dequant(kt, *oracle_rows(kt, k[b, :n, g, :].cpu().numpy()), desc.head_dim)
+    kh = oracle_dequant(kt, *oracle_rows(kt, k[b, :n, g, :].cpu().numpy(), desc.turbo_seed), desc.head_dim,
+                        desc.turbo_seed)
     vh = oracle_dequant(vt, *oracle_rows(vt, v[b, :n, g, :].cpu().numpy(), desc.turbo_seed), desc.head_dim,
                         desc.turbo_seed)
     return oracle_attention_rows(q[b, g * G:(g + 1) * G].cpu().numpy(), kh, vh, 1 / math.sqrt(desc.head_dim))
