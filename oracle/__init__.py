@@ -18,6 +18,8 @@ Modules:
   turbo3      seeded sign vector (splitmix64), Sylvester Hadamard, fast
               Walsh-Hadamard transform, Lloyd-Max codebook, turbo3 rows
   turbo       the same rows at 2 and 4 bits per value (turbo2, turbo4)
+  qjl         turbo3_qjl key rows: the 2-bit row plus 1-bit QJL signs of its
+              residual and the residual's norm
   attention   decode attention (plain softmax definition), split partials
               and their combine
   cache_model bytes per cache row / per cache, the nominal-size model
@@ -31,10 +33,14 @@ Pins (what each function is checked against, in ``tests/test_oracle_*.py``):
   turbo       2-level closed form +-sqrt(2/pi), Max (1960) 4- and 16-level
               tables, hand-packed 2- and 4-bit bytes, the turbo3 oracle at 3
               bits, round-trip error = the quantizer's distortion
+  qjl         unbiased inner products over the projection's draw and the QJL
+              variance bound, residual norm and signs formed in the original
+              domain, the turbo2 row as its 2-bit stage, no residual = turbo2,
+              hand-packed bytes
   attention   brute-force full-matrix softmax(Q K^T) V, closed forms
               (ctx=1, identical keys, q=0), rows summing to 1, split/combine
               identity
 No oracle function is left unpinned.
 """
 
-from . import blocks, turbo3, attention, cache_model  # noqa: F401
+from . import blocks, turbo3, turbo, qjl, attention, cache_model  # noqa: F401

@@ -5,7 +5,8 @@ Test infrastructure only (see ``oracle/__init__.py``).
 Per 32 elements: f16 64 bytes, q8_0 34 bytes (fp16 scale + 32 int8),
 q4_0 18 bytes (fp16 scale + 16 bytes of nibbles), q5_0 22 bytes (fp16 scale, 16 bytes of
 nibbles, a 32-bit word of fifth bits).  turbo2 / turbo3 / turbo4
-per row of d elements: 2d/8, 3d/8, 4d/8 bytes of codes + an fp16 norm.  Nominal costs are on
+per row of d elements: 2d/8, 3d/8, 4d/8 bytes of codes + an fp16 norm; turbo3_qjl
+3d/8 bytes of codes (2-bit levels, 1-bit residual signs) + two fp16 norms.  Nominal costs are on
 ``llama.cpp für Geschwindigkeit und Speicher optimieren``, section
 "KV-Cache-Präzision" (2 / 1 / 0.5 bytes per element); the exact block sizes
 are pinned by the cache sizes the KVSplit page and the llama.cpp issue print
@@ -19,6 +20,8 @@ def row_bytes(kind, d):
     """Bytes one cached row of d elements takes."""
     if kind in ("turbo2", "turbo3", "turbo4"):
         return int(kind[-1]) * d // 8 + 2
+    if kind == "turbo3_qjl":
+        return 3 * d // 8 + 4
     if d % 32:
         raise ValueError("head_dim must be a multiple of 32")
     return BYTES_PER_32[kind] * d // 32

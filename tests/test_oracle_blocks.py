@@ -225,3 +225,12 @@ def test_row_bytes_nominal():
     assert cache_model.row_bytes("q8_0", 128) == 136
     assert cache_model.row_bytes("q4_0", 128) == 72
     assert cache_model.row_bytes("turbo3", 128) * 8 / 128 == 3.125
+
+
+def test_turbo3_qjl_row_bytes():
+    """3 bits of codes per value (2-bit levels + 1-bit residual signs, as the
+    TurboQuant page's "3 bits per value"), plus two fp16 norms: 52 bytes at
+    d = 128, a 4.9x reduction from fp16 (the page: about 5x)."""
+    assert cache_model.row_bytes("turbo3_qjl", 128) == 52
+    assert cache_model.row_bytes("turbo3_qjl", 64) == 28
+    assert abs(cache_model.row_bytes("f16", 128) / cache_model.row_bytes("turbo3_qjl", 128) - 5) < 0.1
