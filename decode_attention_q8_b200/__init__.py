@@ -24,9 +24,9 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-KVQ_F16, KVQ_Q8_0, KVQ_Q4_0, KVQ_TURBO3, KVQ_TURBO2, KVQ_TURBO4, KVQ_Q5_0 = 0, 1, 2, 3, 4, 5, 6
+KVQ_F16, KVQ_Q8_0, KVQ_Q4_0, KVQ_TURBO3, KVQ_TURBO2, KVQ_TURBO4, KVQ_Q5_0, KVQ_TURBO3_QJL = 0, 1, 2, 3, 4, 5, 6, 7
 TYPES = {"f16": KVQ_F16, "q8_0": KVQ_Q8_0, "q4_0": KVQ_Q4_0, "turbo3": KVQ_TURBO3, "turbo2": KVQ_TURBO2,
-         "turbo4": KVQ_TURBO4, "q5_0": KVQ_Q5_0}
+         "turbo4": KVQ_TURBO4, "q5_0": KVQ_Q5_0, "turbo3_qjl": KVQ_TURBO3_QJL}
 
 KVQ_OK, KVQ_ERR_INVALID, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA = 0, 1, 2, 3, 4
 
@@ -51,6 +51,7 @@ class kvq_cache_desc(ctypes.Structure):
         ("reserved", ctypes.c_int32),
         ("max_ctx", ctypes.c_int64),
         ("turbo_seed", ctypes.c_uint64),
+        ("qjl_proj", ctypes.c_void_p),
     ]
 
 
@@ -158,9 +159,13 @@ def _type(t):
     return TYPES[t] if isinstance(t, str) else int(t)
 
 
-def make_desc(n_q_heads, n_kv_heads, head_dim, k_type, v_type, max_ctx, turbo_seed=0):
-    return kvq_cache_desc(n_q_heads, n_kv_heads, head_dim, _type(k_type), _type(v_type), 0,
-                          max_ctx, turbo_seed)
+def make_desc(n_q_heads, n_kv_heads, head_dim, k_type, v_type, max_ctx, turbo_seed=0, qjl_proj=None):
+    """A kvq_cache_desc.  qjl_proj: the turbo3_qjl projection (device fp32
+    [head_dim][head_dim]); the descriptor keeps a reference to it."""
+    d = kvq_cache_desc(n_q_heads, n_kv_heads, head_dim, _type(k_type), _type(v_type), 0,
+                       max_ctx, turbo_seed, _ptr(qjl_proj))
+    d.qjl_tensor = qjl_proj
+    return d
 
 
 # ----------------------------------------------------------------- queries
@@ -203,12 +208,13 @@ def kvq_turbo3_codebook():
 
 
 def kvq_turbo_codebook(type_):
-    """(levels[2^b], thresholds[2^b - 1]) of a turbo type ("turbo2", "turbo3", "turbo4")."""
+    """(levels[2^b], thresholds[2^b - 1]) of a turbo type ("turbo2", "turbo3", "turbo4";
+    "turbo3_qjl": the 4-level codebook of its 2-bit codes)."""
     t = _type(type_)
     lv = (ctypes.c_float * 16)()
     th = (ctypes.c_float * 15)()
     _check(_lib.kvq_turbo_codebook(t, lv, th), "kvq_turbo_codebook")
-    n = {KVQ_TURBO2: 4, KVQ_TURBO3: 8, KVQ_TURBO4: 16}[t]
+    n = {KVQ_TURBO2: 4, KVQ_TURBO3: 8, KVQ_TURBO4: 16, KVQ_TURBO3_QJL: 4}[t]
     return list(lv)[:n], list(th)[:n - 1]
 
 

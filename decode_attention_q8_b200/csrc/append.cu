@@ -1,5 +1,5 @@
-// Quantize-on-append kernel: fp16 K/V rows -> f16 / q8_0 / q4_0 / turbo3 cache
-// rows, K and V of one call in one launch.  The row bodies (formats, rounding,
+// Quantize-on-append kernel: fp16 K/V rows -> f16 / q8_0 / q4_0 / q5_0 / turbo
+// cache rows, K and V of one call in one launch.  The row bodies (formats, rounding,
 // work mapping) are in append_rows.cuh.
 #include <algorithm>
 
@@ -78,6 +78,9 @@ __device__ __forceinline__ void append_turbo_part(const AppendParams& p, int64_t
   }
 }
 
+// QJL: the instance that also takes turbo3_qjl rows (their projection loop
+// needs far more registers; the other types keep the lean instance).
+template <bool QJL>
 __device__ __forceinline__ void append_part(const AppendParams& p, int32_t type, int64_t first, int64_t stride) {
   const int64_t gend = (int64_t)p.B * p.n_tok * p.H * bulk_items(type, p.D);
   switch (type) {
@@ -88,22 +91,28 @@ __device__ __forceinline__ void append_part(const AppendParams& p, int32_t type,
     case KVQ_TURBO2: append_turbo_part<KVQ_TURBO2>(p, first, stride, gend); break;
     case KVQ_TURBO3: append_turbo_part<KVQ_TURBO3>(p, first, stride, gend); break;
     case KVQ_TURBO4: append_turbo_part<KVQ_TURBO4>(p, first, stride, gend); break;
+    case KVQ_TURBO3_QJL:
+      if constexpr (QJL) append_turbo_part<KVQ_TURBO3_QJL>(p, first, stride, gend);
+      break;
   }
 }
 
+template <bool QJL>
 __global__ void __launch_bounds__(kAppendThreads) append_pair_kernel(const AppendPair pp) {
   const int64_t first = (int64_t)blockIdx.x * kAppendThreads + threadIdx.x;
   const int64_t stride = (int64_t)gridDim.x * kAppendThreads;
-  append_part(pp.p[0], pp.type[0], first, stride);
-  if (pp.n == 2) append_part(pp.p[1], pp.type[1], first, stride);
+  append_part<QJL>(pp.p[0], pp.type[0], first, stride);
+  if (pp.n == 2) append_part<QJL>(pp.p[1], pp.type[1], first, stride);
 }
 
 // Resident 256-thread CTAs of the append kernel on the whole current device
 // (one wave); 148 SMs x 4 if the device cannot be asked.
+template <bool QJL>
 int64_t resident_ctas() {
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, append_pair_kernel, kAppendThreads, 0) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, append_pair_kernel<QJL>, kAppendThreads, 0) !=
+          cudaSuccess ||
       sms <= 0 || per_sm <= 0) {
     (void)cudaGetLastError();
     return 148 * 4;
@@ -135,9 +144,13 @@ cudaError_t launch_append(const AppendParams* k, int32_t k_type, const AppendPar
   pp.n = n;
   int64_t need = append_ctas(pp.type[0], pp.p[0]);
   if (n == 2) need = std::max(need, append_ctas(pp.type[1], pp.p[1]));
-  const int64_t ctas = std::min(need, resident_ctas());
+  const bool qjl = is_qjl(pp.type[0]) || (n == 2 && is_qjl(pp.type[1]));
+  const int64_t ctas = std::min(need, qjl ? resident_ctas<true>() : resident_ctas<false>());
   if (ctas <= 0) return cudaSuccess;  // no rows
-  append_pair_kernel<<<(unsigned)ctas, kAppendThreads, 0, st>>>(pp);
+  if (qjl)
+    append_pair_kernel<true><<<(unsigned)ctas, kAppendThreads, 0, st>>>(pp);
+  else
+    append_pair_kernel<false><<<(unsigned)ctas, kAppendThreads, 0, st>>>(pp);
   return cudaGetLastError();
 }
 

@@ -1,5 +1,5 @@
-// Quantize-on-append row bodies: fp16 K/V rows -> f16 / q8_0 / q4_0 / turbo3
-// cache rows.  Used by the append kernel and by the fused decode step.
+// Quantize-on-append row bodies: fp16 K/V rows -> f16 / q8_0 / q4_0 / q5_0 /
+// turbo cache rows.  Used by the append kernel and by the fused decode step.
 //
 // The cache types are those of "llama.cpp für Geschwindigkeit und Speicher
 // optimieren" (section "KV-Cache-Präzision") and, for turbo3, of "Benchmark
@@ -413,8 +413,11 @@ __device__ __forceinline__ void append_f16(const AppendParams& p, int64_t gtid, 
 }
 
 // turbo (BITS = 2, 3 or 4 bits per value): one warp per row, E = D/32
-// contiguous elements per lane.
-template <int BITS, int E>
+// contiguous elements per lane.  QJL (turbo3_qjl, BITS = 2): after the level
+// codes, the residual e = g - c[code] of each element, its norm by the same
+// tree, and the sign bits of u = P e; lane l computes u_i of its own rows
+// i = l*E .. l*E+E-1, taking e_j (j = 0 .. D-1 in order) from its owner lane.
+template <int BITS, int E, bool QJL = false>
 __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
   constexpr int D = 32 * E;
   const int64_t row = gtid >> 5;
@@ -466,13 +469,73 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
   }
   const float r = norm > 0.0f ? __frcp_rn(norm) : 0.0f;
   uint32_t bits = 0;
+  float res[E];  // QJL: residuals in the rotated unit domain
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const float g = __fmul_rn(v[e], r);
     int c = 0;
+    float lv = p.tq.levels[0];  // levels[c] (thresholds ascend), without a dynamic index
 #pragma unroll
-    for (int k = 0; k < (1 << BITS) - 1; ++k) c += (g > p.tq.tau[k]) ? 1 : 0;
+    for (int k = 0; k < (1 << BITS) - 1; ++k) {
+      const bool up = g > p.tq.tau[k];
+      c += up ? 1 : 0;
+      if (QJL) lv = up ? p.tq.levels[k + 1] : lv;
+    }
     bits |= (uint32_t)c << (BITS * e);
+    res[e] = QJL ? __fsub_rn(g, lv) : 0.0f;
+  }
+  float gamma = 0.0f;
+  uint32_t zbits = 0;
+  if constexpr (QJL) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) a[e] = __fmul_rn(res[e], res[e]);
+#pragma unroll
+    for (int h = D / 2; h >= E; h >>= 1) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) a[e] = __fadd_rn(a[e], __shfl_xor_sync(0xffffffffu, a[e], h / E));
+    }
+#pragma unroll
+    for (int h = E / 2; h >= 1; h >>= 1) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) a[e] = __fadd_rn(a[e], a[e + h]);
+    }
+    const float eps = __fsqrt_rn(__shfl_sync(0xffffffffu, a[0], 0));
+    gamma = __fmul_rn(__fmul_rn(norm, eps), p.tq.rsqrt_d);
+    float u[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) u[e] = 0.0f;
+    const float* prow = p.tq.proj + (size_t)(lane * E) * D;  // row lane*E of P
+#pragma unroll 4
+    for (int jl = 0; jl < 32; ++jl) {  // e_j of j = jl*E .. jl*E+E-1, held by lane jl
+      float ej[E];
+#pragma unroll
+      for (int e2 = 0; e2 < E; ++e2) ej[e2] = __shfl_sync(0xffffffffu, res[e2], jl);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        float pv[E];
+        const float* src = prow + (size_t)e * D + jl * E;
+        if constexpr (E % 4 == 0) {
+#pragma unroll
+          for (int k4 = 0; k4 < E; k4 += 4) {
+            const float4 f = __ldg(reinterpret_cast<const float4*>(src + k4));
+            pv[k4] = f.x;
+            pv[k4 + 1] = f.y;
+            pv[k4 + 2] = f.z;
+            pv[k4 + 3] = f.w;
+          }
+        } else if constexpr (E == 2) {
+          const float2 f = __ldg(reinterpret_cast<const float2*>(src));
+          pv[0] = f.x;
+          pv[1] = f.y;
+        } else {
+          pv[0] = __ldg(src);
+        }
+#pragma unroll
+        for (int e2 = 0; e2 < E; ++e2) u[e] = __fadd_rn(u[e], __fmul_rn(pv[e2], ej[e2]));
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) zbits |= (u[e] < 0.0f ? 1u : 0u) << e;
   }
   // The lane's LB = BITS*E bits start at bit LB*lane of the row; a group of L
   // lanes (the fewest whose bits make whole bytes, at most 32) is stored by
@@ -485,6 +548,16 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
     const uint32_t o = __shfl_down_sync(0xffffffffu, bits, j);
     word |= o << (LB * j);
   }
+  // QJL sign bits: E per lane, the same grouping at one bit per value
+  constexpr int LZ = E % 8 == 0 ? 1 : E % 4 == 0 ? 2 : E % 2 == 0 ? 4 : 8;
+  uint32_t zword = zbits;
+  if constexpr (QJL) {
+#pragma unroll
+    for (int j = 1; j < LZ; ++j) {
+      const uint32_t o = __shfl_down_sync(0xffffffffu, zbits, j);
+      zword |= o << (E * j);
+    }
+  }
   const int64_t r_dst = dst_row(p, row);
   if (r_dst < 0) return;  // after the last shuffle
   uint8_t* codes = p.dst.codes + r_dst * p.dst.code_bytes;
@@ -493,7 +566,19 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
 #pragma unroll
     for (int i = 0; i < L * LB / 8; ++i) codes[byte0 + i] = (uint8_t)((word >> (8 * i)) & 0xFF);
   }
-  if (lane == 0) p.dst.scales[r_dst] = __float2half_rn(fminf(norm, 65504.0f));
+  if constexpr (QJL) {
+    if ((lane % LZ) == 0) {
+      const int byte0 = BITS * D / 8 + E * lane / 8;
+#pragma unroll
+      for (int i = 0; i < LZ * E / 8; ++i) codes[byte0 + i] = (uint8_t)((zword >> (8 * i)) & 0xFF);
+    }
+    if (lane == 0) {
+      p.dst.scales[2 * r_dst] = __float2half_rn(fminf(norm, 65504.0f));
+      p.dst.scales[2 * r_dst + 1] = __float2half_rn(fminf(gamma, 65504.0f));
+    }
+  } else {
+    if (lane == 0) p.dst.scales[r_dst] = __float2half_rn(fminf(norm, 65504.0f));
+  }
 }
 
 // Quantize and store work item gtid from its loaded bytes (every lane of the
@@ -504,7 +589,7 @@ __device__ __forceinline__ void finish(const AppendParams& p, int64_t gtid, int6
   else if constexpr (TYPE == KVQ_Q4_0) append_q4_0(p, gtid, gend, raw);
   else if constexpr (TYPE == KVQ_Q5_0) append_q5_0(p, gtid, gend, raw);
   else if constexpr (TYPE == KVQ_F16) append_f16(p, gtid, gend, raw);
-  else append_turbo<turbo_bits(TYPE), E>(p, gtid, gend, raw);
+  else append_turbo<turbo_bits(TYPE), E, is_qjl(TYPE)>(p, gtid, gend, raw);
 }
 
 template <int TYPE, int E>
@@ -533,6 +618,7 @@ __device__ __forceinline__ void append_any(int32_t type, const AppendParams& p, 
     case KVQ_TURBO2: append_turbo_any<KVQ_TURBO2>(p, gtid, gend); break;
     case KVQ_TURBO3: append_turbo_any<KVQ_TURBO3>(p, gtid, gend); break;
     case KVQ_TURBO4: append_turbo_any<KVQ_TURBO4>(p, gtid, gend); break;
+    case KVQ_TURBO3_QJL: append_turbo_any<KVQ_TURBO3_QJL>(p, gtid, gend); break;
   }
 }
 

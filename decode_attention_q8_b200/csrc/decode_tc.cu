@@ -4,7 +4,7 @@
 // Code planes of f16 / q8_0 / q4_0 caches are described row by row
 // ([planes][rows][row bytes], bytes as uint8) with the hardware swizzle whose
 // span equals the row (32, 64 or 128 bytes; wider rows split into 128-byte
-// segments).  turbo3 code planes and all scale planes are described as flat
+// segments).  turbo code planes and all scale planes are described as flat
 // uint32 arrays per plane.  The row extent is ctx_len, so a 16-row tile that
 // runs past the context reads zeros there.
 #include <cudaTypedefs.h>
@@ -100,8 +100,11 @@ bool plane_maps(const Plane& pl, int type, int64_t planes, int64_t ctx, CUtensor
 
 bool decode_supported(int32_t k_type, int32_t v_type, int32_t G, int32_t D) {
   if (G < 1 || G > 16) return false;
-  // turbo keys: with q8_0, q4_0 or the same turbo type as values
-  if (is_turbo(k_type) && v_type != KVQ_Q8_0 && v_type != KVQ_Q4_0 && v_type != k_type) return false;
+  // turbo3_qjl keys: with q8_0, q4_0 or turbo3 values; other turbo keys: with
+  // q8_0, q4_0 or the same turbo type as values
+  if (is_qjl(k_type) && v_type != KVQ_Q8_0 && v_type != KVQ_Q4_0 && v_type != KVQ_TURBO3) return false;
+  if (is_turbo(k_type) && !is_qjl(k_type) && v_type != KVQ_Q8_0 && v_type != KVQ_Q4_0 && v_type != k_type)
+    return false;
   if (D != 64 && D != 128 && D != 256) return false;
   if (D == 256 && k_type == KVQ_F16 && v_type == KVQ_F16) return false;  // stage would not fit
   return true;
@@ -132,6 +135,7 @@ int decode_ctas_per_sm(int32_t k_type, int32_t v_type, int32_t D) {
     case KVQ_TURBO2: return ctas_k<KVQ_TURBO2>(v_type, D);
     case KVQ_TURBO3: return ctas_k<KVQ_TURBO3>(v_type, D);
     case KVQ_TURBO4: return ctas_k<KVQ_TURBO4>(v_type, D);
+    case KVQ_TURBO3_QJL: return ctas_k<KVQ_TURBO3_QJL>(v_type, D);
   }
   return 1;
 }
@@ -158,6 +162,7 @@ cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p,
       case KVQ_TURBO2: return tc::launch_kt2_paged(v_type, nb, nth, a, maps, st);
       case KVQ_TURBO3: return tc::launch_kt3_paged(v_type, nb, nth, a, maps, st);
       case KVQ_TURBO4: return tc::launch_kt4_paged(v_type, nb, nth, a, maps, st);
+      case KVQ_TURBO3_QJL: return tc::launch_kqjl_paged(v_type, nb, nth, a, maps, st);
     }
     return cudaErrorInvalidValue;
   }
@@ -169,6 +174,7 @@ cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p,
     case KVQ_TURBO2: return tc::launch_kt2(v_type, nb, nth, a, maps, st);
     case KVQ_TURBO3: return tc::launch_kt3(v_type, nb, nth, a, maps, st);
     case KVQ_TURBO4: return tc::launch_kt4(v_type, nb, nth, a, maps, st);
+    case KVQ_TURBO3_QJL: return tc::launch_kqjl(v_type, nb, nth, a, maps, st);
   }
   return cudaErrorInvalidValue;
 }

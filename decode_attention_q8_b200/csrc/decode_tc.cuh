@@ -70,10 +70,14 @@ constexpr int kHalf = 16;    // rows per MMA row block (two per tile)
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 __host__ __device__ constexpr int code_bytes(int t, int d) {
-  return t == KVQ_F16 ? 2 * d : t == KVQ_Q8_0 ? d : (t == KVQ_Q4_0 || t == KVQ_Q5_0) ? d / 2 : turbo_bits(t) * d / 8;
+  return t == KVQ_F16 ? 2 * d
+         : t == KVQ_Q8_0 ? d
+         : (t == KVQ_Q4_0 || t == KVQ_Q5_0) ? d / 2
+         : is_qjl(t) ? 3 * d / 8
+                     : turbo_bits(t) * d / 8;
 }
 __host__ __device__ constexpr int n_scales(int t, int d) {
-  return t == KVQ_F16 ? 0 : is_turbo(t) ? 1 : t == KVQ_Q5_0 ? 3 * d / 32 : d / 32;
+  return t == KVQ_F16 ? 0 : is_qjl(t) ? 2 : is_turbo(t) ? 1 : t == KVQ_Q5_0 ? 3 * d / 32 : d / 32;
 }
 // swizzle of a code plane: 16-byte chunk index XOR ((offset >> 7) & mask)
 __host__ __device__ constexpr int swz_mask(int t, int d) {
@@ -97,8 +101,13 @@ __host__ __device__ constexpr int stage_bytes(int kt, int vt, int d) {
 // Turbo keys: one entry per level, half2(c_hi, c_lo) with c = c_hi + c_lo to
 // ~2^-22 (the scores enter an exponential, so fp16 levels alone are too coarse).
 __host__ __device__ constexpr int key_table_entries(int t) { return is_turbo(t) ? 1 << turbo_bits(t) : 0; }
+// turbo3_qjl keys: the projected queries P q_rot of up to 16 heads as fp16 hi
+// and lo parts, rows padded to d + 8 halves (the MMA B-fragment reads of the 8
+// heads of an n-tile then fall in distinct banks).
+__host__ __device__ constexpr int qjl_stride(int d) { return d + 8; }
 __host__ __device__ constexpr int table_bytes(int kt, int vt, int d) {
-  return (turbo_table_entries(vt) + key_table_entries(kt)) * 32 * 4 + (is_turbo(kt) ? 16 * d * 4 : 0);
+  return (turbo_table_entries(vt) + key_table_entries(kt)) * 32 * 4 + (is_turbo(kt) ? 16 * d * 4 : 0) +
+         (is_qjl(kt) ? 16 * qjl_stride(d) * 4 : 0);
 }
 __host__ __device__ constexpr int cta_smem(int kt, int vt, int d, int nw, int stages) {
   return 1024 + nw * round_up_c(stages * stage_bytes(kt, vt, d), 1024) + table_bytes(kt, vt, d) + nw * stages * 8 +
@@ -137,6 +146,17 @@ struct Layout {
   static constexpr int VS = round_up_c(kSub * NSV * 2, 128);
   static constexpr int STAGE = KC + VC + KS + VS;
   static constexpr int WARP = round_up_c(kStages * STAGE, 1024);
+  // Stage rings of a warp: code tiles, then scale tiles.  A swizzled code tile
+  // starts on its swizzle atom (128 bytes per 16-byte chunk the pattern
+  // permutes), so with turbo keys and swizzled values the value tiles go first.
+  static constexpr bool VFIRST = is_turbo(KT) && !is_turbo(VT);
+  static constexpr int KOFF = VFIRST ? kStages * VC : 0;
+  static constexpr int VOFF = VFIRST ? 0 : kStages * KC;
+  static constexpr int SOFF = kStages * (KC + VC);
+  static_assert(KOFF % (128 * (swz_mask(KT, D) + 1)) == 0 && KC % (128 * (swz_mask(KT, D) + 1)) == 0,
+                "key code tiles on their swizzle atom");
+  static_assert(VOFF % (128 * (swz_mask(VT, D) + 1)) == 0 && VC % (128 * (swz_mask(VT, D) + 1)) == 0,
+                "value code tiles on their swizzle atom");
   static constexpr int TABLE = table_bytes(KT, VT, D);
   static constexpr int BARS = NW * kStages * 8;
   static constexpr int TX = kSub * (RBK + 2 * NSK + RBV + 2 * NSV);  // bytes landing per tile
@@ -433,6 +453,9 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   uint32_t* ktable = table + turbo_table_entries(VT) * 32;
   __half* qhi = reinterpret_cast<__half*>(ktable + key_table_entries(KT) * 32);  // [16][D]
   __half* qlo = qhi + 16 * D;                                                        // [16][D]
+  constexpr int PST = qjl_stride(D);
+  __half* phi = qlo + 16 * D;    // turbo3_qjl: P q_rot, [16][PST]
+  __half* plo = phi + 16 * PST;  // [16][PST]
   if constexpr (is_turbo(KT)) {
     constexpr int NE = key_table_entries(KT);
     for (int e = threadIdx.x; e < NE * 32; e += L::NW * 32) {
@@ -443,10 +466,10 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   }
   __syncthreads();
 
-  auto kc_of = [&](int st) { return wbase + st * L::KC; };
-  auto vc_of = [&](int st) { return wbase + S * L::KC + st * L::VC; };
-  auto ks_of = [&](int st) { return wbase + S * (L::KC + L::VC) + st * L::KS; };
-  auto vs_of = [&](int st) { return wbase + S * (L::KC + L::VC + L::KS) + st * L::VS; };
+  auto kc_of = [&](int st) { return wbase + L::KOFF + st * L::KC; };
+  auto vc_of = [&](int st) { return wbase + L::VOFF + st * L::VC; };
+  auto ks_of = [&](int st) { return wbase + L::SOFF + st * L::KS; };
+  auto vs_of = [&](int st) { return wbase + L::SOFF + S * L::KS + st * L::VS; };
 
   // tile j of this warp covers rows t0 + 32*(warp + NW*j) ... (logical rows of
   // the sequence; in a paged pool, page pg's rows from r0 mod the page size)
@@ -578,6 +601,39 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       }
     }
     __syncthreads();
+    // turbo3_qjl: the sign bits z of a key row give <q, x_hat> its second term
+    // sqrt(pi/2) / D^1.5 * gamma * <P q_rot, 1 - 2z>, so each rotated query is
+    // projected once: p[h][i] = sum_j P[i][j] q_rot[h][j] in fp32 (q_rot =
+    // hi + lo), one (row i, 4 heads) item per thread and round, stored as fp16
+    // hi + lo parts (the padding heads give zeros).
+    if constexpr (is_qjl(KT)) {
+      constexpr int NH = 8 * NTH;
+      for (int it = threadIdx.x; it < D * (NH / 4); it += L::NW * 32) {
+        const int i = it % D, h0 = (it / D) * 4;
+        const float4* prow = reinterpret_cast<const float4*>(p.tqk.proj + (size_t)i * D);
+        float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int j4 = 0; j4 < D / 4; ++j4) {
+          const float4 pv = __ldg(prow + j4);
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) {
+            const __half2* qh = reinterpret_cast<const __half2*>(qhi + (h0 + hh) * D + 4 * j4);
+            const __half2* ql = reinterpret_cast<const __half2*>(qlo + (h0 + hh) * D + 4 * j4);
+            const float2 h01 = __half22float2(qh[0]), h23 = __half22float2(qh[1]);
+            const float2 l01 = __half22float2(ql[0]), l23 = __half22float2(ql[1]);
+            acc4[hh] += pv.x * (h01.x + l01.x) + pv.y * (h01.y + l01.y) + pv.z * (h23.x + l23.x) +
+                        pv.w * (h23.y + l23.y);
+          }
+        }
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) {
+          const __half hi = __float2half_rn(acc4[hh]);
+          phi[(h0 + hh) * PST + i] = hi;
+          plo[(h0 + hh) * PST + i] = __float2half_rn(acc4[hh] - __half2float(hi));
+        }
+      }
+      __syncthreads();
+    }
   }
 
   // ---- queries: B fragments of Q^T per (block, k-step) and, for quantized
@@ -709,6 +765,20 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         hi = prmt(e0, e1, 0x5410);
         lo = prmt(e0, e1, 0x7632);
       };
+      // turbo3_qjl: the 16 sign bits of a row's k-step (bit i of the z field,
+      // after the D/4 bytes of level codes); bits j, j+1 of a window as the
+      // fp16 pair (1 - 2 z_j, 1 - 2 z_j+1)
+      auto zwindow = [&](int row, int kstep) -> uint32_t {
+        const int byte0 = D / 4 + 2 * kstep;
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(kcp + row * L::RBK + (byte0 & ~3));
+        return w >> (8 * (byte0 & 3));
+      };
+      auto zpair = [](uint32_t f, int j) -> uint32_t {
+        return 0x3C003C00u | (((f >> j) & 1u) << 15) | (((f >> (j + 1)) & 1u) << 31);
+      };
+      float sz[NTH][4];  // turbo3_qjl: <P q_rot, 1 - 2z> of rows g, g+8
+#pragma unroll
+      for (int nt = 0; nt < NTH; ++nt) sz[nt][0] = sz[nt][1] = sz[nt][2] = sz[nt][3] = 0.f;
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
 #pragma unroll
@@ -719,6 +789,14 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           pair(fb, 2 * c, h[1], l[1]);
           pair(fa, 2 * c + 8, h[2], l[2]);
           pair(fb, 2 * c + 8, h[3], l[3]);
+          uint32_t zq[4] = {0u, 0u, 0u, 0u};
+          if constexpr (is_qjl(KT)) {
+            const uint32_t za = zwindow(g, 2 * blk + s2), zb = zwindow(g + 8, 2 * blk + s2);
+            zq[0] = zpair(za, 2 * c);
+            zq[1] = zpair(zb, 2 * c);
+            zq[2] = zpair(za, 2 * c + 8);
+            zq[3] = zpair(zb, 2 * c + 8);
+          }
           const int d0 = 32 * blk + 16 * s2 + 2 * c;
 #pragma unroll
           for (int nt = 0; nt < NTH; ++nt) {
@@ -729,17 +807,38 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
             mma16816(sc[nt], h[0], h[1], h[2], h[3], qb[nt][blk][s2][0], qb[nt][blk][s2][1], sc[nt]);
             mma16816(sc[nt], h[0], h[1], h[2], h[3], bl0, bl1, sc[nt]);
             mma16816(sc[nt], l[0], l[1], l[2], l[3], qb[nt][blk][s2][0], qb[nt][blk][s2][1], sc[nt]);
+            if constexpr (is_qjl(KT)) {  // the +-1 signs are exact: (p_hi + p_lo) . (1 - 2z)
+              const __half* ph = phi + (nt * 8 + g) * PST + d0;
+              const __half* pl = plo + (nt * 8 + g) * PST + d0;
+              mma16816(sz[nt], zq[0], zq[1], zq[2], zq[3], *reinterpret_cast<const uint32_t*>(ph),
+                       *reinterpret_cast<const uint32_t*>(ph + 8), sz[nt]);
+              mma16816(sz[nt], zq[0], zq[1], zq[2], zq[3], *reinterpret_cast<const uint32_t*>(pl),
+                       *reinterpret_cast<const uint32_t*>(pl + 8), sz[nt]);
+            }
           }
         }
       }
-      // the rows' norms / D
-      const float nA = __half2float(ksc[g]) * (1.0f / D), nB = __half2float(ksc[g + 8]) * (1.0f / D);
+      // the rows' norms / D (turbo3_qjl: plus the QJL term, gamma * sqrt(pi/2) / D^1.5)
+      const float nA = __half2float(ksc[g * L::NSK]) * (1.0f / D);
+      const float nB = __half2float(ksc[(g + 8) * L::NSK]) * (1.0f / D);
+      if constexpr (is_qjl(KT)) {
+        constexpr float kQ = 1.2533141373155003f / D * (D == 64 ? 0.125f : D == 128 ? 0.08838834764831845f : 0.0625f);
+        const float gA = __half2float(ksc[g * L::NSK + 1]) * kQ, gB = __half2float(ksc[(g + 8) * L::NSK + 1]) * kQ;
 #pragma unroll
-      for (int nt = 0; nt < NTH; ++nt) {
-        sc[nt][0] *= qs * nA;
-        sc[nt][1] *= qs * nA;
-        sc[nt][2] *= qs * nB;
-        sc[nt][3] *= qs * nB;
+        for (int nt = 0; nt < NTH; ++nt) {
+          sc[nt][0] = qs * (nA * sc[nt][0] + gA * sz[nt][0]);
+          sc[nt][1] = qs * (nA * sc[nt][1] + gA * sz[nt][1]);
+          sc[nt][2] = qs * (nB * sc[nt][2] + gB * sz[nt][2]);
+          sc[nt][3] = qs * (nB * sc[nt][3] + gB * sz[nt][3]);
+        }
+      } else {
+#pragma unroll
+        for (int nt = 0; nt < NTH; ++nt) {
+          sc[nt][0] *= qs * nA;
+          sc[nt][1] *= qs * nA;
+          sc[nt][2] *= qs * nB;
+          sc[nt][3] *= qs * nB;
+        }
       }
       return;
     }
@@ -1084,8 +1183,8 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     const int nv1 = rem <= kHalf ? 0 : (rem - kHalf < kHalf ? rem - kHalf : kHalf);
     const bool two = nv1 > 0;
     const bool tail0 = nv0 < kHalf, tail1 = two && nv1 < kHalf;
-    const uint32_t kc0 = wbase32 + st * L::KC;
-    const uint32_t vc32 = wbase32 + S * L::KC + st * L::VC;
+    const uint32_t kc0 = wbase32 + L::KOFF + st * L::KC;
+    const uint32_t vc32 = wbase32 + L::VOFF + st * L::VC;
     const __half* ks0 = reinterpret_cast<const __half*>(ks_of(st));
     const unsigned char* vc0 = vc_of(st);
     const __half* vs0 = reinterpret_cast<const __half*>(vs_of(st));
@@ -1556,7 +1655,12 @@ cudaError_t launch_v(int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStre
 
 template <int KT, bool PAGED>
 cudaError_t launch_k(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st) {
-  if constexpr (is_turbo(KT)) {  // turbo keys: q8_0, q4_0 or the same turbo type as values
+  if constexpr (is_qjl(KT)) {  // turbo3_qjl keys: q8_0, q4_0 or turbo3 values
+    if (vt == KVQ_Q8_0) return launch_v<KT, KVQ_Q8_0, PAGED>(nb, nth, a, m, st);
+    if (vt == KVQ_Q4_0) return launch_v<KT, KVQ_Q4_0, PAGED>(nb, nth, a, m, st);
+    if (vt == KVQ_TURBO3) return launch_v<KT, KVQ_TURBO3, PAGED>(nb, nth, a, m, st);
+    return cudaErrorInvalidValue;
+  } else if constexpr (is_turbo(KT)) {  // turbo keys: q8_0, q4_0 or the same turbo type as values
     if (vt == KVQ_Q8_0) return launch_v<KT, KVQ_Q8_0, PAGED>(nb, nth, a, m, st);
     if (vt == KVQ_Q4_0) return launch_v<KT, KVQ_Q4_0, PAGED>(nb, nth, a, m, st);
     if (vt == KT) return launch_v<KT, KT, PAGED>(nb, nth, a, m, st);
@@ -1584,6 +1688,7 @@ cudaError_t launch_kq5(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m
 cudaError_t launch_kt2(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kt3(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kt4(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kqjl(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kf16_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq8_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kq4_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
@@ -1591,6 +1696,7 @@ cudaError_t launch_kq5_paged(int vt, int nb, int nth, const TcArgs& a, const TcM
 cudaError_t launch_kt2_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kt3_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 cudaError_t launch_kt4_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
+cudaError_t launch_kqjl_paged(int vt, int nb, int nth, const TcArgs& a, const TcMaps& m, cudaStream_t st);
 
 }  // namespace tc
 }  // namespace kvq

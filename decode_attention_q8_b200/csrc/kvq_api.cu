@@ -27,6 +27,7 @@ int32_t code_bytes_of(int32_t type, int32_t d) {
     case KVQ_TURBO2:
     case KVQ_TURBO3:
     case KVQ_TURBO4: return turbo_bits(type) * d / 8;
+    case KVQ_TURBO3_QJL: return 3 * d / 8;
   }
   return 0;
 }
@@ -40,6 +41,7 @@ int32_t n_scales_of(int32_t type, int32_t d) {
     case KVQ_TURBO2:
     case KVQ_TURBO3:
     case KVQ_TURBO4: return 1;
+    case KVQ_TURBO3_QJL: return 2;
   }
   return 0;
 }
@@ -51,7 +53,7 @@ thread_local std::string g_last_cuda_error;
 constexpr int64_t kMaxCtx = (int64_t)1 << 31;
 constexpr int64_t kMinChunk = 256;  // fewest rows per split the heuristic plans
 
-bool known_type(int32_t t) { return t >= KVQ_F16 && t <= KVQ_Q5_0; }
+bool known_type(int32_t t) { return t >= KVQ_F16 && t <= KVQ_TURBO3_QJL; }
 bool pow2(int32_t v) { return v > 0 && (v & (v - 1)) == 0; }
 bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
 int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
@@ -143,7 +145,16 @@ TurboConsts turbo_consts(const kvq_cache_desc* d, int32_t type) {
   std::memcpy(t.levels, cb.levels, sizeof(t.levels));
   std::memcpy(t.tau, cb.tau, sizeof(t.tau));
   sign_bits(d->turbo_seed, d->head_dim, t.sign_bits);
+  if (is_qjl(type)) {
+    t.proj = d->qjl_proj;
+    t.rsqrt_d = (float)(1.0 / std::sqrt((double)d->head_dim));
+  }
   return t;
+}
+
+// turbo3_qjl keys read their projection: present and 16-byte aligned.
+bool qjl_ok(const kvq_cache_desc* d) {
+  return !is_qjl(d->k_type) || (d->qjl_proj != nullptr && aligned(d->qjl_proj, 16));
 }
 
 // ---- splits -----------------------------------------------------------------
@@ -317,6 +328,7 @@ kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void*
   if (!aligned(k_cache, 256) || !aligned(v_cache, 256) || !aligned(q, 16) || !aligned(workspace, 256))
     return KVQ_ERR_INVALID;
   if (ctx_lens != nullptr && !aligned(ctx_lens, 4)) return KVQ_ERR_INVALID;
+  if (!qjl_ok(d)) return KVQ_ERR_INVALID;
   const int32_t G = d->n_q_heads / d->n_kv_heads;
   if (!decode_supported(d->k_type, d->v_type, G, d->head_dim)) return KVQ_ERR_UNSUPPORTED;
   const int32_t S = resolve_splits(d, batch, ctx_len, n_splits);
@@ -369,6 +381,7 @@ kvq_status append_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, co
   if ((do_k && (!aligned(k_cache, 256) || !aligned(k_new, 16))) ||
       (do_v && (!aligned(v_cache, 256) || !aligned(v_new, 16))))
     return KVQ_ERR_INVALID;
+  if (do_k && !qjl_ok(d)) return KVQ_ERR_INVALID;
   const int64_t rows = (int64_t)batch * n_tok * d->n_kv_heads;
   if (rows * (d->head_dim / 4) > ((int64_t)1 << 40)) return KVQ_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -494,6 +507,7 @@ kvq_status kvq_check_desc(const kvq_cache_desc* d) {
   if (!known_type(d->k_type) || !known_type(d->v_type)) return KVQ_ERR_INVALID;
   if (d->head_dim % kBlock || d->head_dim > kMaxHeadDim) return KVQ_ERR_UNSUPPORTED;
   if ((is_turbo(d->k_type) || is_turbo(d->v_type)) && !pow2(d->head_dim)) return KVQ_ERR_UNSUPPORTED;
+  if (is_qjl(d->v_type)) return KVQ_ERR_UNSUPPORTED;  // a key format
   if (d->n_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }

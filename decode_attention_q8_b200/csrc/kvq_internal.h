@@ -25,17 +25,22 @@ struct Plane {
   int32_t n_scales;
 };
 
-// Turbo value formats: 2, 3 or 4 bits per value, else 0.
+// Turbo formats: bits of a row's level codes (2, 3 or 4), else 0.  turbo3_qjl
+// rows hold 2-bit level codes and, after them, one QJL sign bit per value.
 __host__ __device__ constexpr int turbo_bits(int32_t t) {
-  return t == KVQ_TURBO2 ? 2 : t == KVQ_TURBO3 ? 3 : t == KVQ_TURBO4 ? 4 : 0;
+  return t == KVQ_TURBO2 || t == KVQ_TURBO3_QJL ? 2 : t == KVQ_TURBO3 ? 3 : t == KVQ_TURBO4 ? 4 : 0;
 }
 __host__ __device__ constexpr bool is_turbo(int32_t t) { return turbo_bits(t) != 0; }
+__host__ __device__ constexpr bool is_qjl(int32_t t) { return t == KVQ_TURBO3_QJL; }
 
-// A turbo type's codebook (2^b levels, 2^b - 1 thresholds) and sign bits.
+// A turbo type's codebook (2^b levels, 2^b - 1 thresholds) and sign bits;
+// for turbo3_qjl also the QJL projection and fl(1/sqrt(head_dim)).
 struct TurboConsts {
   float levels[16];
   float tau[15];
   uint32_t sign_bits[kMaxHeadDim / 32];  // bit i set -> s_i = -1
+  const float* proj;                     // [D][D] fp32, row-major (turbo3_qjl)
+  float rsqrt_d;
 };
 
 struct AppendParams {

@@ -53,6 +53,27 @@
  *              midpoints), code i in bits b*i .. b*i+b-1.  The TurboQuant page's
  *              FAQ ("¿Qué formato TurboQuant debería usar?") puts values at 2 to 3
  *              bits; 4 bits is the next width.  d/4 + 2 and d/2 + 2 bytes.
+ *   KVQ_TURBO3_QJL (keys only; head_dim a power of two) the TurboQuant page's
+ *              three parts at 3 bits per value (same section: rotation, optimal
+ *              scalar quantizer, QJL to keep inner products), read after the
+ *              published QJL / TurboQuant constructions: the turbo2 row (2-bit
+ *              codes, norm), then a 1-bit QJL code of its residual.  With g, norm
+ *              and code as for turbo2 (binary32, one rounding per operation):
+ *              e_i = fl(g_i - c32[code_i]) (c32 the binary32 4-level codebook);
+ *              u_i = sum_j P[i][j] * e_j summed left to right for j = 0 .. d-1,
+ *              P = desc->qjl_proj; z_i = 1 where u_i < 0;
+ *              eps = sqrtf(tree sum of fl(e_i^2));
+ *              gamma = fp16(min(fl(fl(norm * eps) * fl(1/sqrt(d))), 65504)),
+ *              the residual's norm.  Code row: the 2-bit codes (d/4 bytes),
+ *              then z_i in bit i of a d/8-byte field; scale row: (norm, gamma).
+ *              3d/8 + 4 bytes.  Decoded key:
+ *              x_hat = (norm/d) s H_un c[code]
+ *                      + sqrt(pi/2)/d * gamma * s H_un P^T (1 - 2z) / sqrt(d),
+ *              i.e. QJL of the residual r with S = P H_un diag(s) / sqrt(d),
+ *              whose entries are i.i.d. N(0,1) when P's are, so <q, x_hat> is
+ *              an unbiased estimate of <q, x> over the draw of P.  Decodes with
+ *              q8_0, q4_0 or turbo3 values; as a value type
+ *              KVQ_ERR_UNSUPPORTED.
  *   Turbo keys: a key row x_hat gives the score <q, x_hat> = (norm/d) *
  *   <H_un (s * q), c[code]>, so the decode rotates each query once.  The same
  *   page's FAQ finds keys more sensitive to compression than values.  Turbo keys
@@ -64,10 +85,11 @@
  *   rows_per_plane T = max_ctx rounded up to a multiple of 16;
  *   code plane  at byte 0:           [batch][n_kv_heads][T][code_bytes]
  *   scale plane at byte scale_offset: [batch][n_kv_heads][T][n_scales] fp16
- *   with code_bytes = 2d (f16), d (q8_0), d/2 (q4_0), 3d/8 (turbo3);
+ *   with code_bytes = 2d (f16), d (q8_0), d/2 (q4_0, q5_0), b*d/8 (turbo b),
+ *   3d/8 (turbo3_qjl);
  *   n_scales = 0 (f16), d/32 (q8_0, q4_0), 3d/32 (q5_0: the d/32 block scales,
  *   then the d/32 qh words, each as two fp16 slots, little-endian), 1 (turbo
- *   types, the norm);
+ *   types, the norm), 2 (turbo3_qjl: norm, gamma);
  *   scale_offset = code plane bytes rounded up to a multiple of 256.
  *   Within a row, q8_0 codes and q4_0 bytes are in block order, exactly as the
  *   block formats above; scale n of a row belongs to block n.
@@ -115,7 +137,8 @@ typedef enum {
   KVQ_TURBO3 = 3,
   KVQ_TURBO2 = 4,
   KVQ_TURBO4 = 5,
-  KVQ_Q5_0 = 6
+  KVQ_Q5_0 = 6,
+  KVQ_TURBO3_QJL = 7
 } kvq_type;
 
 typedef enum {
@@ -131,11 +154,16 @@ typedef struct {
   int32_t n_q_heads;   /* query heads, a multiple of n_kv_heads */
   int32_t n_kv_heads;  /* KV heads */
   int32_t head_dim;    /* multiple of 32, at most 256 */
-  int32_t k_type;      /* kvq_type of the key cache: F16, Q8_0 or Q4_0 */
-  int32_t v_type;      /* kvq_type of the value cache: any */
+  int32_t k_type;      /* kvq_type of the key cache: any */
+  int32_t v_type;      /* kvq_type of the value cache: any but TURBO3_QJL */
   int32_t reserved;    /* must be 0 */
   int64_t max_ctx;     /* rows the cache holds per (batch, KV head), >= 1 */
-  uint64_t turbo_seed; /* seed of the turbo3 sign vector (V only) */
+  uint64_t turbo_seed; /* seed of the turbo sign vector (K and V turbo types) */
+  /* TURBO3_QJL keys: the QJL projection P, device memory owned by the caller,
+   * fp32 [head_dim][head_dim] row-major (row i projects onto code bit i),
+   * 16-byte aligned, unchanged while the cache is in use; read by the append
+   * and decode calls (NULL there: KVQ_ERR_INVALID).  Ignored otherwise. */
+  const float* qjl_proj;
 } kvq_cache_desc;
 
 /* Byte layout of one cache tensor, as described above. */
@@ -194,9 +222,10 @@ KVQ_API size_t kvq_workspace_bytes(const kvq_cache_desc* desc, int32_t batch, in
  * the 7 binary32 thresholds between them.  Host only; no device needed. */
 KVQ_API kvq_status kvq_turbo3_codebook(float levels[8], float thresholds[7]);
 
-/* The codebook of a turbo type (KVQ_TURBO2, KVQ_TURBO3, KVQ_TURBO4): its 2^b
- * binary32 levels (ascending) into levels[] and the 2^b - 1 binary32
- * thresholds into thresholds[] (room for 16 and 15).  Host only. */
+/* The codebook of a turbo type (KVQ_TURBO2, KVQ_TURBO3, KVQ_TURBO4; for
+ * KVQ_TURBO3_QJL the 4-level codebook of its 2-bit codes): its 2^b binary32
+ * levels (ascending) into levels[] and the 2^b - 1 binary32 thresholds into
+ * thresholds[] (room for 16 and 15).  Host only. */
 KVQ_API kvq_status kvq_turbo_codebook(int32_t type, float* levels, float* thresholds);
 
 /* The turbo3 sign vector (+1.f / -1.f) for `seed`, head_dim entries (every

@@ -11,6 +11,8 @@ seeded fp16 generator:
               (base seed + 1000*layer + {0: Q, 1: K, 2: V});
   shapes      new K/V rows  [batch][n_tok][n_kv][head_dim]
               queries       [batch][n_q][head_dim]
+  projection  the turbo3_qjl key projection: float32 [head_dim][head_dim]
+              N(0,1) draws on the host (qjl_projection)
 
 The pages' own workloads (TinyLlama, Llama-3.1-70B and gpt-oss-20b runs)
 need trained weights; these synthetic tensors of the same shapes stand in for
@@ -86,6 +88,13 @@ def normal_f16(shape, seed, device="cpu", outlier_channels=(), outlier_scale=1.0
         idx = torch.tensor(outlier_channels, device=device)
         x[..., idx] *= outlier_scale
     return x.to(torch.float16)
+
+
+def qjl_projection(seed, head_dim):
+    """float32 [head_dim][head_dim] of N(0,1) draws on the host: the random
+    projection a turbo3_qjl key cache is coded with (the caller moves it to
+    the device for the library; the oracle takes the same host array)."""
+    return torch.randn((head_dim, head_dim), generator=_gen(seed, "cpu"), dtype=torch.float32)
 
 
 def layer_inputs(w: Workload, layer=0, device="cpu", n_tok=None, batch=None):

@@ -7,7 +7,7 @@ import numpy as np
 import torch
 
 import decode_attention_q8_b200 as kvq
-from oracle import attention, blocks, turbo, turbo3
+from oracle import attention, blocks, qjl, turbo, turbo3
 
 SENTINEL = 0xA5
 
@@ -36,8 +36,9 @@ def rows_of(cache_cpu, layout, b, h, n_kv, t0, t1):
     return codes, scales
 
 
-def oracle_rows(kind, x_f16, seed=0):
-    """Oracle codes/scales of rows x_f16 [n, D] in the same per-row form."""
+def oracle_rows(kind, x_f16, seed=0, proj=None):
+    """Oracle codes/scales of rows x_f16 [n, D] in the same per-row form
+    (proj: the turbo3_qjl projection, float32 [D][D] on the host)."""
     x = np.asarray(x_f16, np.float16)
     n, D = x.shape
     if kind == "f16":
@@ -57,10 +58,13 @@ def oracle_rows(kind, x_f16, seed=0):
     if kind in ("turbo2", "turbo4"):
         nrm, codes = turbo.quantize(x, seed, turbo.BITS[kind])
         return codes, nrm.reshape(n, 1)
+    if kind == "turbo3_qjl":
+        scales, codes = qjl.quantize(x, seed, proj)
+        return codes, scales
     raise ValueError(kind)
 
 
-def oracle_dequant(kind, codes, scales, D, seed=0):
+def oracle_dequant(kind, codes, scales, D, seed=0, proj=None):
     """float64 [n, D] decoded rows (oracle definitions) from stored codes/scales."""
     if kind == "f16":
         return blocks.dequantize_f16(np.ascontiguousarray(codes).view(np.float16))
@@ -76,6 +80,8 @@ def oracle_dequant(kind, codes, scales, D, seed=0):
         return turbo3.dequantize_turbo3(scales[:, 0], codes, seed, D)
     if kind in ("turbo2", "turbo4"):
         return turbo.dequantize(scales[:, 0], codes, seed, D, turbo.BITS[kind])
+    if kind == "turbo3_qjl":
+        return qjl.dequantize(scales, codes, seed, proj, D)
     raise ValueError(kind)
 
 

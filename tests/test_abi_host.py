@@ -46,11 +46,12 @@ def test_row_bytes_match_oracle_model():
         for d in (32, 64, 128, 256):
             assert kvq.kvq_row_bytes(t, d) == cache_model.row_bytes(t, d)
     for d in (32, 64, 128, 256):
-        for t in ("turbo2", "turbo3", "turbo4"):
+        for t in ("turbo2", "turbo3", "turbo4", "turbo3_qjl"):
             assert kvq.kvq_row_bytes(t, d) == cache_model.row_bytes(t, d)
     assert kvq.kvq_row_bytes("q8_0", 48) == 0
     assert kvq.kvq_row_bytes("turbo3", 96) == 0
-    assert kvq.kvq_row_bytes(7, 128) == 0
+    assert kvq.kvq_row_bytes("turbo3_qjl", 96) == 0
+    assert kvq.kvq_row_bytes(8, 128) == 0
     assert kvq.kvq_row_bytes("turbo2", 96) == 0
 
 
@@ -126,12 +127,14 @@ def test_check_desc():
         (kvq.make_desc(64, 8, 96, "q8_0", "turbo3", 16), kvq.KVQ_ERR_UNSUPPORTED),   # WHT needs 2^k
         (kvq.make_desc(64, 8, 96, "turbo2", "q4_0", 16), kvq.KVQ_ERR_UNSUPPORTED),
         (kvq.make_desc(64, 8, 96, "q8_0", "turbo4", 16), kvq.KVQ_ERR_UNSUPPORTED),
-        (kvq.make_desc(64, 8, 128, 7, "q4_0", 16), kvq.KVQ_ERR_INVALID),           # past the last type
+        (kvq.make_desc(64, 8, 128, 8, "q4_0", 16), kvq.KVQ_ERR_INVALID),           # past the last type
+        (kvq.make_desc(64, 8, 128, "q8_0", "turbo3_qjl", 16), kvq.KVQ_ERR_UNSUPPORTED),  # a key format
+        (kvq.make_desc(64, 8, 96, "turbo3_qjl", "q8_0", 16), kvq.KVQ_ERR_UNSUPPORTED),
     ]
     for desc, st in bad:
         assert kvq.kvq_check_desc(desc) == st
     # turbo keys are a valid description (the decode pairs them with q8_0, q4_0 or the same type)
-    for kt in ("turbo2", "turbo3", "turbo4"):
+    for kt in ("turbo2", "turbo3", "turbo4", "turbo3_qjl"):
         assert kvq.kvq_check_desc(kvq.make_desc(64, 8, 128, kt, "q4_0", 16)) == kvq.KVQ_OK
     d = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 16)
     d.reserved = 1
@@ -348,3 +351,21 @@ def test_auto_splits_bounded_and_nonempty():
             chunk = -(-(-(-ctx // s)) // 32) * 32
             assert (s - 1) * chunk < ctx
     assert kvq.kvq_auto_splits(d, 1, 0) == 0
+
+
+def test_qjl_keys_need_their_projection():
+    """turbo3_qjl keys: append, decode and the fused step read the projection,
+    so a missing or misaligned one is INVALID before any launch; the decode
+    pairs them with q8_0, q4_0 or turbo3 values only."""
+    for proj in (None, FAKE + 4):
+        d = kvq.make_desc(32, 8, 128, "turbo3_qjl", "q8_0", 64, qjl_proj=proj)
+        assert _append(d) == kvq.KVQ_ERR_INVALID
+        assert _decode(d) == kvq.KVQ_ERR_INVALID
+        assert _step(d) == kvq.KVQ_ERR_INVALID
+    for vt in ("f16", "q5_0", "turbo2", "turbo4"):
+        d = kvq.make_desc(32, 8, 128, "turbo3_qjl", vt, 64, qjl_proj=FAKE)
+        assert _decode(d) == kvq.KVQ_ERR_UNSUPPORTED
+        assert _step(d) == kvq.KVQ_ERR_UNSUPPORTED
+    lv, th = kvq.kvq_turbo_codebook("turbo3_qjl")
+    lv2, th2 = kvq.kvq_turbo_codebook("turbo2")
+    assert list(lv) == list(lv2) and list(th) == list(th2)

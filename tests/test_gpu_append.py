@@ -41,7 +41,9 @@ def _adversarial_rows(n, D, rng):
 
 def _check_append(k_type, v_type, D, B, H, max_ctx, pos, n_tok, seed, adversarial=False):
     rng = np.random.default_rng(seed)
-    desc = kvq.make_desc(H, H, D, k_type, v_type, max_ctx, turbo_seed=seed * 7919 + 1)
+    proj = synth.qjl_projection(seed + 5, D) if k_type == "turbo3_qjl" else None
+    desc = kvq.make_desc(H, H, D, k_type, v_type, max_ctx, turbo_seed=seed * 7919 + 1,
+                         qjl_proj=None if proj is None else proj.cuda())
     if adversarial:
         k_new = _adversarial_rows(B * n_tok * H, D, rng).reshape(B, n_tok, H, D)
         v_new = _adversarial_rows(B * n_tok * H, D, rng).reshape(B, n_tok, H, D)
@@ -58,7 +60,8 @@ def _check_append(k_type, v_type, D, B, H, max_ctx, pos, n_tok, seed, adversaria
         for b in range(B):
             for h in range(H):
                 codes, scales = rows_of(host, lay, b, h, H, pos, pos + n_tok)
-                ecodes, escales = oracle_rows(kind, new[b, :, h, :], desc.turbo_seed)
+                ecodes, escales = oracle_rows(kind, new[b, :, h, :], desc.turbo_seed,
+                                              None if proj is None else proj.numpy())
                 np.testing.assert_array_equal(codes, ecodes, err_msg=f"{kind} codes b{b} h{h}")
                 np.testing.assert_array_equal(scales.view(np.uint16), escales.view(np.uint16),
                                               err_msg=f"{kind} scales b{b} h{h}")
@@ -71,14 +74,15 @@ def _check_append(k_type, v_type, D, B, H, max_ctx, pos, n_tok, seed, adversaria
 @pytest.mark.parametrize("k_type,v_type", [("q8_0", "q4_0"), ("q4_0", "q8_0"), ("f16", "turbo3"),
                                            ("q8_0", "turbo3"), ("f16", "f16"), ("q8_0", "turbo2"),
                                            ("q4_0", "turbo4"), ("q5_0", "q5_0"), ("q8_0", "q5_0"),
-                                           ("turbo3", "turbo3"), ("turbo2", "q8_0"), ("turbo4", "turbo4")])
+                                           ("turbo3", "turbo3"), ("turbo2", "q8_0"), ("turbo4", "turbo4"),
+                                           ("turbo3_qjl", "q8_0"), ("turbo3_qjl", "turbo3")])
 @pytest.mark.parametrize("D", [32, 64, 128, 256])
 def test_append_bit_exact(k_type, v_type, D):
     _check_append(k_type, v_type, D, B=2, H=3, max_ctx=100, pos=37, n_tok=21, seed=D)
 
 
 @pytest.mark.parametrize("k_type,v_type", [("q8_0", "q4_0"), ("q4_0", "turbo3"), ("q8_0", "turbo2"),
-                                           ("f16", "turbo4"), ("q5_0", "q5_0")])
+                                           ("f16", "turbo4"), ("q5_0", "q5_0"), ("turbo3_qjl", "q4_0")])
 def test_append_adversarial_blocks(k_type, v_type):
     _check_append(k_type, v_type, 128, B=1, H=2, max_ctx=64, pos=0, n_tok=64, seed=3, adversarial=True)
 

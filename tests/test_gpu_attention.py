@@ -21,8 +21,11 @@ pytestmark = pytest.mark.gpu
 def _setup(k_type, v_type, B, n_q, n_kv, D, ctx, seed, max_ctx=None, outliers=(3, 17), oscale=10.0,
            turbo_seed=None):
     max_ctx = max_ctx or ctx
+    proj = synth.qjl_projection(seed + 11, D) if k_type == "turbo3_qjl" else None
     desc = kvq.make_desc(n_q, n_kv, D, k_type, v_type, max_ctx,
-                         turbo_seed=(seed * 31 + 7) if turbo_seed is None else turbo_seed)
+                         turbo_seed=(seed * 31 + 7) if turbo_seed is None else turbo_seed,
+                         qjl_proj=None if proj is None else proj.cuda())
+    desc.qjl_host = None if proj is None else proj.numpy()
     w = synth.Workload("case", B, 1, n_q, n_kv, D, ctx, k_type, v_type, outliers, oscale, seed)
     q, k, v = synth.layer_inputs(w, device="cuda")
     kc, vc = alloc_cache(desc, B, 0), alloc_cache(desc, B, 1)
@@ -33,11 +36,12 @@ def _setup(k_type, v_type, B, n_q, n_kv, D, ctx, seed, max_ctx=None, outliers=(3
 def _oracle_out(desc, q, k, v, b, g, ctx, scale):
     """Oracle outputs [G, D] of the query heads of KV head g in batch row b."""
     G = desc.n_q_heads // desc.n_kv_heads
-    names = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4", 6: "q5_0"}
+    names = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4", 6: "q5_0", 7: "turbo3_qjl"}
     kt, vt = names[desc.k_type], names[desc.v_type]
     kx = k[b, :ctx, g, :].cpu().numpy()
     vx = v[b, :ctx, g, :].cpu().numpy()
-    kh = oracle_dequant(kt, *oracle_rows(kt, kx, desc.turbo_seed), desc.head_dim, desc.turbo_seed)
+    proj = getattr(desc, "qjl_host", None)
+    kh = oracle_dequant(kt, *oracle_rows(kt, kx, desc.turbo_seed, proj), desc.head_dim, desc.turbo_seed, proj)
     vh = oracle_dequant(vt, *oracle_rows(vt, vx, desc.turbo_seed), desc.head_dim, desc.turbo_seed)
     return oracle_attention_rows(q[b, g * G:(g + 1) * G].cpu().numpy(), kh, vh, scale)
 
@@ -94,6 +98,20 @@ def test_turbo_keys(k_type, v_type, G, D):
     for S in (0, 3):
         out = decode(desc, kc, vc, q, 2, 400, 1 / math.sqrt(D), S)
         _check_all(desc, q, k, v, out, 400, 1 / math.sqrt(D), f"{k_type}/{v_type} G={G} D={D} S={S}")
+
+
+@pytest.mark.parametrize("v_type", ["q8_0", "q4_0", "turbo3"])
+@pytest.mark.parametrize("G", [1, 8, 16])
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_qjl_keys(v_type, G, D):
+    """turbo3_qjl keys: the rotated query scores the 2-bit levels (scaled by
+    norm / D) and, projected once by P, the QJL sign bits (scaled by
+    gamma * sqrt(pi/2) / D^1.5)."""
+    n_kv = 2
+    desc, q, k, v, kc, vc = _setup("turbo3_qjl", v_type, 2, n_kv * G, n_kv, D, 400, seed=G * 5 + D + 1)
+    for S in (0, 3):
+        out = decode(desc, kc, vc, q, 2, 400, 1 / math.sqrt(D), S)
+        _check_all(desc, q, k, v, out, 400, 1 / math.sqrt(D), f"qjl/{v_type} G={G} D={D} S={S}")
 
 
 @pytest.mark.parametrize("k_type,v_type", [("q5_0", "q5_0"), ("q5_0", "q8_0"), ("q8_0", "q5_0")])

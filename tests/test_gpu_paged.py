@@ -19,11 +19,14 @@ from kvq_testlib import SENTINEL, alloc_cache, assert_attention_close, oracle_at
 
 pytestmark = pytest.mark.gpu
 
-NAMES = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4", 6: "q5_0"}
+NAMES = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4", 6: "q5_0", 7: "turbo3_qjl"}
 
 
 def _inputs(k_type, v_type, B, n_q, n_kv, D, rows, max_ctx, seed):
-    desc = kvq.make_desc(n_q, n_kv, D, k_type, v_type, max_ctx, turbo_seed=seed * 31 + 7)
+    proj = synth.qjl_projection(seed + 17, D) if k_type == "turbo3_qjl" else None
+    desc = kvq.make_desc(n_q, n_kv, D, k_type, v_type, max_ctx, turbo_seed=seed * 31 + 7,
+                         qjl_proj=None if proj is None else proj.cuda())
+    desc.qjl_host = None if proj is None else proj.numpy()
     w = synth.Workload("paged", B, 1, n_q, n_kv, D, rows, k_type, v_type, (3, 17), 10.0, seed)
     q, k, v = synth.layer_inputs(w, device="cuda")
     return desc, q, k, v
@@ -73,7 +76,8 @@ def _pages_equal_contiguous(desc, pools, table, page_rows, n_pages, cont, B, len
 
 
 @pytest.mark.parametrize("k_type,v_type,page_rows", [("q8_0", "q4_0", 64), ("q8_0", "turbo3", 32),
-                                                     ("q4_0", "q4_0", 256), ("f16", "q8_0", 128)])
+                                                     ("q4_0", "q4_0", 256), ("f16", "q8_0", 128),
+                                                     ("turbo3_qjl", "q4_0", 64)])
 def test_paged_equals_contiguous(k_type, v_type, page_rows):
     B, n_q, n_kv, D, rows = 3, 16, 4, 128, 1500
     max_pages = (rows + page_rows - 1) // page_rows
@@ -103,7 +107,8 @@ def test_paged_equals_contiguous(k_type, v_type, page_rows):
     # and one group against the oracle directly
     G = n_q // n_kv
     b, g, n = 0, 1, lens[0]
-    kh = oracle_dequant(k_type, *oracle_rows(k_type, k[b, :n, g].cpu().numpy()), D)
+    kh = oracle_dequant(k_type, *oracle_rows(k_type, k[b, :n, g].cpu().numpy(), desc.turbo_seed, desc.qjl_host), D,
+                        desc.turbo_seed, desc.qjl_host)
     vh = oracle_dequant(v_type, *oracle_rows(v_type, v[b, :n, g].cpu().numpy(), desc.turbo_seed), D, desc.turbo_seed)
     assert_attention_close(got.cpu().numpy()[b, g * G:(g + 1) * G],
                            oracle_attention_rows(q[b, g * G:(g + 1) * G].cpu().numpy(), kh, vh, scale), "paged oracle")

@@ -16,12 +16,15 @@ from kvq_testlib import (alloc_cache, assert_attention_close, decode, oracle_att
 
 pytestmark = pytest.mark.gpu
 
-NAMES = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4", 6: "q5_0"}
+NAMES = {0: "f16", 1: "q8_0", 2: "q4_0", 3: "turbo3", 4: "turbo2", 5: "turbo4", 6: "q5_0", 7: "turbo3_qjl"}
 
 
 def _inputs(k_type, v_type, B, n_q, n_kv, D, ctx, seed, max_ctx=None, turbo_seed=None):
+    proj = synth.qjl_projection(seed + 13, D) if k_type == "turbo3_qjl" else None
     desc = kvq.make_desc(n_q, n_kv, D, k_type, v_type, max_ctx or ctx,
-                         turbo_seed=(seed * 31 + 7) if turbo_seed is None else turbo_seed)
+                         turbo_seed=(seed * 31 + 7) if turbo_seed is None else turbo_seed,
+                         qjl_proj=None if proj is None else proj.cuda())
+    desc.qjl_host = None if proj is None else proj.numpy()
     w = synth.Workload("case", B, 1, n_q, n_kv, D, ctx, k_type, v_type, (3, 17), 10.0, seed)
     q, k, v = synth.layer_inputs(w, device="cuda")
     return desc, q, k, v
@@ -44,8 +47,9 @@ def _step(desc, kc, vc, q, k, v, B, ctx, scale, S, ws):
 def _oracle(desc, q, k, v, b, g, ctx, scale):
     G = desc.n_q_heads // desc.n_kv_heads
     kt, vt = NAMES[desc.k_type], NAMES[desc.v_type]
-    kh = oracle_dequant(kt, *oracle_rows(kt, k[b, :ctx, g, :].cpu().numpy(), desc.turbo_seed), desc.head_dim,
-                        desc.turbo_seed)
+    proj = getattr(desc, "qjl_host", None)
+    kh = oracle_dequant(kt, *oracle_rows(kt, k[b, :ctx, g, :].cpu().numpy(), desc.turbo_seed, proj),
+                        desc.head_dim, desc.turbo_seed, proj)
     vh = oracle_dequant(vt, *oracle_rows(vt, v[b, :ctx, g, :].cpu().numpy(), desc.turbo_seed), desc.head_dim,
                         desc.turbo_seed)
     return oracle_attention_rows(q[b, g * G:(g + 1) * G].cpu().numpy(), kh, vh, scale)
@@ -66,7 +70,8 @@ def _check_row_bytes(desc, kc, vc, k, v, B, row, what):
         for b in range(B):
             for g in range(desc.n_kv_heads):
                 codes, scales = rows_of(host, lay, b, g, desc.n_kv_heads, row, row + 1)
-                ec, es = oracle_rows(kind, x[b, row:row + 1, g, :].cpu().numpy(), desc.turbo_seed)
+                ec, es = oracle_rows(kind, x[b, row:row + 1, g, :].cpu().numpy(), desc.turbo_seed,
+                                     getattr(desc, "qjl_host", None))
                 np.testing.assert_array_equal(codes, ec, err_msg=f"{what} {kind} codes b{b} g{g}")
                 np.testing.assert_array_equal(scales.view(np.uint16), es.view(np.uint16),
                                               err_msg=f"{what} {kind} scales b{b} g{g}")
@@ -76,7 +81,8 @@ def _pairs():
     plain = [(k, v) for k in ("f16", "q8_0", "q4_0", "q5_0")
              for v in ("f16", "q8_0", "q4_0", "turbo3", "turbo2", "turbo4", "q5_0")]
     turbo_keys = [(k, v) for k in ("turbo2", "turbo3", "turbo4") for v in ("q8_0", "q4_0", k)]
-    return plain + turbo_keys
+    qjl_keys = [("turbo3_qjl", v) for v in ("q8_0", "q4_0", "turbo3")]
+    return plain + turbo_keys + qjl_keys
 
 
 @pytest.mark.parametrize("k_type,v_type", _pairs())
