@@ -29,11 +29,13 @@ __host__ __device__ constexpr int bulk_items(int32_t type, int d) {
 struct AppendPair {
   AppendParams p[2];
   int32_t type[2];
-  int32_t n;  // tensors in the call (1 or 2)
+  int32_t n;           // tensors in the call (1 or 2)
+  int32_t stage_proj;  // turbo3_qjl keys: copy P to shared memory first
 };
 
 template <int TYPE, int E>
-__device__ __forceinline__ void append_stream(const AppendParams& p, int64_t first, int64_t stride, int64_t gend) {
+__device__ __forceinline__ void append_stream(const AppendParams& p, int64_t first, int64_t stride, int64_t gend,
+                                              const float* pt = nullptr) {
   for (int64_t base = first; (base & ~(int64_t)31) < gend; base += kAppendRound * stride) {
     uint4 raw[kAppendRound];
 #pragma unroll
@@ -41,7 +43,7 @@ __device__ __forceinline__ void append_stream(const AppendParams& p, int64_t fir
 #pragma unroll
     for (int u = 0; u < kAppendRound; ++u) {
       const int64_t g = base + u * stride;
-      if ((g & ~(int64_t)31) < gend) rows::finish<TYPE, E>(p, g, gend, raw[u]);  // warp-uniform
+      if ((g & ~(int64_t)31) < gend) rows::finish<TYPE, E>(p, g, gend, raw[u], pt);  // warp-uniform
     }
   }
 }
@@ -69,19 +71,21 @@ __device__ __forceinline__ void append_blocks(const AppendParams& p, int64_t fir
 }
 
 template <int TYPE>
-__device__ __forceinline__ void append_turbo_part(const AppendParams& p, int64_t first, int64_t stride, int64_t gend) {
+__device__ __forceinline__ void append_turbo_part(const AppendParams& p, int64_t first, int64_t stride, int64_t gend,
+                                                  const float* pt = nullptr) {
   switch (p.D) {
-    case 32: append_stream<TYPE, 1>(p, first, stride, gend); break;
-    case 64: append_stream<TYPE, 2>(p, first, stride, gend); break;
-    case 128: append_stream<TYPE, 4>(p, first, stride, gend); break;
-    case 256: append_stream<TYPE, 8>(p, first, stride, gend); break;
+    case 32: append_stream<TYPE, 1>(p, first, stride, gend, pt); break;
+    case 64: append_stream<TYPE, 2>(p, first, stride, gend, pt); break;
+    case 128: append_stream<TYPE, 4>(p, first, stride, gend, pt); break;
+    case 256: append_stream<TYPE, 8>(p, first, stride, gend, pt); break;
   }
 }
 
 // QJL: the instance that also takes turbo3_qjl rows (their projection loop
 // needs far more registers; the other types keep the lean instance).
 template <bool QJL>
-__device__ __forceinline__ void append_part(const AppendParams& p, int32_t type, int64_t first, int64_t stride) {
+__device__ __forceinline__ void append_part(const AppendParams& p, int32_t type, int64_t first, int64_t stride,
+                                            const float* pt) {
   const int64_t gend = (int64_t)p.B * p.n_tok * p.H * bulk_items(type, p.D);
   switch (type) {
     case KVQ_F16: append_stream<KVQ_F16, 0>(p, first, stride, gend); break;
@@ -92,26 +96,47 @@ __device__ __forceinline__ void append_part(const AppendParams& p, int32_t type,
     case KVQ_TURBO3: append_turbo_part<KVQ_TURBO3>(p, first, stride, gend); break;
     case KVQ_TURBO4: append_turbo_part<KVQ_TURBO4>(p, first, stride, gend); break;
     case KVQ_TURBO3_QJL:
-      if constexpr (QJL) append_turbo_part<KVQ_TURBO3_QJL>(p, first, stride, gend);
+      if constexpr (QJL) append_turbo_part<KVQ_TURBO3_QJL>(p, first, stride, gend, pt);
       break;
   }
 }
+
+// The QJL instance first copies the keys' projection P transposed into shared
+// memory when it fits (D <= kQjlSmemDim) and a CTA has enough rows to repay
+// the copy (at least kQjlStageRows), so each step of a row's projection reads
+// one contiguous line; every output still sums its D terms in order.
+constexpr int kQjlSmemDim = 128;
+constexpr int kQjlStageRows = 32;
 
 template <bool QJL>
 __global__ void __launch_bounds__(kAppendThreads) append_pair_kernel(const AppendPair pp) {
   const int64_t first = (int64_t)blockIdx.x * kAppendThreads + threadIdx.x;
   const int64_t stride = (int64_t)gridDim.x * kAppendThreads;
-  append_part<QJL>(pp.p[0], pp.type[0], first, stride);
-  if (pp.n == 2) append_part<QJL>(pp.p[1], pp.type[1], first, stride);
+  const float* pt = nullptr;
+  if constexpr (QJL) {
+    extern __shared__ float pt_smem[];
+    const AppendParams& pk = pp.p[0];  // turbo3_qjl is a key type: the first tensor
+    if (pp.stage_proj) {
+      const int D = pk.D;
+      for (int t = threadIdx.x; t < D * D; t += kAppendThreads) {
+        const int i = t / D, j = t - i * D;  // coalesced read of P[i][j]
+        pt_smem[j * D + i] = __ldg(pk.tq.proj + t);
+      }
+      __syncthreads();
+      pt = pt_smem;
+    }
+  }
+  append_part<QJL>(pp.p[0], pp.type[0], first, stride, pt);
+  if (pp.n == 2) append_part<QJL>(pp.p[1], pp.type[1], first, stride, pt);
 }
 
 // Resident 256-thread CTAs of the append kernel on the whole current device
 // (one wave); 148 SMs x 4 if the device cannot be asked.
 template <bool QJL>
-int64_t resident_ctas() {
+int64_t resident_ctas(size_t smem) {
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, append_pair_kernel<QJL>, kAppendThreads, 0) !=
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, append_pair_kernel<QJL>, kAppendThreads, smem) !=
           cudaSuccess ||
       sms <= 0 || per_sm <= 0) {
     (void)cudaGetLastError();
@@ -145,12 +170,28 @@ cudaError_t launch_append(const AppendParams* k, int32_t k_type, const AppendPar
   int64_t need = append_ctas(pp.type[0], pp.p[0]);
   if (n == 2) need = std::max(need, append_ctas(pp.type[1], pp.p[1]));
   const bool qjl = is_qjl(pp.type[0]) || (n == 2 && is_qjl(pp.type[1]));
-  const int64_t ctas = std::min(need, qjl ? resident_ctas<true>() : resident_ctas<false>());
-  if (ctas <= 0) return cudaSuccess;  // no rows
-  if (qjl)
-    append_pair_kernel<true><<<(unsigned)ctas, kAppendThreads, 0, st>>>(pp);
-  else
+  if (!qjl) {
+    const int64_t ctas = std::min(need, resident_ctas<false>(0));
+    if (ctas <= 0) return cudaSuccess;  // no rows
     append_pair_kernel<false><<<(unsigned)ctas, kAppendThreads, 0, st>>>(pp);
+    return cudaGetLastError();
+  }
+  // turbo3_qjl keys come first (a key type); P transposed in shared memory
+  const int D = pp.p[0].D;
+  const bool can_stage = is_qjl(pp.type[0]) && D <= kQjlSmemDim;
+  static bool attr_set = false;  // idempotent; a race only repeats the call
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(append_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)(sizeof(float) * kQjlSmemDim * kQjlSmemDim));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int64_t ctas = std::min(need, resident_ctas<true>(can_stage ? sizeof(float) * D * D : 0));
+  if (ctas <= 0) return cudaSuccess;
+  const int64_t key_rows = (int64_t)pp.p[0].B * pp.p[0].n_tok * pp.p[0].H;
+  pp.stage_proj = can_stage && key_rows >= kQjlStageRows * ctas ? 1 : 0;
+  const size_t smem = pp.stage_proj ? sizeof(float) * D * D : 0;
+  append_pair_kernel<true><<<(unsigned)ctas, kAppendThreads, smem, st>>>(pp);
   return cudaGetLastError();
 }
 

@@ -417,8 +417,12 @@ __device__ __forceinline__ void append_f16(const AppendParams& p, int64_t gtid, 
 // codes, the residual e = g - c[code] of each element, its norm by the same
 // tree, and the sign bits of u = P e; lane l computes u_i of its own rows
 // i = l*E .. l*E+E-1, taking e_j (j = 0 .. D-1 in order) from its owner lane.
+// P comes from pt, a transposed copy in shared memory (pt[j*D + i] = P[i][j]:
+// the warp reads one contiguous line per j), or, when pt is null, from global
+// memory row by row.
 template <int BITS, int E, bool QJL = false>
-__device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
+__device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw,
+                                             const float* pt) {
   constexpr int D = 32 * E;
   const int64_t row = gtid >> 5;
   const int lane = (int)(gtid & 31);
@@ -504,9 +508,38 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
     float u[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) u[e] = 0.0f;
+    if (pt != nullptr) {
+#pragma unroll 2
+      for (int jl = 0; jl < 32; ++jl) {
+#pragma unroll
+        for (int e2 = 0; e2 < E; ++e2) {
+          const float ej = __shfl_sync(0xffffffffu, res[e2], jl);
+          const float* col = pt + (jl * E + e2) * D + lane * E;  // P[lane*E .. lane*E+E-1][j]
+          float pv[E];
+          if constexpr (E % 4 == 0) {
+#pragma unroll
+            for (int k4 = 0; k4 < E; k4 += 4) {
+              const float4 f = *reinterpret_cast<const float4*>(col + k4);
+              pv[k4] = f.x;
+              pv[k4 + 1] = f.y;
+              pv[k4 + 2] = f.z;
+              pv[k4 + 3] = f.w;
+            }
+          } else if constexpr (E == 2) {
+            const float2 f = *reinterpret_cast<const float2*>(col);
+            pv[0] = f.x;
+            pv[1] = f.y;
+          } else {
+            pv[0] = col[0];
+          }
+#pragma unroll
+          for (int e = 0; e < E; ++e) u[e] = __fadd_rn(u[e], __fmul_rn(pv[e], ej));
+        }
+      }
+    }
     const float* prow = p.tq.proj + (size_t)(lane * E) * D;  // row lane*E of P
 #pragma unroll 4
-    for (int jl = 0; jl < 32; ++jl) {  // e_j of j = jl*E .. jl*E+E-1, held by lane jl
+    for (int jl = 0; jl < (pt == nullptr ? 32 : 0); ++jl) {  // e_j of j = jl*E .. jl*E+E-1, held by lane jl
       float ej[E];
 #pragma unroll
       for (int e2 = 0; e2 < E; ++e2) ej[e2] = __shfl_sync(0xffffffffu, res[e2], jl);
@@ -584,12 +617,13 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
 // Quantize and store work item gtid from its loaded bytes (every lane of the
 // warp calls this: the bodies shuffle; items at or past gend store nothing).
 template <int TYPE, int E>
-__device__ __forceinline__ void finish(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw) {
+__device__ __forceinline__ void finish(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw,
+                                       const float* pt = nullptr) {
   if constexpr (TYPE == KVQ_Q8_0) append_q8_0(p, gtid, gend, raw);
   else if constexpr (TYPE == KVQ_Q4_0) append_q4_0(p, gtid, gend, raw);
   else if constexpr (TYPE == KVQ_Q5_0) append_q5_0(p, gtid, gend, raw);
   else if constexpr (TYPE == KVQ_F16) append_f16(p, gtid, gend, raw);
-  else append_turbo<turbo_bits(TYPE), E, is_qjl(TYPE)>(p, gtid, gend, raw);
+  else append_turbo<turbo_bits(TYPE), E, is_qjl(TYPE)>(p, gtid, gend, raw, pt);
 }
 
 template <int TYPE, int E>

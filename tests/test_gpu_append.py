@@ -121,3 +121,25 @@ def test_append_rejects_out_of_range_without_writing():
         kvq.kvq_append_quantize(desc, kc, vc, rows, rows, 1, 30, 4)
     torch.cuda.synchronize()
     assert bool((kc == SENTINEL).all()) and bool((vc == SENTINEL).all())
+
+
+@pytest.mark.parametrize("D", [32, 64, 128])
+def test_qjl_bulk_append_staged_projection(D):
+    """A prefill large enough that every CTA holds many rows: the append kernel
+    then reads the projection from a transposed shared-memory copy.  The bytes
+    must still match the oracle's left-to-right sums bit for bit."""
+    B, H, n_tok = 1, 8, 8192
+    proj = synth.qjl_projection(D + 3, D)
+    desc = kvq.make_desc(H, H, D, "turbo3_qjl", "q8_0", n_tok, turbo_seed=D * 3 + 1, qjl_proj=proj.cuda())
+    k_new = synth.normal_f16((B, n_tok, H, D), D + 100, outlier_channels=(3, 17), outlier_scale=10.0)
+    v_new = synth.normal_f16((B, n_tok, H, D), D + 101)
+    kc, vc = alloc_cache(desc, B, 0), alloc_cache(desc, B, 1)
+    kvq.kvq_append_quantize(desc, kc, vc, k_new.cuda(), v_new.cuda(), B, 0, n_tok)
+    torch.cuda.synchronize()
+    lay = kvq.kvq_cache_layout(desc, B, 0)
+    host = kc.cpu().numpy()
+    for h in range(H):
+        codes, scales = rows_of(host, lay, 0, h, H, 0, n_tok)
+        ecodes, escales = oracle_rows("turbo3_qjl", k_new[0, :, h, :].numpy(), desc.turbo_seed, proj.numpy())
+        np.testing.assert_array_equal(codes, ecodes, err_msg=f"codes h{h}")
+        np.testing.assert_array_equal(scales.view(np.uint16), escales.view(np.uint16), err_msg=f"scales h{h}")
