@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_pair_kernel(const Appen
       const int D = pk.D;
       for (int t = threadIdx.x; t < D * D; t += kAppendThreads) {
         const int i = t / D, j = t - i * D;  // coalesced read of P[i][j]
-        pt_smem[j * D + i] = __ldg(pk.tq.proj + t);
+        pt_smem[j * D + i] = __ldg(qjl_proj(pk.tq) + t);
       }
       __syncthreads();
       pt = pt_smem;

@@ -504,7 +504,7 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
       for (int e = 0; e < E; ++e) a[e] = __fadd_rn(a[e], a[e + h]);
     }
     const float eps = __fsqrt_rn(__shfl_sync(0xffffffffu, a[0], 0));
-    gamma = __fmul_rn(__fmul_rn(norm, eps), p.tq.rsqrt_d);
+    gamma = __fmul_rn(__fmul_rn(norm, eps), qjl_rsqrt_d(p.tq));
     float u[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) u[e] = 0.0f;
@@ -537,7 +537,7 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
         }
       }
     }
-    const float* prow = p.tq.proj + (size_t)(lane * E) * D;  // row lane*E of P
+    const float* prow = qjl_proj(p.tq) + (size_t)(lane * E) * D;  // row lane*E of P
 #pragma unroll 4
     for (int jl = 0; jl < (pt == nullptr ? 32 : 0); ++jl) {  // e_j of j = jl*E .. jl*E+E-1, held by lane jl
       float ej[E];

@@ -55,6 +55,10 @@
 //        64-entry table of one row's two consecutive dims, paired across rows
 //        by a byte permute.
 //   turbo3 values accumulate in the rotated domain; kvq_combine rotates back.
+//   Turbo keys score the rotated query H_un (s * q) against level-table A
+//   operands (hi/lo fp16 parts, three MMAs per k-step); turbo3_qjl keys add the
+//   query projected once more by the QJL matrix against their sign bits as +-1
+//   A operands (two more MMAs).  Both are set up once per CTA, below.
 #pragma once
 
 #include <cuda.h>
@@ -610,7 +614,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       constexpr int NH = 8 * NTH;
       for (int it = threadIdx.x; it < D * (NH / 4); it += L::NW * 32) {
         const int i = it % D, h0 = (it / D) * 4;
-        const float4* prow = reinterpret_cast<const float4*>(p.tqk.proj + (size_t)i * D);
+        const float4* prow = reinterpret_cast<const float4*>(qjl_proj(p.tqk) + (size_t)i * D);
         float acc4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
         for (int j4 = 0; j4 < D / 4; ++j4) {

@@ -146,8 +146,11 @@ TurboConsts turbo_consts(const kvq_cache_desc* d, int32_t type) {
   std::memcpy(t.tau, cb.tau, sizeof(t.tau));
   sign_bits(d->turbo_seed, d->head_dim, t.sign_bits);
   if (is_qjl(type)) {
-    t.proj = d->qjl_proj;
-    t.rsqrt_d = (float)(1.0 / std::sqrt((double)d->head_dim));
+    const uint64_t addr = (uint64_t)(uintptr_t)d->qjl_proj;
+    const uint32_t lo = (uint32_t)addr, hi = (uint32_t)(addr >> 32);
+    std::memcpy(&t.tau[kQjlSlot], &lo, 4);
+    std::memcpy(&t.tau[kQjlSlot + 1], &hi, 4);
+    t.tau[kQjlSlot + 2] = (float)(1.0 / std::sqrt((double)d->head_dim));
   }
   return t;
 }

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cstring>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -33,15 +34,24 @@ __host__ __device__ constexpr int turbo_bits(int32_t t) {
 __host__ __device__ constexpr bool is_turbo(int32_t t) { return turbo_bits(t) != 0; }
 __host__ __device__ constexpr bool is_qjl(int32_t t) { return t == KVQ_TURBO3_QJL; }
 
-// A turbo type's codebook (2^b levels, 2^b - 1 thresholds) and sign bits;
-// for turbo3_qjl also the QJL projection and fl(1/sqrt(head_dim)).
+// A turbo type's codebook (2^b levels, 2^b - 1 thresholds) and sign bits.
+// turbo3_qjl uses 4 levels and 3 thresholds; the last three threshold slots
+// carry its QJL projection P ([D][D] fp32, row-major; the address as two
+// 32-bit words, low first) and fl(1/sqrt(D)), so the struct (and with it every
+// kernel's parameter block) keeps one layout for all types.
 struct TurboConsts {
   float levels[16];
   float tau[15];
   uint32_t sign_bits[kMaxHeadDim / 32];  // bit i set -> s_i = -1
-  const float* proj;                     // [D][D] fp32, row-major (turbo3_qjl)
-  float rsqrt_d;
 };
+constexpr int kQjlSlot = 12;  // tau[12], tau[13]: P's address; tau[14]: fl(1/sqrt(D))
+__host__ __device__ inline const float* qjl_proj(const TurboConsts& t) {
+  uint32_t lo, hi;
+  memcpy(&lo, &t.tau[kQjlSlot], 4);
+  memcpy(&hi, &t.tau[kQjlSlot + 1], 4);
+  return reinterpret_cast<const float*>(((uint64_t)hi << 32) | lo);
+}
+__host__ __device__ inline float qjl_rsqrt_d(const TurboConsts& t) { return t.tau[kQjlSlot + 2]; }
 
 struct AppendParams {
   const __half* src;   // [B][n_tok][H][D]
