@@ -369,3 +369,40 @@ def test_qjl_keys_need_their_projection():
     lv, th = kvq.kvq_turbo_codebook("turbo3_qjl")
     lv2, th2 = kvq.kvq_turbo_codebook("turbo2")
     assert list(lv) == list(lv2) and list(th) == list(th2)
+
+
+def test_binding_structs_and_enums_match_the_header(tmp_path):
+    """The ctypes mirrors have the C structs' sizes and field offsets, and the
+    binding's type and status codes are the header's enum values (the header is
+    compiled by gcc as plain C)."""
+    structs = {"kvq_cache_desc": kvq.kvq_cache_desc, "kvq_plane_layout": kvq.kvq_plane_layout,
+               "kvq_paged": kvq.kvq_paged}
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "kvq.h"', 'int main(void) {']
+    for name, cls in structs.items():
+        lines.append(f'  printf("{name} size %zu\\n", sizeof({name}));')
+        for field, _ in cls._fields_:
+            lines.append(f'  printf("{name} {field} %zu\\n", offsetof({name}, {field}));')
+    names = ["KVQ_F16", "KVQ_Q8_0", "KVQ_Q4_0", "KVQ_TURBO3", "KVQ_TURBO2", "KVQ_TURBO4", "KVQ_Q5_0",
+             "KVQ_TURBO3_QJL", "KVQ_OK", "KVQ_ERR_INVALID", "KVQ_ERR_UNSUPPORTED", "KVQ_ERR_WORKSPACE",
+             "KVQ_ERR_CUDA"]
+    for n in names:
+        lines.append(f'  printf("enum {n} %d\\n", (int){n});')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    seen = 0
+    for line in filter(None, out):
+        a, b, c = line.split()
+        if a == "enum":
+            assert getattr(kvq, b) == int(c), b
+        elif b == "size":
+            assert ctypes.sizeof(structs[a]) == int(c), a
+        else:
+            assert getattr(structs[a], b).offset == int(c), (a, b)
+        seen += 1
+    assert seen == len(names) + sum(1 + len(c._fields_) for c in structs.values())
+    assert set(kvq.TYPES.values()) == set(range(8))
