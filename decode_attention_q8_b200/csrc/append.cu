@@ -179,13 +179,10 @@ cudaError_t launch_append(const AppendParams* k, int32_t k_type, const AppendPar
   // turbo3_qjl keys come first (a key type); P transposed in shared memory
   const int D = pp.p[0].D;
   const bool can_stage = is_qjl(pp.type[0]) && D <= kQjlSmemDim;
-  static bool attr_set = false;  // idempotent; a race only repeats the call
-  if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(append_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)(sizeof(float) * kQjlSmemDim * kQjlSmemDim));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  const cudaError_t e =
+      set_smem_limit_once(append_pair_kernel<true>, (int)(sizeof(float) * kQjlSmemDim * kQjlSmemDim), attr_done);
+  if (e != cudaSuccess) return e;
   const int64_t ctas = std::min(need, resident_ctas<true>(can_stage ? sizeof(float) * D * D : 0));
   if (ctas <= 0) return cudaSuccess;
   const int64_t key_rows = (int64_t)pp.p[0].B * pp.p[0].n_tok * pp.p[0].H;

@@ -1629,12 +1629,9 @@ template <int KT, int VT, int NB, int NTH, bool PAGED>
 cudaError_t launch_one(const TcArgs& a, const TcMaps& m, cudaStream_t st) {
   using L = Layout<KT, VT, NB * 32>;
   auto kern = decode_tc_kernel<KT, VT, NB, NTH, PAGED>;
-  static bool attr_set = false;  // idempotent; a race only repeats the call
-  if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  const cudaError_t e = set_smem_limit_once(kern, L::TOTAL, attr_done);
+  if (e != cudaSuccess) return e;
   const dim3 grid(a.p.S, a.p.n_kv, a.p.B);
   kern<<<grid, L::NW * 32, L::TOTAL, st>>>(a, m.kc, m.ks, m.vc, m.vs);
   return cudaGetLastError();

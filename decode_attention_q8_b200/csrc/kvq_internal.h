@@ -1,6 +1,7 @@
 // Internal declarations shared by the libkvq translation units (host + device).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <cuda_fp16.h>
@@ -127,6 +128,21 @@ struct CombineParams {
   int32_t rotated;     // turbo values: apply s * H_un * (.) / D
   TurboConsts tq;
 };
+
+// Raises a kernel's dynamic shared memory limit to `bytes` on the current
+// device, once per device (the attribute belongs to the device's context; the
+// bit set `done` remembers devices 0..63, others are set on every call).
+template <typename Kernel>
+cudaError_t set_smem_limit_once(Kernel kern, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev >= 0 && dev < 64 ? (1ull << dev) : 0ull;
+  if (bit != 0 && (done.load(std::memory_order_relaxed) & bit) != 0) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit != 0) done.fetch_or(bit, std::memory_order_relaxed);
+  return e;
+}
 
 // Host-side helpers (kvq_api.cu).
 int64_t rows_per_plane(int64_t max_ctx);
