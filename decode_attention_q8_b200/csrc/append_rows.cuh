@@ -16,10 +16,11 @@
 // block to 8 consecutive threads holding 4 contiguous elements each (one 8-byte
 // load per thread; the block max is a 3-step xor-shuffle reduction inside the 8
 // lanes).  Loading (load_raw) and quantizing (finish) are separate steps, so a
-// thread can have several loads in flight.  turbo3 gives each row to one warp, D/32 contiguous elements per lane;
-// the Walsh-Hadamard butterflies run in registers for strides below D/32 and
-// as xor-shuffles above.  Threads past the work still take part in the
-// shuffles and then return.
+// thread can have several loads in flight.  The turbo types (and turbo3_qjl)
+// give each row to one warp, D/32 contiguous elements per lane; the
+// Walsh-Hadamard butterflies run in registers for strides below D/32 and as
+// xor-shuffles above.  Threads past the work still take part in the shuffles
+// and then return.
 #pragma once
 
 #include "kvq_internal.h"
