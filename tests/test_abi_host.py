@@ -406,3 +406,15 @@ def test_binding_structs_and_enums_match_the_header(tmp_path):
         seen += 1
     assert seen == len(names) + sum(1 + len(c._fields_) for c in structs.values())
     assert set(kvq.TYPES.values()) == set(range(8))
+
+
+def test_qjl_layout():
+    """turbo3_qjl keys: 3d/8 code bytes (2-bit levels, then 1-bit signs) and two
+    fp16 slots per row (norm, gamma) in the scale plane."""
+    desc = kvq.make_desc(32, 8, 128, "turbo3_qjl", "q8_0", 1000, qjl_proj=FAKE)
+    L = kvq.kvq_cache_layout(desc, 2, 0)
+    assert L.code_bytes == 48 and L.n_scales == 2
+    assert L.scale_offset % 256 == 0 and L.scale_offset >= 2 * 8 * 1008 * 48
+    assert L.total_bytes == L.scale_offset + 2 * 8 * 1008 * 2 * 2
+    P = kvq.kvq_paged_layout(desc, 64, 10, 0)
+    assert P.code_bytes == 48 and P.n_scales == 2 and P.rows_per_plane == 64
