@@ -80,3 +80,57 @@ def test_split_combine_identity(bounds):
     ms, ls, accs = attention.partials(q, k, v, 0.25, bounds)
     full = attention.decode_attention(q[None, None], k[None, None], v[None, None], 0.25)[0, 0]
     np.testing.assert_allclose(attention.combine(ms, ls, accs), full, atol=1e-12)
+
+
+@pytest.mark.parametrize("k_type,v_type", [("q8_0", "q4_0"), ("q4_0", "turbo3"), ("f16", "q5_0"),
+                                           ("turbo3_qjl", "turbo2"), ("turbo4", "q8_0")])
+def test_decode_over_stored_cache_is_dequantize_then_attend(k_type, v_type):
+    """orc_decode_cache (the CPU baseline and the full-size check) equals the
+    dequantizers followed by the plain attention, on any thread count."""
+    from oracle import blocks, qjl, turbo
+    B, n_kv, G, T, D, seed = 2, 2, 3, 70, 64, 99
+    rng = np.random.default_rng(hash((k_type, v_type)) % 2 ** 32)
+    proj = rng.standard_normal((D, D)).astype(np.float32)
+
+    def store(kind, x):
+        if kind == "f16":
+            return x.view(np.uint8).reshape(*x.shape[:-1], 2 * D), np.zeros((*x.shape[:-1], 0), np.float16)
+        if kind == "q8_0":
+            d, q = blocks.quantize_q8_0(x)
+            return q.view(np.uint8), d
+        if kind == "q4_0":
+            d, qs = blocks.quantize_q4_0(x)
+            return qs, d
+        if kind == "q5_0":
+            d, qs, qh = blocks.quantize_q5_0(x)
+            return qs, np.concatenate([d, np.ascontiguousarray(qh).view(np.float16)], axis=-1)
+        if kind == "turbo3_qjl":
+            sc, codes = qjl.quantize(x, seed, proj)
+            return codes, sc
+        n, codes = turbo.quantize(x, seed, turbo.BITS[kind])
+        return codes, n[..., None]
+
+    def dequant(kind, codes, sc):
+        if kind == "f16":
+            return blocks.dequantize_f16(np.ascontiguousarray(codes).view(np.float16))
+        if kind == "q8_0":
+            return blocks.dequantize_q8_0(sc, np.ascontiguousarray(codes).view(np.int8))
+        if kind == "q4_0":
+            return blocks.dequantize_q4_0(sc, codes)
+        if kind == "q5_0":
+            nb = D // 32
+            return blocks.dequantize_q5_0(sc[..., :nb], codes, np.ascontiguousarray(sc[..., nb:]).view(np.uint32))
+        if kind == "turbo3_qjl":
+            return qjl.dequantize(sc, codes, seed, proj, D)
+        return turbo.dequantize(sc[..., 0], codes, seed, D, turbo.BITS[kind])
+
+    k = (rng.standard_normal((B, n_kv, T, D)) * 2).astype(np.float16)
+    v = rng.standard_normal((B, n_kv, T, D)).astype(np.float16)
+    q = rng.standard_normal((B, n_kv * G, D)).astype(np.float16)
+    kc, ks = store(k_type, k)
+    vc, vs = store(v_type, v)
+    expect = attention.decode_attention(q.astype(np.float64), dequant(k_type, kc, ks), dequant(v_type, vc, vs), 0.125)
+    got1 = attention.decode_cache(k_type, v_type, kc, ks, vc, vs, q, 0.125, seed=seed, proj=proj, threads=1)
+    got4 = attention.decode_cache(k_type, v_type, kc, ks, vc, vs, q, 0.125, seed=seed, proj=proj, threads=4)
+    np.testing.assert_allclose(got1, expect, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(got1, got4)

@@ -52,6 +52,42 @@ def test_handworked_blocks():
             np.testing.assert_array_equal(qs[0], blk["bytes"], err_msg=blk["name"])
 
 
+def _multiblock_rows():
+    rows, cur = [], None
+    for line in read_golden("blocks_multiblock_rows.txt"):
+        tok = line.split()
+        if tok[0] == "row":
+            cur = {"name": tok[1], "type": tok[2], "d": int(tok[3])}
+            rows.append(cur)
+        else:
+            cur[tok[0]] = tok[1:]
+    return rows
+
+
+def test_dequantizers_on_handworked_multiblock_rows():
+    """Four blocks with four different scales per row: the value of every
+    element follows by hand (exact products).  A wrong code offset, swapped
+    nibbles, a wrong qh bit or one block's scale used for another block fails."""
+    rows = _multiblock_rows()
+    assert [r["type"] for r in rows] == ["q8_0", "q4_0", "q5_0"]
+    for r in rows:
+        d = r["d"]
+        scales = np.array([int(v, 16) for v in r["scales"]], np.uint16).view(np.float16)[None]
+        expect = np.array([float(v) for v in r["x"]])[None]
+        assert expect.shape == (1, d) and scales.shape == (1, d // 32)
+        if r["type"] == "q8_0":
+            q = np.array([int(v) for v in r["q"]], np.int8)[None]
+            got = blocks.dequantize_q8_0(scales, q)
+        elif r["type"] == "q4_0":
+            qs = np.array([int(v, 16) for v in r["bytes"]], np.uint8)[None]
+            got = blocks.dequantize_q4_0(scales, qs)
+        else:
+            qs = np.array([int(v, 16) for v in r["bytes"]], np.uint8)[None]
+            qh = np.array([int(v, 16) for v in r["qh"]], np.uint32)[None]
+            got = blocks.dequantize_q5_0(scales, qs, qh)
+        np.testing.assert_array_equal(got, expect, err_msg=r["name"])
+
+
 def test_q8_0_rounding_and_bounds():
     rng = np.random.default_rng(1)
     x16 = np.concatenate([_rand_blocks(rng, 4000), _adversarial_blocks(rng)])
@@ -70,12 +106,13 @@ def test_q8_0_rounding_and_bounds():
     grid = np.arange(-127, 128, dtype=np.float64)
     best = np.abs(r[..., None] - grid).min(axis=-1)
     assert np.all(np.abs(r - qq) <= best + 1e-5)
-    # round trip with the stored fp16 scale: |x - d_h q| <= d/2 + 127 |d - d_h|
+    # round trip through the dequantizer (stored fp16 scale): |x - x_hat| <= d/2 + 127 |d - d_h|
     dh = d_h[:, 0].astype(np.float64)[nz]
-    err = np.abs(x[nz] - dh[:, None] * qq)
+    err = np.abs(x[nz] - blocks.dequantize_q8_0(d_h, q)[nz])
     bound = d[nz] / 2 * (1 + 1e-5) + 127 * np.abs(d[nz] - dh)
     assert np.all(err <= bound[:, None] + 1e-12)
     assert np.all(q[~nz] == 0)
+    assert np.all(blocks.dequantize_q8_0(d_h, q)[~nz] == 0)
 
 
 def test_q8_0_exact_ties_round_away():
@@ -107,11 +144,17 @@ def test_q4_0_codes_and_bounds():
     assert np.all(np.abs(r - c)[unclamped] <= 0.5 + 1e-5)
     # clamped elements (opposite sign to m, |x/d| in [7.5, 8]) sit at the top code 7
     assert np.all(c[r > 7.5 + 1e-5] == 7)
+    # round trip through the packed bytes and the dequantizer (stored fp16 scale)
+    d_p, qs = blocks.quantize_q4_0(x16)
+    np.testing.assert_array_equal(d_p.view(np.uint16), d_h.view(np.uint16))
+    x_hat = blocks.dequantize_q4_0(d_p, qs)
     dh = d_h[:, 0].astype(np.float64)[nz]
-    err = np.abs(x[nz] - dh[:, None] * c)
+    np.testing.assert_array_equal(x_hat[nz], dh[:, None] * c)      # value = d_h * (code - 8)
+    err = np.abs(x[nz] - x_hat[nz])
     bound_un = np.abs(d)[:, None] / 2 * (1 + 1e-5) + 16 * np.abs(d - dh)[:, None]
     bound_cl = np.abs(d)[:, None] * (1 + 1e-5) + 16 * np.abs(d - dh)[:, None]
     assert np.all(np.where(unclamped, err <= bound_un + 1e-12, err <= bound_cl + 1e-12))
+    assert np.all(x_hat[~nz] == 0)
 
 
 def test_q4_0_ties_lowest_index():
@@ -155,8 +198,11 @@ def test_q5_0_codes_and_bounds():
     unclamped = r < 15.5 - 1e-5
     assert np.all(np.abs(r - c)[unclamped] <= 0.5 + 1e-5)
     assert np.all(c[r > 15.5 + 1e-5] == 15)
+    d_p, qs, qh = blocks.quantize_q5_0(x16)
+    x_hat = blocks.dequantize_q5_0(d_p, qs, qh)
     dh = d_h[:, 0].astype(np.float64)[nz]
-    err = np.abs(x[nz] - dh[:, None] * c)
+    np.testing.assert_array_equal(x_hat[nz], dh[:, None] * c)      # value = d_h * (code - 16)
+    err = np.abs(x[nz] - x_hat[nz])
     bound_un = np.abs(d)[:, None] / 2 * (1 + 1e-5) + 32 * np.abs(d - dh)[:, None]
     bound_cl = np.abs(d)[:, None] * (1 + 1e-5) + 32 * np.abs(d - dh)[:, None]
     assert np.all(np.where(unclamped, err <= bound_un + 1e-12, err <= bound_cl + 1e-12))

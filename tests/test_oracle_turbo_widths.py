@@ -24,6 +24,11 @@ def _printed():
     return tab
 
 
+def _upper_tail(x):
+    """P(Z > x) for Z ~ N(0,1) (math.erfc, no cancellation)."""
+    return 0.0 if x == np.inf else 0.5 * math.erfc(x / math.sqrt(2.0))
+
+
 def _last_digit(text):
     """One unit in the last printed digit (the 1960 table is good to about that)."""
     dec = len(text.split(".")[1]) if "." in text else 0
@@ -50,7 +55,7 @@ def test_levels_and_thresholds_match_max_1960(n):
     assert np.allclose(lv, -lv[::-1], atol=0) and np.allclose(th, (lv[:-1] + lv[1:]) / 2)
     # distortion 1 - sum c_k^2 P(cell k) (centroid condition), against the printed value
     edges = np.concatenate([[-np.inf], th, [np.inf]])
-    p = [turbo3._upper_tail(a) - turbo3._upper_tail(b) if a != -np.inf else 1 - turbo3._upper_tail(b)
+    p = [_upper_tail(a) - _upper_tail(b) if a != -np.inf else 1 - _upper_tail(b)
          for a, b in zip(edges[:-1], edges[1:])]
     mse = 1.0 - float(np.sum(lv ** 2 * np.array(p)))
     text = tab[(n, "mse")][0]
