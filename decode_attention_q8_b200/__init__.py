@@ -37,7 +37,7 @@ EXPORTED = (
     "kvq_decode_attention", "kvq_combine", "kvq_decode_attention_noalloc", "kvq_decode_step",
     "kvq_decode_attention_varlen", "kvq_decode_step_varlen", "kvq_append_quantize_varlen",
     "kvq_paged_layout", "kvq_paged_cache_bytes", "kvq_append_quantize_paged", "kvq_decode_attention_paged",
-    "kvq_decode_step_paged", "kvq_partials_region", "kvq_combine_ranks",
+    "kvq_decode_step_paged", "kvq_partials_region", "kvq_combine_ranks", "kvq_workspace_status_offset",
 )
 
 
@@ -48,7 +48,7 @@ class kvq_cache_desc(ctypes.Structure):
         ("head_dim", ctypes.c_int32),
         ("k_type", ctypes.c_int32),
         ("v_type", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("flags", ctypes.c_int32),
         ("max_ctx", ctypes.c_int64),
         ("turbo_seed", ctypes.c_uint64),
         ("qjl_proj", ctypes.c_void_p),
@@ -116,6 +116,7 @@ _sigs = {
     "kvq_partials_region": (ctypes.c_int, [_D, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t),
                                            ctypes.POINTER(ctypes.c_size_t)]),
     "kvq_combine_ranks": (ctypes.c_int, [_D, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P]),
+    "kvq_workspace_status_offset": (ctypes.c_int, [_D, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -159,10 +160,14 @@ def _type(t):
     return TYPES[t] if isinstance(t, str) else int(t)
 
 
-def make_desc(n_q_heads, n_kv_heads, head_dim, k_type, v_type, max_ctx, turbo_seed=0, qjl_proj=None):
+KVQ_FLAG_OVERLAP_PREVIOUS = 1
+
+
+def make_desc(n_q_heads, n_kv_heads, head_dim, k_type, v_type, max_ctx, turbo_seed=0, qjl_proj=None, flags=0):
     """A kvq_cache_desc.  qjl_proj: the turbo3_qjl projection (device fp32
-    [head_dim][head_dim]); the descriptor keeps a reference to it."""
-    d = kvq_cache_desc(n_q_heads, n_kv_heads, head_dim, _type(k_type), _type(v_type), 0,
+    [head_dim][head_dim]); the descriptor keeps a reference to it.  flags:
+    KVQ_FLAG_* bits (see include/kvq.h)."""
+    d = kvq_cache_desc(n_q_heads, n_kv_heads, head_dim, _type(k_type), _type(v_type), flags,
                        max_ctx, turbo_seed, _ptr(qjl_proj))
     d.qjl_tensor = qjl_proj
     return d
@@ -198,6 +203,18 @@ def kvq_auto_splits(desc, batch, ctx_len):
 
 def kvq_workspace_bytes(desc, batch, n_splits=0):
     return _lib.kvq_workspace_bytes(ctypes.byref(desc), batch, n_splits)
+
+
+def kvq_workspace_status_offset(desc, batch):
+    """Byte offset of the workspace's status word (bits: 1 a tile wait gave up,
+    2 a combine wait gave up, 4 a block-table entry outside the pool)."""
+    off = ctypes.c_size_t()
+    _check(_lib.kvq_workspace_status_offset(ctypes.byref(desc), batch, ctypes.byref(off)),
+           "kvq_workspace_status_offset")
+    return off.value
+
+
+STATUS_TILE_WAIT, STATUS_COMBINE_WAIT, STATUS_BAD_PAGE = 1, 2, 4
 
 
 def kvq_turbo3_codebook():

@@ -72,6 +72,10 @@ constexpr int kNWMax = 8;    // warps per CTA (4 for the widest f16 stages)
 constexpr int kSub = 32;     // cache rows per warp tile (one TMA box per plane)
 constexpr int kHalf = 16;    // rows per MMA row block (two per tile)
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+// Bits of the workspace status word (kvq_workspace_status_offset), set when a
+// wait gives up or a block-table entry is outside the pool; the affected
+// outputs are NaN.
+constexpr uint32_t kStatusTileWait = 1u, kStatusCombineWait = 2u, kStatusBadPage = 4u;
 
 __host__ __device__ constexpr int code_bytes(int t, int d) {
   return t == KVQ_F16 ? 2 * d
@@ -397,31 +401,36 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   // split).  Raw words here; their fragment form is built further down.
   //   q8_0 / q4_0: 16-byte segments 2*blk, 2*blk+1, lane c's bytes 4c..4c+3
   //   f16: dims 32*blk + 8*i + 2c, +1 for i = 0..3
+  // A launch that overlaps the previous kernel (p.pdl) reads them only after
+  // that kernel has completed, which may have written them.
   uint32_t qraw[NTH][NB][4];
+  auto load_queries = [&]() {
 #pragma unroll
-  for (int nt = 0; nt < NTH; ++nt) {
-    const int head = nt * 8 + g;
-    const bool hv = head < p.G;
-    const __half* qrow = p.q + ((int64_t)b * p.n_q + (int64_t)kvh * p.G + (hv ? head : 0)) * D;
+    for (int nt = 0; nt < NTH; ++nt) {
+      const int head = nt * 8 + g;
+      const bool hv = head < p.G;
+      const __half* qrow = p.q + ((int64_t)b * p.n_q + (int64_t)kvh * p.G + (hv ? head : 0)) * D;
 #pragma unroll
-    for (int blk = 0; blk < NB; ++blk) {
-      uint32_t* w = qraw[nt][blk];
-      w[0] = w[1] = w[2] = w[3] = 0u;
-      if (hv) {
-        if (KT == KVQ_F16) {
+      for (int blk = 0; blk < NB; ++blk) {
+        uint32_t* w = qraw[nt][blk];
+        w[0] = w[1] = w[2] = w[3] = 0u;
+        if (hv) {
+          if (KT == KVQ_F16) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) w[i] = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 8 * i + 2 * c);
-        } else {
-          const uint2 s0 = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 4 * c);
-          const uint2 s1 = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 16 + 4 * c);
-          w[0] = s0.x;
-          w[1] = s0.y;
-          w[2] = s1.x;
-          w[3] = s1.y;
+            for (int i = 0; i < 4; ++i) w[i] = *reinterpret_cast<const uint32_t*>(qrow + blk * 32 + 8 * i + 2 * c);
+          } else {
+            const uint2 s0 = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 4 * c);
+            const uint2 s1 = *reinterpret_cast<const uint2*>(qrow + blk * 32 + 16 + 4 * c);
+            w[0] = s0.x;
+            w[1] = s0.y;
+            w[2] = s1.x;
+            w[3] = s1.y;
+          }
         }
       }
     }
-  }
+  };
+  if (!p.pdl) load_queries();
 
   // Paged pool: the page of each of this warp's tiles, a window of 32 tiles
   // per register (lane i: tile j0 + i), read with the queries, before any tile
@@ -482,6 +491,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   auto page_ok = [&](int pg) -> int {
     if (pg < 0 || pg >= p.n_pages) {
       atomicExch(&cta_failed, 1);
+      atomicOr(p.status, kStatusBadPage);
       return 0;
     }
     return pg;
@@ -543,6 +553,16 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   for (int j = 0; j < S; ++j) {
     const int pg = paged ? __shfl_sync(0xffffffffu, pg_win, j) : 0;
     if (lane == 0 && j < my_tiles && !(warp == wt && j == jt)) issue(j, j, pg);
+  }
+  // The kernel after this one on the stream may be scheduled from here on (a
+  // no-op unless it was launched to overlap this one).  A launch that overlaps
+  // the previous kernel has requested cache tiles only, which that kernel does
+  // not write; everything else waits until that kernel has completed and its
+  // writes are visible.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (p.pdl) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    load_queries();
   }
   if (warp == wt) {
     constexpr int rk = rows::row_threads(KT, D), rv = rows::row_threads(VT, D);
@@ -1297,7 +1317,10 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     // CTA's partials NaN so the outputs show the failure.
     const int last = min(my_tiles, failed_at + S);
     for (int jj = failed_at; jj < last; ++jj) (void)mbar_wait(&bars[jj % S], (uint32_t)((jj / S) & 1));
-    if (lane == 0) atomicExch(&cta_failed, 1);
+    if (lane == 0) {
+      atomicExch(&cta_failed, 1);
+      atomicOr(p.status, kStatusTileWait);
+    }
   }
   __syncwarp();
 
@@ -1450,6 +1473,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         while (*reinterpret_cast<volatile unsigned int*>(p.epochs + plane) == e0) {
           if (global_ns() - w0 > kWaitLimitNs) {
             failed = 1;
+            atomicOr(p.status, kStatusCombineWait);
             break;
           }
           __nanosleep(64);
@@ -1527,7 +1551,10 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           // a copy did not land within the limit: let it drain (bounded
           // again) so nothing writes shared memory after the CTA exits; the
           // heads' outputs read NaN
-          if (threadIdx.x == 0) (void)mbar_wait(cbar, cphase);
+          if (threadIdx.x == 0) {
+            (void)mbar_wait(cbar, cphase);
+            atomicOr(p.status, kStatusCombineWait);
+          }
           __syncthreads();
           comb_failed = 1;
           break;
@@ -1633,8 +1660,23 @@ cudaError_t launch_one(const TcArgs& a, const TcMaps& m, cudaStream_t st) {
   const cudaError_t e = set_smem_limit_once(kern, L::TOTAL, attr_done);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.p.S, a.p.n_kv, a.p.B);
-  kern<<<grid, L::NW * 32, L::TOTAL, st>>>(a, m.kc, m.ks, m.vc, m.vs);
-  return cudaGetLastError();
+  if (!a.p.pdl) {
+    kern<<<grid, L::NW * 32, L::TOTAL, st>>>(a, m.kc, m.ks, m.vc, m.vs);
+    return cudaGetLastError();
+  }
+  // programmatic dependent launch: may start once the previous kernel on the
+  // stream has triggered (griddepcontrol.launch_dependents) or finished
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(L::NW * 32);
+  cfg.dynamicSmemBytes = L::TOTAL;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, m.kc, m.ks, m.vc, m.vs);
 }
 
 template <int KT, int VT, int NB, bool PAGED>

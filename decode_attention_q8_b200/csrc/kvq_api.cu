@@ -232,17 +232,18 @@ int32_t resolve_splits(const kvq_cache_desc* d, int32_t batch, int64_t ctx, int3
 }
 
 struct WsLayout {
-  int64_t m_off, l_off, acc_off, cnt_off, total;
+  int64_t m_off, l_off, acc_off, cnt_off, status_off, total;
 };
 
-// Counters first (arrival counters, then epoch words, one of each per group):
-// their place depends on batch and n_kv only, so calls with different split
-// counts on one workspace keep them intact.
+// Counters first (arrival counters, then epoch words, one of each per group,
+// then the status word): their place depends on batch and n_kv only, so calls
+// with different split counts on one workspace keep them intact.
 WsLayout ws_layout(const kvq_cache_desc* d, int32_t batch, int32_t S) {
   WsLayout w;
   const int64_t rows = (int64_t)batch * d->n_q_heads * S;
   w.cnt_off = 0;
-  w.m_off = round_up((int64_t)batch * d->n_kv_heads * 8, 256);
+  w.status_off = (int64_t)batch * d->n_kv_heads * 8;
+  w.m_off = round_up(w.status_off + 4, 256);
   w.l_off = w.m_off + round_up(rows * 4, 256);
   w.acc_off = w.l_off + round_up(rows * 4, 256);
   w.total = w.acc_off + rows * d->head_dim * 4;
@@ -353,6 +354,7 @@ kvq_status fill_decode(const kvq_cache_desc* d, const void* k_cache, const void*
   p.ws_m = reinterpret_cast<float*>(ws + w.m_off);
   p.ws_l = reinterpret_cast<float*>(ws + w.l_off);
   p.ws_acc = reinterpret_cast<float*>(ws + w.acc_off);
+  p.status = reinterpret_cast<uint32_t*>(ws + w.status_off);
   p.B = batch;
   p.n_q = d->n_q_heads;
   p.n_kv = d->n_kv_heads;
@@ -465,6 +467,9 @@ kvq_status step_impl(const kvq_cache_desc* d, void* k_cache, void* v_cache, cons
     if (is_turbo(type)) a.tq = turbo_consts(d, type);
   }
   p.out = out;
+  // overlap with the previous kernel only where nothing the step reads before
+  // the grid dependency resolves can come from it (no device lengths, no table)
+  p.pdl = (d->flags & KVQ_FLAG_OVERLAP_PREVIOUS) && ctx_lens == nullptr && pg == nullptr ? 1 : 0;
   p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + w.cnt_off);
   p.epochs = p.counters + (int64_t)batch * d->n_kv_heads;
   p.comb_ctas = combining_ctas(d, batch, p.S);
@@ -505,7 +510,7 @@ size_t kvq_row_bytes(int32_t type, int32_t head_dim) {
 kvq_status kvq_check_desc(const kvq_cache_desc* d) {
   if (!d) return KVQ_ERR_INVALID;
   if (d->n_q_heads < 1 || d->n_kv_heads < 1 || d->n_q_heads % d->n_kv_heads) return KVQ_ERR_INVALID;
-  if (d->head_dim < 1 || d->reserved != 0) return KVQ_ERR_INVALID;
+  if (d->head_dim < 1 || (d->flags & ~KVQ_FLAG_OVERLAP_PREVIOUS) != 0) return KVQ_ERR_INVALID;
   if (d->max_ctx < 1 || d->max_ctx > kMaxCtx) return KVQ_ERR_INVALID;
   if (!known_type(d->k_type) || !known_type(d->v_type)) return KVQ_ERR_INVALID;
   if (d->head_dim % kBlock || d->head_dim > kMaxHeadDim) return KVQ_ERR_UNSUPPORTED;
@@ -586,6 +591,14 @@ size_t kvq_workspace_bytes(const kvq_cache_desc* d, int32_t batch, int32_t n_spl
   if (kvq_check_desc(d) != KVQ_OK || batch < 1 || batch > 65535 || n_splits < 0 || n_splits > kMaxSplits) return 0;
   const int32_t S = n_splits > 0 ? n_splits : auto_splits_bound(d, batch, d->max_ctx);
   return (size_t)ws_layout(d, batch, S).total;
+}
+
+kvq_status kvq_workspace_status_offset(const kvq_cache_desc* d, int32_t batch, size_t* offset) {
+  const kvq_status st = kvq_check_desc(d);
+  if (st != KVQ_OK) return st;
+  if (batch < 1 || batch > 65535 || offset == nullptr) return KVQ_ERR_INVALID;
+  *offset = (size_t)ws_layout(d, batch, 1).status_off;
+  return KVQ_OK;
 }
 
 kvq_status kvq_turbo3_codebook(float levels[8], float thresholds[7]) {

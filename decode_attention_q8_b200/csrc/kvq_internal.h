@@ -111,7 +111,9 @@ struct DecodeParams {
   float* out;            // [B][n_q][D] combined output, or null (partials only)
   uint32_t* counters;    // [B][n_kv] split arrival counters, zero between calls
   uint32_t* epochs;      // [B][n_kv] bumped by each group's last arrival (any start value)
+  uint32_t* status;      // workspace status word; bits set by a wait that gave up (kvq.h)
   int32_t comb_ctas;     // CTAs per group that combine (the last arrivals), 1 .. G
+  int32_t pdl;           // 1: launched to overlap the previous kernel (KVQ_FLAG_OVERLAP_PREVIOUS)
 };
 
 struct CombineParams {

@@ -8,8 +8,10 @@
 // the split partials go to a fixed-size array in device memory that this
 // file declares at file scope.
 //
-// The array (kStaticScratchBytes) lives in every GPU's memory from the moment
-// the library is first used on that GPU until the process exits.  All calls on
+// The array (kStaticScratchBytes) is reserved in a GPU's memory when the CUDA
+// runtime loads this library's module on that GPU -- at context creation under
+// eager module loading (CUDA_MODULE_LOADING=EAGER), at the first use of the
+// module under lazy loading -- and stays until the process exits.  All calls on
 // one GPU share it and it keeps the previous call's contents; every entry the
 // decode kernel reads back is written first in the same call, so nothing needs
 // clearing.  Two calls whose kernels overlap on the GPU (different streams,
@@ -18,7 +20,10 @@
 // In host code the array's name is only a host-side stand-in, not a device
 // address; the device address is looked up with cudaGetSymbolAddress once per
 // GPU, with that GPU current, on the first call made there.  That first call
-// should therefore come before any stream capture.
+// should therefore come before any stream capture.  The address is kept for the
+// life of the process: after cudaDeviceReset (or anything else that destroys
+// the device's primary context) it is stale, and this entry point must not be
+// used again in that process.
 #include <mutex>
 
 #include "kvq_internal.h"
@@ -69,8 +74,10 @@ extern "C" kvq_status kvq_decode_attention_noalloc(const kvq_cache_desc* desc, c
   if (n_splits < 0 || n_splits > kvq::kMaxSplits) return KVQ_ERR_INVALID;
   int32_t S = n_splits;
   if (S == 0) {
+    // automatic count, lowered to the largest count whose partials fit the scratch
     S = kvq_auto_splits(desc, batch, ctx_len);
     if (S == 0) return KVQ_ERR_INVALID;
+    while (S > 1 && kvq_workspace_bytes(desc, batch, S) > kvq::kStaticScratchBytes) --S;
   }
   const size_t need = kvq_workspace_bytes(desc, batch, S);
   if (need == 0) return KVQ_ERR_INVALID;

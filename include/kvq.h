@@ -149,6 +149,19 @@ typedef enum {
   KVQ_ERR_CUDA = 4          /* the CUDA runtime refused a launch or a query */
 } kvq_status;
 
+/* kvq_cache_desc.flags.
+ * KVQ_FLAG_OVERLAP_PREVIOUS: kvq_decode_step (uniform ctx_len, contiguous
+ *   cache) is launched so that it may start while the kernel before it on the
+ *   stream is still finishing (programmatic dependent launch).  Until that
+ *   kernel has completed, the step only reads cache rows 0 .. ctx_len-2 of this
+ *   layer (it requests its first tiles); q, k_new, v_new, the workspace and out
+ *   are touched only after it.  The caller promises that the kernel right
+ *   before the step on the stream does not write those cache rows -- true when
+ *   it is another layer's step, a projection producing q, k_new and v_new, or
+ *   anything but an append into this same cache.  In a CUDA graph the same
+ *   holds for the node before it.  Other entry points ignore the flag. */
+#define KVQ_FLAG_OVERLAP_PREVIOUS 1
+
 /* One layer's cache description (K and V of one layer share it). */
 typedef struct {
   int32_t n_q_heads;   /* query heads, a multiple of n_kv_heads */
@@ -156,7 +169,7 @@ typedef struct {
   int32_t head_dim;    /* multiple of 32, at most 256 */
   int32_t k_type;      /* kvq_type of the key cache: any */
   int32_t v_type;      /* kvq_type of the value cache: any but TURBO3_QJL */
-  int32_t reserved;    /* must be 0 */
+  int32_t flags;       /* KVQ_FLAG_* bits; 0 for none */
   int64_t max_ctx;     /* rows the cache holds per (batch, KV head), >= 1 */
   uint64_t turbo_seed; /* seed of the turbo sign vector (K and V turbo types) */
   /* TURBO3_QJL keys: the QJL projection P, device memory owned by the caller,
@@ -213,10 +226,24 @@ KVQ_API int32_t kvq_auto_splits(const kvq_cache_desc* desc, int32_t batch, int64
 /* Workspace bytes kvq_decode_attention / kvq_combine / kvq_decode_step need
  * for n_splits (0 = automatic, resolved as kvq_auto_splits would for ctx_len =
  * max_ctx); 0 on error.  Layout: uint32 arrival counters [batch][n_kv_heads]
- * and uint32 epoch words [batch][n_kv_heads] (used by kvq_decode_step only;
- * their place does not depend on n_splits), then m and l fp32 [batch][n_q][S]
+ * and uint32 epoch words [batch][n_kv_heads] (used by kvq_decode_step only),
+ * then one uint32 status word (see kvq_workspace_status_offset) -- the place
+ * of these does not depend on n_splits -- then m and l fp32 [batch][n_q][S]
  * each, then acc fp32 [batch][n_q][S][head_dim], each part 256-byte aligned. */
 KVQ_API size_t kvq_workspace_bytes(const kvq_cache_desc* desc, int32_t batch, int32_t n_splits);
+
+/* Byte offset of the workspace's status word for `batch` (the same for every
+ * split count).  The decode kernels OR bits into it when something made them
+ * write NaN instead of a result, and never clear it:
+ *   bit 0  a wait for a cache tile's copy gave up (bounded at about 2 s);
+ *   bit 1  kvq_decode_step: a wait in the in-kernel combine gave up (another
+ *          CTA's arrival or copy never came, e.g. a workspace whose arrival
+ *          counters were not zero);
+ *   bit 2  paged decode: a block-table entry outside [0, n_pages).
+ * The affected outputs are NaN.  To check a call, zero the word before it and
+ * read it back (a 4-byte device-to-host copy on the same stream) after it; the
+ * library itself neither reads nor clears it.  Host only. */
+KVQ_API kvq_status kvq_workspace_status_offset(const kvq_cache_desc* desc, int32_t batch, size_t* offset);
 
 /* The turbo3 codebook this library uses: 8 binary32 levels (ascending) and
  * the 7 binary32 thresholds between them.  Host only; no device needed. */
@@ -306,12 +333,19 @@ KVQ_API kvq_status kvq_combine_ranks(const kvq_cache_desc* desc, const void* par
  * allocator during another stream's graph capture, a foreign-language host that
  * only passes pointers it was given).
  *   Scratch: one 8 MiB array in each GPU's memory (a file-scope __device__
- *   variable), held from the library's first use on that GPU until the process
- *   exits.  Problems whose workspace (kvq_workspace_bytes for the split count
- *   used) exceeds 8 MiB return KVQ_ERR_WORKSPACE without launching anything.
+ *   variable), reserved when the CUDA runtime loads the library's module on
+ *   that GPU -- at context creation under eager module loading
+ *   (CUDA_MODULE_LOADING=EAGER), at the module's first use under lazy loading
+ *   -- and held until the process exits.  Problems whose workspace
+ *   (kvq_workspace_bytes for the split count used) exceeds 8 MiB return
+ *   KVQ_ERR_WORKSPACE without launching anything when n_splits is given; with
+ *   n_splits = 0 the automatic count is lowered to the largest count whose
+ *   partials fit (KVQ_ERR_WORKSPACE only if even one split does not fit).
  *   Set-up: the first call on a GPU looks up the array's device address there
  *   (cudaGetSymbolAddress, with that GPU current); make that first call before
- *   any stream capture.
+ *   any stream capture.  The address is kept for the life of the process, so
+ *   this entry point must not be used after cudaDeviceReset (or anything else
+ *   that destroys the device's primary context) in the same process.
  *   Sharing: every call on a GPU uses the same array, which keeps the previous
  *   call's contents (each call writes every entry before reading it back).
  *   Calls that overlap on the GPU (unordered streams) race and give wrong

@@ -137,8 +137,10 @@ def test_check_desc():
     for kt in ("turbo2", "turbo3", "turbo4", "turbo3_qjl"):
         assert kvq.kvq_check_desc(kvq.make_desc(64, 8, 128, kt, "q4_0", 16)) == kvq.KVQ_OK
     d = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 16)
-    d.reserved = 1
+    d.flags = 2                                        # an undefined flag bit
     assert kvq.kvq_check_desc(d) == kvq.KVQ_ERR_INVALID
+    d.flags = kvq.KVQ_FLAG_OVERLAP_PREVIOUS
+    assert kvq.kvq_check_desc(d) == kvq.KVQ_OK
     assert kvq.raw_status("kvq_check_desc", None) == kvq.KVQ_ERR_INVALID
 
 
@@ -303,13 +305,13 @@ def test_paged_entry_points_reject_before_launch():
 
 
 def test_partials_region_is_the_workspace_tail():
-    """The partials (m, l, acc) follow the counters and epoch words and run to
-    the end of the workspace."""
+    """The partials (m, l, acc) follow the counters, the epoch words and the
+    status word, and run to the end of the workspace."""
     d = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 32768)
     r256 = lambda v: (v + 255) // 256 * 256
-    for B, S in ((1, 37), (4, 9), (16, 3)):
+    for B, S in ((1, 37), (4, 9), (16, 3), (32, 5)):
         off, n = kvq.kvq_partials_region(d, B, S)
-        assert off == r256(B * 8 * 8)
+        assert off == r256(B * 8 * 8 + 4)
         assert off + n == kvq.kvq_workspace_bytes(d, B, S)
     for bad in ((0, 4), (1, 0), (1, 5000)):
         with pytest.raises(kvq.KvqError):
@@ -328,9 +330,9 @@ def test_workspace_bytes_formula():
     B, S = 4, 9
     rows = B * 64 * S
     r256 = lambda v: (v + 255) // 256 * 256
-    # the fused step's arrival counters and epoch words, [B][n_kv] uint32 each, then m, l, acc,
-    # each part 256-aligned
-    assert kvq.kvq_workspace_bytes(d, B, S) == r256(B * 8 * 8) + 2 * r256(rows * 4) + rows * 128 * 4
+    # the fused step's arrival counters and epoch words, [B][n_kv] uint32 each, the status
+    # word, then m, l, acc, each part 256-aligned
+    assert kvq.kvq_workspace_bytes(d, B, S) == r256(B * 8 * 8 + 4) + 2 * r256(rows * 4) + rows * 128 * 4
     assert kvq.kvq_workspace_bytes(d, 0, S) == 0
     # the automatic split count never needs more workspace than n_splits = 0 reserves
     auto_ws = kvq.kvq_workspace_bytes(d, B, 0)
@@ -418,3 +420,19 @@ def test_qjl_layout():
     assert L.total_bytes == L.scale_offset + 2 * 8 * 1008 * 2 * 2
     P = kvq.kvq_paged_layout(desc, 64, 10, 0)
     assert P.code_bytes == 48 and P.n_scales == 2 and P.rows_per_plane == 64
+
+
+def test_workspace_status_word_place():
+    """The status word follows the arrival counters and epoch words
+    (8 bytes per (batch row, KV head)), does not move with the split count, and
+    the split partials start after it."""
+    desc = kvq.make_desc(64, 8, 128, "q8_0", "q4_0", 32768)
+    for batch in (1, 4, 4096):
+        off = kvq.kvq_workspace_status_offset(desc, batch)
+        assert off == batch * 8 * 8
+        for S in (1, 9, 300):
+            p_off, p_bytes = kvq.kvq_partials_region(desc, batch, S)
+            assert p_off >= off + 4 and p_off % 256 == 0
+            assert kvq.kvq_workspace_bytes(desc, batch, S) == p_off + p_bytes
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_workspace_status_offset(desc, 0)

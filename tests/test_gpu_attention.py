@@ -239,3 +239,43 @@ def test_full_size_sampled(name):
                 np.testing.assert_array_equal(scales.view(np.uint16), es.view(np.uint16))
     del kc, vc, k, v
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["llama70b_ctx32k_b4", "turbo3_ctx32k"])
+def test_full_size_layer_every_byte_and_output(name):
+    """One full-size layer in the benchmark's launch configuration: rows
+    0 .. ctx-2 by the bulk append, the last row by the fused decode step
+    (automatic splits).  Every stored byte of both caches (70B: 1 M rows per
+    tensor) equals the oracle's quantization of the same fp16 rows, and every
+    output equals the oracle's decode over the oracle's own cache."""
+    from oracle import attention
+    w = synth.WORKLOADS[name]
+    B, ctx, D, n_kv = w.batch, w.ctx, w.head_dim, w.n_kv
+    desc = kvq.make_desc(w.n_q, n_kv, D, w.k_type, w.v_type, ctx, turbo_seed=w.turbo_seed)
+    q, k, v = synth.layer_inputs(w, layer=0, device="cuda")
+    kc, vc = alloc_cache(desc, B, 0), alloc_cache(desc, B, 1)
+    kvq.kvq_append_quantize(desc, kc, vc, k, v, B, 0, ctx - 1)
+    ws = torch.zeros(kvq.kvq_workspace_bytes(desc, B, 0), dtype=torch.uint8, device="cuda")
+    out = torch.empty((B, w.n_q, D), dtype=torch.float32, device="cuda")
+    kvq.kvq_decode_step(desc, kc, vc, q, k[:, ctx - 1].contiguous(), v[:, ctx - 1].contiguous(), B, ctx, w.scale,
+                        0, ws, out)
+    torch.cuda.synchronize()
+    stored = {}
+    for which, cache, x, kind in ((0, kc, k, w.k_type), (1, vc, v, w.v_type)):
+        lay = kvq.kvq_cache_layout(desc, B, which)
+        host = cache.cpu().numpy()
+        T, cb, ns = lay.rows_per_plane, lay.code_bytes, lay.n_scales
+        rows = x.cpu().numpy().transpose(0, 2, 1, 3).reshape(-1, D)           # [B * n_kv * ctx, D]
+        ec, es = oracle_rows(kind, rows, w.turbo_seed)
+        got_c = host[:B * n_kv * T * cb].reshape(B * n_kv, T, cb)[:, :ctx]
+        got_s = host[lay.scale_offset:lay.scale_offset + B * n_kv * T * ns * 2].view(np.float16)
+        got_s = got_s.reshape(B * n_kv, T, ns)[:, :ctx]
+        np.testing.assert_array_equal(got_c, ec.reshape(B * n_kv, ctx, cb), err_msg=f"{name} codes {which}")
+        np.testing.assert_array_equal(got_s.view(np.uint16), es.reshape(B * n_kv, ctx, ns).view(np.uint16),
+                                      err_msg=f"{name} scales {which}")
+        stored[which] = (ec.reshape(B, n_kv, ctx, cb), es.reshape(B, n_kv, ctx, ns))
+    del kc, vc, k, v
+    expect = attention.decode_cache(w.k_type, w.v_type, *stored[0], *stored[1], q.cpu().numpy(), w.scale,
+                                    seed=w.turbo_seed, threads=0)
+    assert_attention_close(out.cpu().numpy(), expect, f"{name} every output")
+    torch.cuda.empty_cache()

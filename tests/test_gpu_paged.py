@@ -207,6 +207,9 @@ def test_page_ids_outside_the_pool():
     kvq.kvq_combine(desc, ws, B, rows, 0, out)
     o = out.cpu().numpy()
     assert np.isnan(o[1]).all() and np.isnan(o[2]).all()
+    # the workspace's status word names the cause (it started at zero)
+    off = kvq.kvq_workspace_status_offset(desc, B)
+    assert int(ws[off:off + 4].view(torch.int32).item()) == kvq.STATUS_BAD_PAGE
     G = n_q // n_kv
     for g in range(n_kv):
         kh = oracle_dequant("q8_0", *oracle_rows("q8_0", k[0, :, g].cpu().numpy()), D)

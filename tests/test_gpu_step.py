@@ -255,8 +255,9 @@ def test_missing_arrival_times_out_to_nan():
     outside [0, S) (the contract asks for 0), so no CTA of that group becomes
     its last arrival.  The CTAs that would share its combine wait for an epoch
     bump that never comes; each wait gives up after its bound (about 2 s) and
-    writes NaN for its heads.  The other groups are unaffected, and the GPU
-    context stays usable: the next call on a zeroed workspace is correct."""
+    writes NaN for its heads and sets the combine-wait bit of the workspace's
+    status word.  The other groups are unaffected, and the GPU context stays
+    usable: the next call on a zeroed workspace is correct, with status 0."""
     import time
     B, n_q, n_kv, D, ctx, S = 1, 64, 8, 128, 16384, 40   # 8 heads x 40 splits: several CTAs combine
     desc, q, k, v = _inputs("q8_0", "q4_0", B, n_q, n_kv, D, ctx, seed=17)
@@ -281,6 +282,10 @@ def test_missing_arrival_times_out_to_nan():
     assert nan_heads and sorted(nan_heads + untouched) == list(range(G)), (nan_heads, untouched)
     assert waited > 1.0, waited
     assert torch.equal(out[:, G:], good[:, G:])       # the other groups
+    off = kvq.kvq_workspace_status_offset(desc, B)
+    assert int(ws[off:off + 4].view(torch.int32).item()) == kvq.STATUS_COMBINE_WAIT
     # the context is usable: a fresh workspace gives the right output again
-    again = _step(desc, kc, vc, q, k, v, B, ctx, scale, S, _workspace(desc, B, S))
+    ws2 = _workspace(desc, B, S)
+    again = _step(desc, kc, vc, q, k, v, B, ctx, scale, S, ws2)
     assert torch.equal(again, good)
+    assert int(ws2[off:off + 4].view(torch.int32).item()) == 0
