@@ -254,7 +254,7 @@ def test_full_size_layer_every_byte_and_output(name):
     desc = kvq.make_desc(w.n_q, n_kv, D, w.k_type, w.v_type, ctx, turbo_seed=w.turbo_seed)
     q, k, v = synth.layer_inputs(w, layer=0, device="cuda")
     kc, vc = alloc_cache(desc, B, 0), alloc_cache(desc, B, 1)
-    kvq.kvq_append_quantize(desc, kc, vc, k, v, B, 0, ctx - 1)
+    kvq.kvq_append_quantize(desc, kc, vc, k[:, :ctx - 1].contiguous(), v[:, :ctx - 1].contiguous(), B, 0, ctx - 1)
     ws = torch.zeros(kvq.kvq_workspace_bytes(desc, B, 0), dtype=torch.uint8, device="cuda")
     out = torch.empty((B, w.n_q, D), dtype=torch.float32, device="cuda")
     kvq.kvq_decode_step(desc, kc, vc, q, k[:, ctx - 1].contiguous(), v[:, ctx - 1].contiguous(), B, ctx, w.scale,

@@ -39,7 +39,8 @@ class Chain:
         for layer in range(L):
             q, k, v = synth.layer_inputs(w, layer=layer, device="cuda")
             kc, vc = alloc_cache(self.descs[0], B, 0), alloc_cache(self.descs[0], B, 1)
-            kvq.kvq_append_quantize(self.descs[0], kc, vc, k, v, B, 0, ctx - 1)
+            kvq.kvq_append_quantize(self.descs[0], kc, vc, k[:, :ctx - 1].contiguous(), v[:, :ctx - 1].contiguous(),
+                                    B, 0, ctx - 1)
             self.q.append(q)
             self.k.append(k)
             self.v.append(v)
