@@ -372,6 +372,8 @@ EXTRA_WORKLOADS = (
     ("k4v4_ctx128k_b4", "k4v4_ctx128k_b4", None, 0),
     ("k4v4_ctx128k_b16", "k4v4_ctx128k_b16", None, 0),
     ("turbo3_ctx32k", "turbo3_ctx32k", None, 0),
+    ("turbo3_ctx32k_b4", "turbo3_ctx32k_b4", None, 0),
+    ("qjl_ctx32k_b4", "qjl_ctx32k_b4", None, 0),
 )
 
 
@@ -393,8 +395,10 @@ class StepRun:
         # append of another layer's cache), which writes nothing this one reads
         # before the dependency resolves
         flags = kvq.KVQ_FLAG_OVERLAP_PREVIOUS if overlap else 0
+        # turbo3_qjl keys: the seeded projection, on the device for the library
+        self.proj = synth.qjl_projection(w.seed, w.head_dim).to(dev) if w.k_type == "turbo3_qjl" else None
         self.desc = kvq.make_desc(w.n_q, w.n_kv, w.head_dim, w.k_type, w.v_type, w.ctx, turbo_seed=w.turbo_seed,
-                                  flags=flags)
+                                  qjl_proj=self.proj, flags=flags)
         B, ctx = w.batch, w.ctx
         stream = torch.cuda.current_stream(dev)  # prefill and the timed steps run on it
         self.kcs, self.vcs, self.qs, self.kn, self.vn = [], [], [], [], []

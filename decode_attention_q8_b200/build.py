@@ -69,10 +69,12 @@ def build(force=False, verbose=False):
     if failed:
         raise RuntimeError("\n".join(failed))
     if force or _stale(LIB, objs):
-        cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-Xcompiler", "-fPIC", "-o", LIB, *objs]
+        tmp = LIB + f".tmp{os.getpid()}"
+        cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-Xcompiler", "-fPIC", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+        os.replace(tmp, LIB)   # atomic: a reader never sees a partly written library
     return LIB
 
 

@@ -172,6 +172,10 @@ struct Layout {
   static constexpr int MERGE = NW * ((D / 16) * 32 * 4 + 16) * 4;  // fragment chunks + m, l per warp
   static constexpr int TOTAL = 1024 + NW * WARP + TABLE + BARS + 16;
   static_assert(TOTAL == cta_smem(KT, VT, D, NW, kStages), "layout and budget agree");
+  // The value level table is a static shared array (its address is then a
+  // constant the table loads fold in); the rest is dynamic shared memory.
+  static constexpr int VTAB = turbo_table_entries(VT) * 32 * 4;
+  static constexpr int DYN = TOTAL - VTAB;
   static_assert(MERGE <= NW * WARP, "merge area must fit in the stage memory");
   static_assert(TOTAL <= 227 * 1024, "shared memory per CTA");
 };
@@ -322,6 +326,14 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// largest (g * fb) mod 4 over the 8 lane groups g: how far a lane group's
+// code bytes can start past a 4-byte boundary
+__host__ __device__ constexpr int max_lane_misalign(int fb) {
+  int m = 0;
+  for (int g = 0; g < 8; ++g) m = (g * fb) % 4 > m ? (g * fb) % 4 : m;
+  return m;
+}
+
 template <int MASK>
 __device__ __forceinline__ int swz(int off) {
   return off ^ (((off >> 7) & MASK) << 4);
@@ -376,8 +388,11 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   unsigned char* wbase = smem + warp * L::WARP;
   const uint32_t wbase32 = smem_addr(wbase);
   __shared__ int cta_failed;
+  // value level table (static, see Layout), then in dynamic memory the key
+  // table and query rows of turbo keys, then the ring barriers
+  __shared__ __align__(128) uint32_t s_vtab[L::VTAB > 0 ? L::VTAB / 4 : 1];
   uint32_t* table = reinterpret_cast<uint32_t*>(smem + L::NW * L::WARP);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::NW * L::WARP + L::TABLE) + warp * S;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::NW * L::WARP + (L::TABLE - L::VTAB)) + warp * S;
 
   const int s_idx = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   // rows of this batch row, and its split length (whole 32-row tiles)
@@ -457,13 +472,13 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     constexpr int TB = turbo_bits(VT), NE = turbo_table_entries(VT);
     for (int e = threadIdx.x; e < NE * 32; e += L::NW * 32) {
       const int idx = e >> 5;
-      table[e] = TB <= 3 ? pack_half2(p.tq.levels[idx & ((1 << TB) - 1)], p.tq.levels[idx >> TB])
+      s_vtab[e] = TB <= 3 ? pack_half2(p.tq.levels[idx & ((1 << TB) - 1)], p.tq.levels[idx >> TB])
                          : pack_half2(p.tq.levels[idx], p.tq.levels[idx]);
     }
   }
-  // turbo keys: their level table after the value table, ktable[x * 32 + lane]
-  // = half2(c_hi[x], c_lo[x]); then the rotated queries as fp16 hi and lo parts
-  uint32_t* ktable = table + turbo_table_entries(VT) * 32;
+  // turbo keys: their level table, ktable[x * 32 + lane] = half2(c_hi[x],
+  // c_lo[x]); then the rotated queries as fp16 hi and lo parts
+  uint32_t* ktable = table;
   __half* qhi = reinterpret_cast<__half*>(ktable + key_table_entries(KT) * 32);  // [16][D]
   __half* qlo = qhi + 16 * D;                                                        // [16][D]
   constexpr int PST = qjl_stride(D);
@@ -1028,7 +1043,63 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       // b <= 3: table[x * 32 + lane] = half2(c[x mod 2^b], c[x >> b]), the levels
       // of one row's two consecutive dims; b = 4: half2(c[x], c[x]), two
       // lookups per dim pair.  A byte permute then pairs rows 2c and 2c+1.
-      const uint32_t* tl = table + lane;
+      if constexpr (TB <= 3 && (TB * D) % 64 == 0) {
+        // Lane group g's codes of a row start on byte g * FB.  They are read as
+        // aligned words and realigned by one byte permute per word (selector
+        // from the lane's byte offset), so every pair index below sits at a
+        // constant bit position: one shift moves it to bit 7 and one and-or
+        // makes the byte offset (x << 7) | (lane << 2) of its table entry in the
+        // static table.
+        constexpr int FB = TB * D / 64;
+        constexpr int NOUT = (FB + 3) / 4;
+        constexpr int SMAX = max_lane_misalign(FB);
+        constexpr int NLD = (FB + SMAX + 3) / 4;
+        constexpr int PW = 2 * TB;                                   // bits of a pair index
+        constexpr uint32_t PMASK = ((1u << PW) - 1u) << 7;
+        const int off = g * FB;
+        const uint32_t sel = 0x3210u + 0x1111u * (uint32_t)(off & 3);
+        const uint32_t lane4 = (uint32_t)lane << 2;
+        const unsigned char* tab = reinterpret_cast<const unsigned char*>(s_vtab);
+        auto load_field = [&](int row, uint32_t (&o)[NOUT]) {
+          const uint32_t* wp = reinterpret_cast<const uint32_t*>(vc + row * L::RBV + (off & ~3));
+          uint32_t w[NLD + 1];
+#pragma unroll
+          for (int i = 0; i < NLD; ++i) w[i] = wp[i];
+          w[NLD] = 0u;
+#pragma unroll
+          for (int i = 0; i < NOUT; ++i) o[i] = prmt(w[i], w[i + 1], sel);
+        };
+        // table entry of the pair at bit position pos of a field (pos is a
+        // constant once the loop below is unrolled)
+        auto entry = [&](const uint32_t (&o)[NOUT], int pos) -> uint32_t {
+          const int i = pos / 32, r = pos % 32;
+          uint32_t x;
+          if (r + PW > 32) x = __funnelshift_r(o[i], o[i + 1 < NOUT ? i + 1 : i], r - 7);
+          else if (r >= 7) x = o[i] >> (r - 7);
+          else x = o[i] << (7 - r);
+          return *reinterpret_cast<const uint32_t*>(tab + ((x & PMASK) | lane4));
+        };
+        uint32_t oA[NOUT], oB[NOUT], oC[NOUT], oD[NOUT];
+        load_field(2 * c, oA);
+        load_field(2 * c + 1, oB);
+        load_field(2 * c + 8, oC);
+        load_field(2 * c + 9, oD);
+#pragma unroll
+        for (int mt = 0; mt < NMT; ++mt) {
+          const uint32_t tA = entry(oA, PW * mt), tB = entry(oB, PW * mt);
+          const uint32_t tC = entry(oC, PW * mt), tD = entry(oD, PW * mt);
+          uint32_t a[4];
+          a[0] = prmt(tA, tB, 0x5410);  // dim 2mt:   rows 2c, 2c+1
+          a[1] = prmt(tA, tB, 0x7632);  // dim 2mt+1
+          a[2] = prmt(tC, tD, 0x5410);  // dim 2mt:   rows 2c+8, 2c+9
+          a[3] = prmt(tC, tD, 0x7632);
+#pragma unroll
+          for (int nt = 0; nt < NTH; ++nt)
+            mma16816(acc[nt][mt], a[0], a[1], a[2], a[3], pbw[nt][0], pbw[nt][1], acc[nt][mt]);
+        }
+        return;
+      }
+      const uint32_t* tl = s_vtab + lane;
 #pragma unroll
       for (int h = 0; h < HALVES; ++h) {
         const unsigned long long fA = field(2 * c, h), fB = field(2 * c + 1, h);
@@ -1214,14 +1285,70 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     const __half* vs0 = reinterpret_cast<const __half*>(vs_of(st));
 
     float sc0[NTH][4], sc1[NTH][4];
-    qk_tile(kc0, kc_of(st), ks0, sc0);
-    if (two) {
-      qk_tile(kc0 + kHalf * L::RBK, kc_of(st) + kHalf * L::RBK, ks0 + kHalf * L::NSK, sc1);
-    } else {
+    uint32_t pb0[NTH][2], pb1[NTH][2];
+    // ---------------- online softmax over the 32 rows (heads 2c, 2c+1).  The
+    // running max only moves when a score passes it, which after the first
+    // tiles is rare: only then are the row maxima reduced across the warp and
+    // the state rescaled.  Every P stays <= 1 either way.
+    auto softmax = [&]() {
 #pragma unroll
-      for (int nt = 0; nt < NTH; ++nt) sc1[nt][0] = sc1[nt][1] = sc1[nt][2] = sc1[nt][3] = -INFINITY;
-    }
-    if (rem < kSub) {
+      for (int nt = 0; nt < NTH; ++nt) {
+        float mx0 = fmaxf(fmaxf(sc0[nt][0], sc0[nt][2]), fmaxf(sc1[nt][0], sc1[nt][2]));
+        float mx1 = fmaxf(fmaxf(sc0[nt][1], sc0[nt][3]), fmaxf(sc1[nt][1], sc1[nt][3]));
+        if (__any_sync(0xffffffffu, mx0 > m_run[nt][0] || mx1 > m_run[nt][1])) {
+#pragma unroll
+          for (int o = 4; o <= 16; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+          }
+          const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+          const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
+          m_run[nt][0] = mn0;
+          m_run[nt][1] = mn1;
+          l_run[nt][0] *= al0;
+          l_run[nt][1] *= al1;
+#pragma unroll
+          for (int i = 0; i < NMT; ++i) {
+            acc[nt][i][0] *= al0;
+            acc[nt][i][1] *= al1;
+            acc[nt][i][2] *= al0;
+            acc[nt][i][3] *= al1;
+          }
+          if (kVQ) {
+            off[nt][0] *= al0;
+            off[nt][1] *= al1;
+          }
+        }
+        const float p0 = fast_exp2(sc0[nt][0] - m_run[nt][0]), p1 = fast_exp2(sc0[nt][1] - m_run[nt][1]);
+        const float p2 = fast_exp2(sc0[nt][2] - m_run[nt][0]), p3 = fast_exp2(sc0[nt][3] - m_run[nt][1]);
+        const float q0 = fast_exp2(sc1[nt][0] - m_run[nt][0]), q1 = fast_exp2(sc1[nt][1] - m_run[nt][1]);
+        const float q2 = fast_exp2(sc1[nt][2] - m_run[nt][0]), q3 = fast_exp2(sc1[nt][3] - m_run[nt][1]);
+        l_run[nt][0] += (p0 + p2) + (q0 + q2);
+        l_run[nt][1] += (p1 + p3) + (q1 + q3);
+        pb0[nt][0] = movmatrix_trans(pack_half2(p0, p1));
+        pb0[nt][1] = movmatrix_trans(pack_half2(p2, p3));
+        pb1[nt][0] = movmatrix_trans(pack_half2(q0, q1));
+        pb1[nt][1] = movmatrix_trans(pack_half2(q2, q3));
+      }
+    };
+    if (rem >= kSub) {
+      // A whole tile: both halves with no masks, in one basic block, so the
+      // two halves' dependency chains interleave.
+      qk_tile(kc0, kc_of(st), ks0, sc0);
+      qk_tile(kc0 + kHalf * L::RBK, kc_of(st) + kHalf * L::RBK, ks0 + kHalf * L::NSK, sc1);
+      softmax();
+      pv_tile(vc0, vc32, vs0, pb0, false, 0xFFFFFFFFu, 0xFFFFFFFFu);
+      pv_tile(vc0 + kHalf * L::RBV, vc32 + kHalf * L::RBV, vs0 + kHalf * L::NSV, pb1, false, 0xFFFFFFFFu,
+              0xFFFFFFFFu);
+    } else {
+      // the split's last tile: rows past its end masked out
+      qk_tile(kc0, kc_of(st), ks0, sc0);
+      if (two) {
+        qk_tile(kc0 + kHalf * L::RBK, kc_of(st) + kHalf * L::RBK, ks0 + kHalf * L::NSK, sc1);
+      } else {
+#pragma unroll
+        for (int nt = 0; nt < NTH; ++nt) sc1[nt][0] = sc1[nt][1] = sc1[nt][2] = sc1[nt][3] = -INFINITY;
+      }
 #pragma unroll
       for (int nt = 0; nt < NTH; ++nt) {
         if (g >= nv0) sc0[nt][0] = sc0[nt][1] = -INFINITY;
@@ -1229,64 +1356,20 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         if (g >= nv1) sc1[nt][0] = sc1[nt][1] = -INFINITY;
         if (g + 8 >= nv1) sc1[nt][2] = sc1[nt][3] = -INFINITY;
       }
-    }
-
-    // ---------------- online softmax over the 32 rows (heads 2c, 2c+1).  The
-    // running max only moves when a score passes it, which after the first
-    // tiles is rare: only then are the row maxima reduced across the warp and
-    // the state rescaled.  Every P stays <= 1 either way.
-    uint32_t pb0[NTH][2], pb1[NTH][2];
-#pragma unroll
-    for (int nt = 0; nt < NTH; ++nt) {
-      float mx0 = fmaxf(fmaxf(sc0[nt][0], sc0[nt][2]), fmaxf(sc1[nt][0], sc1[nt][2]));
-      float mx1 = fmaxf(fmaxf(sc0[nt][1], sc0[nt][3]), fmaxf(sc1[nt][1], sc1[nt][3]));
-      if (__any_sync(0xffffffffu, mx0 > m_run[nt][0] || mx1 > m_run[nt][1])) {
-#pragma unroll
-        for (int o = 4; o <= 16; o <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-        }
-        const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-        const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
-        m_run[nt][0] = mn0;
-        m_run[nt][1] = mn1;
-        l_run[nt][0] *= al0;
-        l_run[nt][1] *= al1;
-#pragma unroll
-        for (int i = 0; i < NMT; ++i) {
-          acc[nt][i][0] *= al0;
-          acc[nt][i][1] *= al1;
-          acc[nt][i][2] *= al0;
-          acc[nt][i][3] *= al1;
-        }
-        if (kVQ) {
-          off[nt][0] *= al0;
-          off[nt][1] *= al1;
-        }
+      softmax();
+      // In a tail half, P rows past the split end contribute exactly 0 whatever
+      // the row's scale holds (b operand halves: rows 2c, 2c+1 | 2c+8, 2c+9).
+      auto pmask = [&](int nv, uint32_t& lo, uint32_t& hi) {
+        lo = (2 * c < nv ? 0x0000FFFFu : 0u) | (2 * c + 1 < nv ? 0xFFFF0000u : 0u);
+        hi = (2 * c + 8 < nv ? 0x0000FFFFu : 0u) | (2 * c + 9 < nv ? 0xFFFF0000u : 0u);
+      };
+      uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
+      if (tail0) pmask(nv0, mlo, mhi);
+      pv_tile(vc0, vc32, vs0, pb0, tail0, mlo, mhi);
+      if (two) {
+        if (tail1) pmask(nv1, mlo, mhi);
+        pv_tile(vc0 + kHalf * L::RBV, vc32 + kHalf * L::RBV, vs0 + kHalf * L::NSV, pb1, tail1, mlo, mhi);
       }
-      const float p0 = fast_exp2(sc0[nt][0] - m_run[nt][0]), p1 = fast_exp2(sc0[nt][1] - m_run[nt][1]);
-      const float p2 = fast_exp2(sc0[nt][2] - m_run[nt][0]), p3 = fast_exp2(sc0[nt][3] - m_run[nt][1]);
-      const float q0 = fast_exp2(sc1[nt][0] - m_run[nt][0]), q1 = fast_exp2(sc1[nt][1] - m_run[nt][1]);
-      const float q2 = fast_exp2(sc1[nt][2] - m_run[nt][0]), q3 = fast_exp2(sc1[nt][3] - m_run[nt][1]);
-      l_run[nt][0] += (p0 + p2) + (q0 + q2);
-      l_run[nt][1] += (p1 + p3) + (q1 + q3);
-      pb0[nt][0] = movmatrix_trans(pack_half2(p0, p1));
-      pb0[nt][1] = movmatrix_trans(pack_half2(p2, p3));
-      pb1[nt][0] = movmatrix_trans(pack_half2(q0, q1));
-      pb1[nt][1] = movmatrix_trans(pack_half2(q2, q3));
-    }
-    // In a tail half, P rows past the split end contribute exactly 0 whatever
-    // the row's scale holds (b operand halves: rows 2c, 2c+1 | 2c+8, 2c+9).
-    auto pmask = [&](int nv, uint32_t& lo, uint32_t& hi) {
-      lo = (2 * c < nv ? 0x0000FFFFu : 0u) | (2 * c + 1 < nv ? 0xFFFF0000u : 0u);
-      hi = (2 * c + 8 < nv ? 0x0000FFFFu : 0u) | (2 * c + 9 < nv ? 0xFFFF0000u : 0u);
-    };
-    uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
-    if (tail0) pmask(nv0, mlo, mhi);
-    pv_tile(vc0, vc32, vs0, pb0, tail0, mlo, mhi);
-    if (two) {
-      if (tail1) pmask(nv1, mlo, mhi);
-      pv_tile(vc0 + kHalf * L::RBV, vc32 + kHalf * L::RBV, vs0 + kHalf * L::NSV, pb1, tail1, mlo, mhi);
     }
 
     // release the stage and refill it with this warp's tile j + S
@@ -1657,11 +1740,11 @@ cudaError_t launch_one(const TcArgs& a, const TcMaps& m, cudaStream_t st) {
   using L = Layout<KT, VT, NB * 32>;
   auto kern = decode_tc_kernel<KT, VT, NB, NTH, PAGED>;
   static std::atomic<uint64_t> attr_done{0};
-  const cudaError_t e = set_smem_limit_once(kern, L::TOTAL, attr_done);
+  const cudaError_t e = set_smem_limit_once(kern, L::DYN, attr_done);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.p.S, a.p.n_kv, a.p.B);
   if (!a.p.pdl) {
-    kern<<<grid, L::NW * 32, L::TOTAL, st>>>(a, m.kc, m.ks, m.vc, m.vs);
+    kern<<<grid, L::NW * 32, L::DYN, st>>>(a, m.kc, m.ks, m.vc, m.vs);
     return cudaGetLastError();
   }
   // programmatic dependent launch: may start once the previous kernel on the
@@ -1669,7 +1752,7 @@ cudaError_t launch_one(const TcArgs& a, const TcMaps& m, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(L::NW * 32);
-  cfg.dynamicSmemBytes = L::TOTAL;
+  cfg.dynamicSmemBytes = L::DYN;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -71,6 +71,13 @@ WORKLOADS = {
     # TurboQuant-style V: 70B shape, batch 1, 32K, K q8_0 / V turbo3
     "turbo3_ctx32k": Workload("turbo3_ctx32k", 1, 80, 64, 8, 128, 32768, "q8_0", "turbo3",
                               (3, 17, 66, 101), 8.0, 20260105, turbo_seed=TURBO3_SEED),
+    # the same at batch 4 (the steady-state rate of the turbo3 value path)
+    "turbo3_ctx32k_b4": Workload("turbo3_ctx32k_b4", 4, 80, 64, 8, 128, 32768, "q8_0", "turbo3",
+                                 (3, 17, 66, 101), 8.0, 20260105, turbo_seed=TURBO3_SEED),
+    # the TurboQuant page's three parts on keys (2-bit levels + 1-bit QJL residual),
+    # 70B shape, batch 4, 32K, K turbo3_qjl / V q8_0
+    "qjl_ctx32k_b4": Workload("qjl_ctx32k_b4", 4, 80, 64, 8, 128, 32768, "turbo3_qjl", "q8_0",
+                              (3, 17, 66, 101), 8.0, 20260106, turbo_seed=TURBO3_SEED),
 }
 
 
