@@ -171,3 +171,19 @@ def test_reference_arm_line_on_rank_zero():
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_loads_nothing_of_the_library():
+    """The oracle arm runs the C++ oracle only: after it, neither the library's
+    binding nor libkvq.so is loaded in the process."""
+    code = ("import runpy, sys\n"
+            "sys.argv = ['bench.py', '--impl', 'reference', '--workload', 'tiny', '--steps', '1', '--warmup', '0']\n"
+            f"runpy.run_path({os.path.join(ROOT, 'bench.py')!r}, run_name='__main__')\n"
+            "maps = open('/proc/self/maps').read()\n"
+            "print('LIB' if ('decode_attention_q8_b200' in sys.modules or 'libkvq' in maps) else 'CLEAN')\n"
+            "print('ORACLE' if 'liboracle' in maps else 'NO-ORACLE')\n")
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    out = r.stdout.strip().splitlines()
+    assert out[-2:] == ["CLEAN", "ORACLE"], out
