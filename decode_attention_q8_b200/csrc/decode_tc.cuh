@@ -579,6 +579,13 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     asm volatile("griddepcontrol.wait;" ::: "memory");
     load_queries();
   }
+  // Fused step with a shared combine: the group's epoch word as it stands
+  // before this CTA arrives (the combine below waits for it to change).  Read
+  // here, off the critical path at the end; the fence before the arrival
+  // orders this read before it.
+  __shared__ unsigned int comb_epoch0;
+  if (p.out != nullptr && p.comb_ctas > 1 && threadIdx.x == 0)
+    comb_epoch0 = *reinterpret_cast<volatile unsigned int*>(p.epochs + plane);
   if (warp == wt) {
     constexpr int rk = rows::row_threads(KT, D), rv = rows::row_threads(VT, D);
 #pragma unroll
@@ -1539,10 +1546,10 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     __threadfence();  // this CTA's partials are visible device-wide ...
     __syncthreads();
     if (threadIdx.x == 0) {  // ... before its arrival is counted
-      // the epoch is read before this CTA arrives: rank 0 bumps it only after
-      // the last arrival, so a waiter cannot miss the bump
-      const unsigned int e0 = p.comb_ctas > 1 ? *reinterpret_cast<volatile unsigned int*>(p.epochs + plane) : 0u;
-      if (p.comb_ctas > 1) __threadfence();
+      // the epoch was read before this CTA arrives (at the top, ordered by the
+      // fence above): rank 0 bumps it only after the last arrival, so a waiter
+      // cannot miss the bump
+      const unsigned int e0 = p.comb_ctas > 1 ? comb_epoch0 : 0u;
       const unsigned int ticket = atomicInc(p.counters + plane, (unsigned)(p.S - 1));
       // a counter left outside [0, S) by a caller (it must start at 0) gives a
       // ticket above S - 1: a huge rank, so that CTA only arrives
