@@ -106,9 +106,16 @@ __host__ __device__ constexpr int stage_bytes(int kt, int vt, int d) {
 // stages per warp (rounded to the 1024-byte swizzle atom), the turbo level
 // tables (values, then keys) and, for turbo keys, the rotated queries of up to 16
 // heads, the ring barriers and a few bytes of slack.
-// Turbo keys: one entry per level, half2(c_hi, c_lo) with c = c_hi + c_lo to
-// ~2^-22 (the scores enter an exponential, so fp16 levels alone are too coarse).
-__host__ __device__ constexpr int key_table_entries(int t) { return is_turbo(t) ? 1 << turbo_bits(t) : 0; }
+// Turbo keys: levels as c = c_hi + c_lo to ~2^-22 (the scores enter an
+// exponential, so fp16 levels alone are too coarse).  At 3 and 4 bits one entry
+// per level, half2(c_hi, c_lo).  At 2 bits (turbo2, turbo3_qjl) one entry per
+// code pair x of two consecutive dims, in two tables: half2(c_hi[x mod 4],
+// c_hi[x >> 2]), then half2(c_lo[x mod 4], c_lo[x >> 2]) -- A-operand registers
+// as they are, one lookup each.
+__host__ __device__ constexpr bool key_pair_table(int t) { return is_turbo(t) && turbo_bits(t) <= 2; }
+__host__ __device__ constexpr int key_table_entries(int t) {
+  return key_pair_table(t) ? 2 << (2 * turbo_bits(t)) : is_turbo(t) ? 1 << turbo_bits(t) : 0;
+}
 // turbo3_qjl keys: the projected queries P q_rot of up to 16 heads as fp16 hi
 // and lo parts, rows padded to d + 8 halves (the MMA B-fragment reads of the 8
 // heads of an n-tile then fall in distinct banks).
@@ -476,15 +483,23 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
                          : pack_half2(p.tq.levels[idx], p.tq.levels[idx]);
     }
   }
-  // turbo keys: their level table, ktable[x * 32 + lane] = half2(c_hi[x],
-  // c_lo[x]); then the rotated queries as fp16 hi and lo parts
+  // turbo keys: their level table, ktable[x * 32 + lane] (one copy per bank);
+  // then the rotated queries as fp16 hi and lo parts
   uint32_t* ktable = table;
   __half* qhi = reinterpret_cast<__half*>(ktable + key_table_entries(KT) * 32);  // [16][D]
   __half* qlo = qhi + 16 * D;                                                        // [16][D]
   constexpr int PST = qjl_stride(D);
   __half* phi = qlo + 16 * D;    // turbo3_qjl: P q_rot, [16][PST]
   __half* plo = phi + 16 * PST;  // [16][PST]
-  if constexpr (is_turbo(KT)) {
+  if constexpr (key_pair_table(KT)) {
+    constexpr int TB = turbo_bits(KT), NP = 1 << (2 * TB);
+    for (int e = threadIdx.x; e < 2 * NP * 32; e += L::NW * 32) {
+      const int x = (e >> 5) & (NP - 1);
+      const float c0 = p.tqk.levels[x & ((1 << TB) - 1)], c1 = p.tqk.levels[x >> TB];
+      const float h0 = __half2float(__float2half_rn(c0)), h1 = __half2float(__float2half_rn(c1));
+      ktable[e] = (e >> 5) < NP ? pack_half2(h0, h1) : pack_half2(c0 - h0, c1 - h1);
+    }
+  } else if constexpr (is_turbo(KT)) {
     constexpr int NE = key_table_entries(KT);
     for (int e = threadIdx.x; e < NE * 32; e += L::NW * 32) {
       const float cl = p.tqk.levels[e >> 5];
@@ -803,13 +818,21 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         if (16 * TB + 8 * (byte0 & 3) > 32) v |= (unsigned long long)(*reinterpret_cast<const uint32_t*>(rp + 4)) << 32;
         return v >> (8 * (byte0 & 3));
       };
-      // dims j, j+1 of the window: (hi pair, lo pair) from two level lookups
+      // dims j, j+1 of the window: (hi pair, lo pair), from the pair tables
+      // at 2 bits, else from two level lookups
       auto pair = [&](unsigned long long f, int j, uint32_t& hi, uint32_t& lo) {
-        constexpr uint32_t M = (1u << TB) - 1;
-        const uint32_t e0 = ktl[((uint32_t)(f >> (TB * j)) & M) << 5];
-        const uint32_t e1 = ktl[((uint32_t)(f >> (TB * j + TB)) & M) << 5];
-        hi = prmt(e0, e1, 0x5410);
-        lo = prmt(e0, e1, 0x7632);
+        if constexpr (key_pair_table(KT)) {
+          constexpr uint32_t NP = 1u << (2 * TB);
+          const uint32_t x = ((uint32_t)(f >> (TB * j)) & (NP - 1)) << 5;
+          hi = ktl[x];
+          lo = ktl[x + NP * 32];
+        } else {
+          constexpr uint32_t M = (1u << TB) - 1;
+          const uint32_t e0 = ktl[((uint32_t)(f >> (TB * j)) & M) << 5];
+          const uint32_t e1 = ktl[((uint32_t)(f >> (TB * j + TB)) & M) << 5];
+          hi = prmt(e0, e1, 0x5410);
+          lo = prmt(e0, e1, 0x7632);
+        }
       };
       // turbo3_qjl: the 16 sign bits of a row's k-step (bit i of the z field,
       // after the D/4 bytes of level codes); bits j, j+1 of a window as the
