@@ -107,12 +107,12 @@ __host__ __device__ constexpr int stage_bytes(int kt, int vt, int d) {
 // tables (values, then keys) and, for turbo keys, the rotated queries of up to 16
 // heads, the ring barriers and a few bytes of slack.
 // Turbo keys: levels as c = c_hi + c_lo to ~2^-22 (the scores enter an
-// exponential, so fp16 levels alone are too coarse).  At 3 and 4 bits one entry
-// per level, half2(c_hi, c_lo).  At 2 bits (turbo2, turbo3_qjl) one entry per
-// code pair x of two consecutive dims, in two tables: half2(c_hi[x mod 4],
-// c_hi[x >> 2]), then half2(c_lo[x mod 4], c_lo[x >> 2]) -- A-operand registers
-// as they are, one lookup each.
-__host__ __device__ constexpr bool key_pair_table(int t) { return is_turbo(t) && turbo_bits(t) <= 2; }
+// exponential, so fp16 levels alone are too coarse).  At 2 and 3 bits (turbo2,
+// turbo3_qjl, turbo3) one entry per code pair x of two consecutive dims, in two
+// tables: half2(c_hi[x mod 2^b], c_hi[x >> b]), then the same of c_lo -- the
+// A-operand registers as they are, one lookup each.  At 4 bits (a 2 x 64 KB
+// pair table) one entry per level, half2(c_hi, c_lo).
+__host__ __device__ constexpr bool key_pair_table(int t) { return is_turbo(t) && turbo_bits(t) <= 3; }
 __host__ __device__ constexpr int key_table_entries(int t) {
   return key_pair_table(t) ? 2 << (2 * turbo_bits(t)) : is_turbo(t) ? 1 << turbo_bits(t) : 0;
 }
@@ -579,10 +579,16 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   const bool owner = append_pos >= t0l && append_pos < t1l;
   const int t_new = owner ? (int)(append_pos - t0l) / kSub : -1;
   const int wt = owner ? t_new % L::NW : -1, jt = owner ? t_new / L::NW : -1;
+  // A launch that overlaps the previous kernel requests only each warp's first
+  // tile before the dependency resolves when the values are turbo rows and the
+  // keys are not (a smaller burst disturbs the previous step's end less; with
+  // turbo keys too it measured slightly slower), the other stages right after
+  // it; every stage otherwise.
+  constexpr int kEarly = is_turbo(VT) && !is_turbo(KT) ? 1 : S;
 #pragma unroll
   for (int j = 0; j < S; ++j) {
     const int pg = paged ? __shfl_sync(0xffffffffu, pg_win, j) : 0;
-    if (lane == 0 && j < my_tiles && !(warp == wt && j == jt)) issue(j, j, pg);
+    if (lane == 0 && j < my_tiles && !(warp == wt && j == jt) && (!p.pdl || j < kEarly)) issue(j, j, pg);
   }
   // The kernel after this one on the stream may be scheduled from here on (a
   // no-op unless it was launched to overlap this one).  A launch that overlaps
@@ -593,6 +599,13 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
   if (p.pdl) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     load_queries();
+    if constexpr (kEarly < S) {
+#pragma unroll
+      for (int j = kEarly; j < S; ++j) {
+        const int pg = paged ? __shfl_sync(0xffffffffu, pg_win, j) : 0;
+        if (lane == 0 && j < my_tiles && !(warp == wt && j == jt)) issue(j, j, pg);
+      }
+    }
   }
   // Fused step with a shared combine: the group's epoch word as it stands
   // before this CTA arrives (the combine below waits for it to change).  Read
@@ -819,7 +832,7 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
         return v >> (8 * (byte0 & 3));
       };
       // dims j, j+1 of the window: (hi pair, lo pair), from the pair tables
-      // at 2 bits, else from two level lookups
+      // at 2 and 3 bits, else from two level lookups
       auto pair = [&](unsigned long long f, int j, uint32_t& hi, uint32_t& lo) {
         if constexpr (key_pair_table(KT)) {
           constexpr uint32_t NP = 1u << (2 * TB);
