@@ -693,12 +693,17 @@ def run_kvq(args):
         dist.destroy_process_group()
 
 
+# Sources of the decode kernel: its own files and the headers it includes
+# (the fused step's row append and the shared parameter structs).
+DECODE_HEADERS = ("append_rows.cuh", "kvq_internal.h")
+
+
 def _decode_source_sha():
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "decode_attention_q8_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.startswith("decode"):
+        if f.startswith("decode") or f in DECODE_HEADERS:
             h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 

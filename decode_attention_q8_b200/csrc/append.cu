@@ -70,14 +70,40 @@ __device__ __forceinline__ void append_blocks(const AppendParams& p, int64_t fir
   }
 }
 
+// Turbo rows other than turbo3_qjl: D/16 lanes per row (rows::append_turbo_wide),
+// kWideRound items (32 bytes of fp16 each) in flight per thread.
+constexpr int kWideRound = 2;
+template <int TYPE, int D>
+__device__ __forceinline__ void append_stream_wide(const AppendParams& p, int64_t first, int64_t stride, int64_t gend) {
+  for (int64_t base = first; (base & ~(int64_t)31) < gend; base += kWideRound * stride) {
+    rows::Raw32 raw[kWideRound];
+#pragma unroll
+    for (int u = 0; u < kWideRound; ++u) raw[u] = rows::load_wide(p, base + u * stride, gend);
+#pragma unroll
+    for (int u = 0; u < kWideRound; ++u) {
+      const int64_t g = base + u * stride;
+      if ((g & ~(int64_t)31) < gend) rows::append_turbo_wide<turbo_bits(TYPE), D>(p, g, gend, raw[u]);  // warp-uniform
+    }
+  }
+}
+
 template <int TYPE>
 __device__ __forceinline__ void append_turbo_part(const AppendParams& p, int64_t first, int64_t stride, int64_t gend,
                                                   const float* pt = nullptr) {
-  switch (p.D) {
-    case 32: append_stream<TYPE, 1>(p, first, stride, gend, pt); break;
-    case 64: append_stream<TYPE, 2>(p, first, stride, gend, pt); break;
-    case 128: append_stream<TYPE, 4>(p, first, stride, gend, pt); break;
-    case 256: append_stream<TYPE, 8>(p, first, stride, gend, pt); break;
+  if constexpr (!is_qjl(TYPE)) {
+    switch (p.D) {
+      case 32: append_stream_wide<TYPE, 32>(p, first, stride, gend); break;
+      case 64: append_stream_wide<TYPE, 64>(p, first, stride, gend); break;
+      case 128: append_stream_wide<TYPE, 128>(p, first, stride, gend); break;
+      case 256: append_stream_wide<TYPE, 256>(p, first, stride, gend); break;
+    }
+  } else {
+    switch (p.D) {
+      case 32: append_stream<TYPE, 1>(p, first, stride, gend, pt); break;
+      case 64: append_stream<TYPE, 2>(p, first, stride, gend, pt); break;
+      case 128: append_stream<TYPE, 4>(p, first, stride, gend, pt); break;
+      case 256: append_stream<TYPE, 8>(p, first, stride, gend, pt); break;
+    }
   }
 }
 

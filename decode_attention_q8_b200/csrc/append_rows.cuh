@@ -16,11 +16,12 @@
 // block to 8 consecutive threads holding 4 contiguous elements each (one 8-byte
 // load per thread; the block max is a 3-step xor-shuffle reduction inside the 8
 // lanes).  Loading (load_raw) and quantizing (finish) are separate steps, so a
-// thread can have several loads in flight.  The turbo types (and turbo3_qjl)
-// give each row to one warp, D/32 contiguous elements per lane; the
-// Walsh-Hadamard butterflies run in registers for strides below D/32 and as
-// xor-shuffles above.  Threads past the work still take part in the shuffles
-// and then return.
+// thread can have several loads in flight.  turbo3_qjl gives each row to one
+// warp, D/32 contiguous elements per lane; the other turbo types give it to
+// D/16 lanes, 16 contiguous elements each (append_turbo_wide).  The
+// Walsh-Hadamard butterflies run in registers for strides below the elements
+// per lane and as xor-shuffles above.  Threads past the work still take part in
+// the shuffles and then return.
 #pragma once
 
 #include "kvq_internal.h"
@@ -615,6 +616,105 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
   }
 }
 
+// Turbo rows other than turbo3_qjl: D/16 lanes per row, 16 contiguous
+// elements per lane (a row's lanes are an aligned group of the warp, 32/(D/16)
+// rows per warp).  The same operations in the same order as append_turbo -- the
+// norm's pairwise tree, each butterfly of the transform, the quantizer -- so the
+// stored bytes are the same; fewer levels cross lanes (log2(D/16) instead of
+// log2(32)), the per-row index work is shared by 32/(D/16) rows, and each lane
+// stores its own 2*BITS code bytes.
+constexpr int kWideElems = 16;
+struct Raw32 {
+  uint4 a, b;  // 16 fp16 elements
+};
+__device__ __forceinline__ Raw32 load_wide(const AppendParams& p, int64_t gtid, int64_t gend) {
+  Raw32 r{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+  if (gtid >= gend) return r;
+  const uint4* src = reinterpret_cast<const uint4*>(p.src + gtid * kWideElems);
+  r.a = __ldg(src);
+  r.b = __ldg(src + 1);
+  return r;
+}
+__device__ __forceinline__ float wide_elem(const Raw32& r, int i) {  // fp16 element i (0..15) as float
+  return raw_elem(i < 8 ? r.a : r.b, i & 7);
+}
+
+template <int BITS, int D>
+__device__ __forceinline__ void append_turbo_wide(const AppendParams& p, int64_t gtid, int64_t gend, const Raw32& raw) {
+  constexpr int LPR = D / kWideElems;  // lanes per row
+  constexpr int E = kWideElems;
+  const int lr = (int)(gtid & (LPR - 1));  // lane within the row (groups are aligned)
+  const int64_t row = gtid / LPR;
+  float v[E];
+  const int i0 = lr * E;  // the lane's first element; its 16 sign bits lie in one word
+  const uint32_t sw = p.tq.sign_bits[i0 >> 5] >> (i0 & 31);
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const float x = wide_elem(raw, e);
+    v[e] = ((sw >> e) & 1u) ? -x : x;
+  }
+  // |v|^2 by the strided pairwise tree a[i] += a[i+h], h = D/2 ... 1
+  float a[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) a[e] = __fmul_rn(v[e], v[e]);
+#pragma unroll
+  for (int h = D / 2; h >= E; h >>= 1) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) a[e] = __fadd_rn(a[e], __shfl_xor_sync(0xffffffffu, a[e], h / E));
+  }
+#pragma unroll
+  for (int h = E / 2; h >= 1; h >>= 1) {
+#pragma unroll
+    for (int e = 0; e < h; ++e) a[e] = __fadd_rn(a[e], a[e + h]);
+  }
+  const float norm = __fsqrt_rn(__shfl_sync(0xffffffffu, a[0], 0, LPR));
+  // unnormalised fast Walsh-Hadamard transform, strides h = 1, 2, ..., D/2
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if ((e & h) == 0) {
+        const float x0 = v[e], x1 = v[e + h];
+        v[e] = __fadd_rn(x0, x1);
+        v[e + h] = __fsub_rn(x0, x1);
+      }
+    }
+  }
+#pragma unroll
+  for (int h = E; h < D; h <<= 1) {
+    const int lm = h / E;
+    const bool upper = (lr & lm) != 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[e], lm);
+      v[e] = upper ? __fsub_rn(o, v[e]) : __fadd_rn(v[e], o);
+    }
+  }
+  const float r = norm > 0.0f ? __frcp_rn(norm) : 0.0f;
+  unsigned long long bits = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const float g = __fmul_rn(v[e], r);
+    int c = 0;
+#pragma unroll
+    for (int k = 0; k < (1 << BITS) - 1; ++k) c += g > p.tq.tau[k] ? 1 : 0;
+    bits |= (unsigned long long)c << (BITS * e);
+  }
+  if (gtid >= gend) return;  // after the last shuffle
+  const int64_t r_dst = dst_row(p, row);
+  if (r_dst < 0) return;
+  // the lane's codes: bits [16 * BITS * lr, 16 * BITS * (lr + 1)) of the row
+  uint8_t* codes = p.dst.codes + r_dst * p.dst.code_bytes + lr * 2 * BITS;
+  if constexpr (BITS % 2 == 0) {
+#pragma unroll
+    for (int k = 0; k < BITS / 2; ++k) reinterpret_cast<uint32_t*>(codes)[k] = (uint32_t)(bits >> (32 * k));
+  } else {
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) reinterpret_cast<uint16_t*>(codes)[k] = (uint16_t)(bits >> (16 * k));
+  }
+  if (lr == 0) p.dst.scales[r_dst] = __float2half_rn(fminf(norm, 65504.0f));
+}
+
 // Quantize and store work item gtid from its loaded bytes (every lane of the
 // warp calls this: the bodies shuffle; items at or past gend store nothing).
 template <int TYPE, int E>
@@ -629,7 +729,10 @@ __device__ __forceinline__ void finish(const AppendParams& p, int64_t gtid, int6
 
 template <int TYPE, int E>
 __device__ __forceinline__ void append_one(const AppendParams& p, int64_t gtid, int64_t gend) {
-  finish<TYPE, E>(p, gtid, gend, load_raw<TYPE, E>(p, gtid, gend));
+  if constexpr (is_turbo(TYPE) && !is_qjl(TYPE))
+    append_turbo_wide<turbo_bits(TYPE), 32 * E>(p, gtid, gend, load_wide(p, gtid, gend));
+  else
+    finish<TYPE, E>(p, gtid, gend, load_raw<TYPE, E>(p, gtid, gend));
 }
 
 // Thread gtid of the flat work of one call's rows of a tensor of `type`;
@@ -659,7 +762,7 @@ __device__ __forceinline__ void append_any(int32_t type, const AppendParams& p, 
 
 // Threads one row of a tensor of `type` and head dim d needs.
 __host__ __device__ constexpr int row_threads(int32_t type, int d) {
-  return type == KVQ_F16 ? d / 8 : is_turbo(type) ? 32 : (d / kBlock) * 8;
+  return type == KVQ_F16 ? d / 8 : is_qjl(type) ? 32 : is_turbo(type) ? d / kWideElems : (d / kBlock) * 8;
 }
 
 }  // namespace rows

@@ -70,6 +70,12 @@ def test_traffic_record_matches_source_hash(tmp_path, monkeypatch):
     assert bench._profiled_traffic("wl_a") == 123456
     (csrc / "decode_x.cu").write_text("// kernel v2\n")      # the kernel changed: counters are stale
     assert bench._profiled_traffic("wl_a") is None
+    # the headers the decode kernel includes count too
+    sha2 = bench._decode_source_sha()
+    (tmp_path / "profiles" / "decode_traffic.txt").write_text(f"wl_a 123456 {sha2}\n")
+    assert bench._profiled_traffic("wl_a") == 123456
+    (csrc / "append_rows.cuh").write_text("// the fused step's row append\n")
+    assert bench._profiled_traffic("wl_a") is None
 
 
 def test_whole_job_throughput_is_weak_scaling():
