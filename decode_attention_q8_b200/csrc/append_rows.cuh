@@ -422,6 +422,31 @@ __device__ __forceinline__ void append_f16(const AppendParams& p, int64_t gtid, 
 // P comes from pt, a transposed copy in shared memory (pt[j*D + i] = P[i][j]:
 // the warp reads one contiguous line per j), or, when pt is null, from global
 // memory row by row.
+// Code of g: the number of thresholds below it, #{k : g > tau[k]} (the
+// thresholds ascend), found by binary search: at 2 and 3 bits each step
+// compares against one threshold chosen by the bits decided so far (three or two
+// compares and a few selects instead of seven or three compares and adds; a NaN
+// fails every compare and gets code 0, as with the count).  4 bits: the count.
+template <int BITS>
+__device__ __forceinline__ int turbo_code(float g, const float* tau) {
+  if constexpr (BITS == 3) {
+    const bool b2 = g > tau[3];
+    const bool b1 = g > (b2 ? tau[5] : tau[1]);
+    const float t0 = b2 ? (b1 ? tau[6] : tau[4]) : (b1 ? tau[2] : tau[0]);
+    const bool b0 = g > t0;
+    return (b2 ? 4 : 0) + (b1 ? 2 : 0) + (b0 ? 1 : 0);
+  } else if constexpr (BITS == 2) {
+    const bool b1 = g > tau[1];
+    const bool b0 = g > (b1 ? tau[2] : tau[0]);
+    return (b1 ? 2 : 0) + (b0 ? 1 : 0);
+  } else {
+    int c = 0;
+#pragma unroll
+    for (int k = 0; k < (1 << BITS) - 1; ++k) c += g > tau[k] ? 1 : 0;
+    return c;
+  }
+}
+
 template <int BITS, int E, bool QJL = false>
 __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid, int64_t gend, const uint4& raw,
                                              const float* pt) {
@@ -479,13 +504,11 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const float g = __fmul_rn(v[e], r);
-    int c = 0;
-    float lv = p.tq.levels[0];  // levels[c] (thresholds ascend), without a dynamic index
+    const int c = turbo_code<BITS>(g, p.tq.tau);
+    float lv = 0.0f;  // QJL: levels[c], without a dynamic index
+    if constexpr (QJL) {
 #pragma unroll
-    for (int k = 0; k < (1 << BITS) - 1; ++k) {
-      const bool up = g > p.tq.tau[k];
-      c += up ? 1 : 0;
-      if (QJL) lv = up ? p.tq.levels[k + 1] : lv;
+      for (int k = 0; k < (1 << BITS); ++k) lv = c == k ? p.tq.levels[k] : lv;
     }
     bits |= (uint32_t)c << (BITS * e);
     res[e] = QJL ? __fsub_rn(g, lv) : 0.0f;
@@ -695,9 +718,7 @@ __device__ __forceinline__ void append_turbo_wide(const AppendParams& p, int64_t
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const float g = __fmul_rn(v[e], r);
-    int c = 0;
-#pragma unroll
-    for (int k = 0; k < (1 << BITS) - 1; ++k) c += g > p.tq.tau[k] ? 1 : 0;
+    const int c = turbo_code<BITS>(g, p.tq.tau);
     bits |= (unsigned long long)c << (BITS * e);
   }
   if (gtid >= gend) return;  // after the last shuffle
