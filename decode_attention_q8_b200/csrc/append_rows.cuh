@@ -59,6 +59,22 @@ __device__ __forceinline__ uint4 load_raw(const AppendParams& p, int64_t gtid, i
   return r;
 }
 
+// Packed binary32 pairs (low word: the first element), each lane rounded to
+// nearest like the scalar __fadd_rn / __fmul_rn.
+__device__ __forceinline__ unsigned long long pack_f32x2(float lo, float hi) {
+  return (unsigned long long)__float_as_uint(lo) | ((unsigned long long)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ unsigned long long add_f32x2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long mul_f32x2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ float raw_elem(const uint4& r, int i) {  // fp16 element i of r as float
   const uint32_t w = i < 2 ? r.x : i < 4 ? r.y : i < 6 ? r.z : r.w;
   const uint16_t h = (uint16_t)(w >> (16 * (i & 1)));
@@ -533,7 +549,32 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
     float u[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) u[e] = 0.0f;
-    if (pt != nullptr) {
+    if constexpr (E % 2 == 0) {
+      if (pt != nullptr) {
+        // two outputs per packed binary32 pair operation (the same two roundings
+        // per term as the scalar loop below, lane by lane)
+        unsigned long long u2[E / 2];
+#pragma unroll
+        for (int k = 0; k < E / 2; ++k) u2[k] = 0ull;
+#pragma unroll 2
+        for (int jl = 0; jl < 32; ++jl) {
+#pragma unroll
+          for (int e2 = 0; e2 < E; ++e2) {
+            const float ej = __shfl_sync(0xffffffffu, res[e2], jl);
+            const unsigned long long* col =
+                reinterpret_cast<const unsigned long long*>(pt + (jl * E + e2) * D + lane * E);
+            const unsigned long long ej2 = pack_f32x2(ej, ej);
+#pragma unroll
+            for (int k = 0; k < E / 2; ++k) u2[k] = add_f32x2(u2[k], mul_f32x2(col[k], ej2));
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < E / 2; ++k) {
+          u[2 * k] = __uint_as_float((uint32_t)u2[k]);
+          u[2 * k + 1] = __uint_as_float((uint32_t)(u2[k] >> 32));
+        }
+      }
+    } else if (pt != nullptr) {
 #pragma unroll 2
       for (int jl = 0; jl < 32; ++jl) {
 #pragma unroll
