@@ -15,7 +15,7 @@ constexpr int kBlockRound = 1;   // q8_0 / q4_0 blocks per thread and round (a b
 // Work items of one row in this kernel: a 32-element block for q8_0 / q4_0,
 // otherwise the row bodies' threads.
 __host__ __device__ constexpr int bulk_items(int32_t type, int d) {
-  return type == KVQ_Q8_0 || type == KVQ_Q4_0 || type == KVQ_Q5_0 ? d / kBlock : rows::row_threads(type, d);
+  return type == KVQ_Q8_0 || type == KVQ_Q4_0 || type == KVQ_Q5_0 ? d / kBlock : rows::bulk_row_threads(type, d);
 }
 
 // K and V rows of one append call in one launch.  Every CTA takes its share of

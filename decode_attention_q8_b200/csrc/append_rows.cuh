@@ -16,9 +16,9 @@
 // block to 8 consecutive threads holding 4 contiguous elements each (one 8-byte
 // load per thread; the block max is a 3-step xor-shuffle reduction inside the 8
 // lanes).  Loading (load_raw) and quantizing (finish) are separate steps, so a
-// thread can have several loads in flight.  turbo3_qjl gives each row to one
-// warp, D/32 contiguous elements per lane; the other turbo types give it to
-// D/16 lanes, 16 contiguous elements each (append_turbo_wide).  The
+// thread can have several loads in flight.  A turbo row takes one warp, D/32
+// contiguous elements per lane; in the bulk append the turbo types other than
+// turbo3_qjl take D/16 lanes, 16 contiguous elements each (append_turbo_wide).  The
 // Walsh-Hadamard butterflies run in registers for strides below the elements
 // per lane and as xor-shuffles above.  Threads past the work still take part in
 // the shuffles and then return.
@@ -443,6 +443,8 @@ __device__ __forceinline__ void append_f16(const AppendParams& p, int64_t gtid, 
 // compares against one threshold chosen by the bits decided so far (three or two
 // compares and a few selects instead of seven or three compares and adds; a NaN
 // fails every compare and gets code 0, as with the count).  4 bits: the count.
+// Used by the bulk body; the one-warp body (also inlined into the fused decode
+// step) keeps the plain count, which measured faster there.
 template <int BITS>
 __device__ __forceinline__ int turbo_code(float g, const float* tau) {
   if constexpr (BITS == 3) {
@@ -520,11 +522,13 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const float g = __fmul_rn(v[e], r);
-    const int c = turbo_code<BITS>(g, p.tq.tau);
-    float lv = 0.0f;  // QJL: levels[c], without a dynamic index
-    if constexpr (QJL) {
+    int c = 0;
+    float lv = p.tq.levels[0];  // levels[c] (thresholds ascend), without a dynamic index
 #pragma unroll
-      for (int k = 0; k < (1 << BITS); ++k) lv = c == k ? p.tq.levels[k] : lv;
+    for (int k = 0; k < (1 << BITS) - 1; ++k) {
+      const bool up = g > p.tq.tau[k];
+      c += up ? 1 : 0;
+      if (QJL) lv = up ? p.tq.levels[k + 1] : lv;
     }
     bits |= (uint32_t)c << (BITS * e);
     res[e] = QJL ? __fsub_rn(g, lv) : 0.0f;
@@ -680,9 +684,9 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
   }
 }
 
-// Turbo rows other than turbo3_qjl: D/16 lanes per row, 16 contiguous
-// elements per lane (a row's lanes are an aligned group of the warp, 32/(D/16)
-// rows per warp).  The same operations in the same order as append_turbo -- the
+// Bulk append of turbo rows other than turbo3_qjl: D/16 lanes per row, 16
+// contiguous elements per lane (a row's lanes are an aligned group of the warp,
+// 32/(D/16) rows per warp).  The same operations in the same order as append_turbo -- the
 // norm's pairwise tree, each butterfly of the transform, the quantizer -- so the
 // stored bytes are the same; fewer levels cross lanes (log2(D/16) instead of
 // log2(32)), the per-row index work is shared by 32/(D/16) rows, and each lane
@@ -791,10 +795,7 @@ __device__ __forceinline__ void finish(const AppendParams& p, int64_t gtid, int6
 
 template <int TYPE, int E>
 __device__ __forceinline__ void append_one(const AppendParams& p, int64_t gtid, int64_t gend) {
-  if constexpr (is_turbo(TYPE) && !is_qjl(TYPE))
-    append_turbo_wide<turbo_bits(TYPE), 32 * E>(p, gtid, gend, load_wide(p, gtid, gend));
-  else
-    finish<TYPE, E>(p, gtid, gend, load_raw<TYPE, E>(p, gtid, gend));
+  finish<TYPE, E>(p, gtid, gend, load_raw<TYPE, E>(p, gtid, gend));
 }
 
 // Thread gtid of the flat work of one call's rows of a tensor of `type`;
@@ -823,8 +824,16 @@ __device__ __forceinline__ void append_any(int32_t type, const AppendParams& p, 
 }
 
 // Threads one row of a tensor of `type` and head dim d needs.
+// (append_one, append_any: a turbo row on one warp.)
 __host__ __device__ constexpr int row_threads(int32_t type, int d) {
-  return type == KVQ_F16 ? d / 8 : is_qjl(type) ? 32 : is_turbo(type) ? d / kWideElems : (d / kBlock) * 8;
+  return type == KVQ_F16 ? d / 8 : is_turbo(type) ? 32 : (d / kBlock) * 8;
+}
+// Threads one row needs in the bulk append: turbo rows other than turbo3_qjl
+// take D/16 lanes there (append_turbo_wide).  The fused decode step appends its
+// one row per head with row_threads: the wide body's registers would weigh on the
+// decode kernel's own.
+__host__ __device__ constexpr int bulk_row_threads(int32_t type, int d) {
+  return is_turbo(type) && !is_qjl(type) ? d / kWideElems : row_threads(type, d);
 }
 
 }  // namespace rows
