@@ -1582,9 +1582,9 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
     __threadfence();  // this CTA's partials are visible device-wide ...
     __syncthreads();
     if (threadIdx.x == 0) {  // ... before its arrival is counted
-      // the epoch was read before this CTA arrives (at the top, ordered by the
-      // fence above): rank 0 bumps it only after the last arrival, so a waiter
-      // cannot miss the bump
+      // the epoch was read before this CTA arrives (once the grid dependency
+      // resolved, ordered by the fence above): rank 0 bumps it only after the
+      // last arrival, so a waiter cannot miss the bump
       const unsigned int e0 = p.comb_ctas > 1 ? comb_epoch0 : 0u;
       const unsigned int ticket = atomicInc(p.counters + plane, (unsigned)(p.S - 1));
       // a counter left outside [0, S) by a caller (it must start at 0) gives a
