@@ -328,6 +328,37 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
+// Packed binary32 pairs (f32x2): each lane rounded once, exactly as the scalar
+// fmaf / __fmul_rn / __fadd_rn / __fsub_rn of the same operands.
+__device__ __forceinline__ unsigned long long f2(float lo, float hi) {
+  unsigned long long d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2split(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2mul(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2sub(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -1017,10 +1048,9 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           float dblk[4];
           mma16816(dblk, a[0][0], a[0][1], a[0][2], a[0][3], qb[nt][blk][0][0], qb[nt][blk][0][1], cq[nt][blk]);
           mma16816(dblk, a[1][0], a[1][1], a[1][2], a[1][3], qb[nt][blk][1][0], qb[nt][blk][1][1], dblk);
-          sc[nt][0] = fmaf(dA[blk], dblk[0], sc[nt][0]);
-          sc[nt][1] = fmaf(dA[blk], dblk[1], sc[nt][1]);
-          sc[nt][2] = fmaf(dB[blk], dblk[2], sc[nt][2]);
-          sc[nt][3] = fmaf(dB[blk], dblk[3], sc[nt][3]);
+          // sc = fmaf(d, dblk, sc), two scores per packed operation
+          f2split(f2fma(f2(dA[blk], dA[blk]), f2(dblk[0], dblk[1]), f2(sc[nt][0], sc[nt][1])), sc[nt][0], sc[nt][1]);
+          f2split(f2fma(f2(dB[blk], dB[blk]), f2(dblk[2], dblk[3]), f2(sc[nt][2], sc[nt][3])), sc[nt][2], sc[nt][3]);
         } else {
           // f16 keys: no scale, no correction; accumulate in place
           mma16816(sc[nt], a[0][0], a[0][1], a[0][2], a[0][3], qb[nt][blk][0][0], qb[nt][blk][0][1], sc[nt]);
@@ -1029,9 +1059,11 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
       }
     }
 #pragma unroll
-    for (int nt = 0; nt < NTH; ++nt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sc[nt][i] *= qs;
+    for (int nt = 0; nt < NTH; ++nt) {
+      const unsigned long long qq = f2(qs, qs);
+      f2split(f2mul(f2(sc[nt][0], sc[nt][1]), qq), sc[nt][0], sc[nt][1]);
+      f2split(f2mul(f2(sc[nt][2], sc[nt][3]), qq), sc[nt][2], sc[nt][3]);
+    }
   };
 
   // PV of one 16-row tile with its P fragments (rows 2c, 2c+1 | 2c+8, 2c+9);
@@ -1362,12 +1394,17 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
             off[nt][1] *= al1;
           }
         }
-        const float p0 = fast_exp2(sc0[nt][0] - m_run[nt][0]), p1 = fast_exp2(sc0[nt][1] - m_run[nt][1]);
-        const float p2 = fast_exp2(sc0[nt][2] - m_run[nt][0]), p3 = fast_exp2(sc0[nt][3] - m_run[nt][1]);
-        const float q0 = fast_exp2(sc1[nt][0] - m_run[nt][0]), q1 = fast_exp2(sc1[nt][1] - m_run[nt][1]);
-        const float q2 = fast_exp2(sc1[nt][2] - m_run[nt][0]), q3 = fast_exp2(sc1[nt][3] - m_run[nt][1]);
-        l_run[nt][0] += (p0 + p2) + (q0 + q2);
-        l_run[nt][1] += (p1 + p3) + (q1 + q3);
+        // exponent arguments and the row sums two heads (2c, 2c+1) at a time
+        const unsigned long long mm = f2(m_run[nt][0], m_run[nt][1]);
+        float x0, x1, x2, x3, y0, y1, y2, y3;
+        f2split(f2sub(f2(sc0[nt][0], sc0[nt][1]), mm), x0, x1);
+        f2split(f2sub(f2(sc0[nt][2], sc0[nt][3]), mm), x2, x3);
+        f2split(f2sub(f2(sc1[nt][0], sc1[nt][1]), mm), y0, y1);
+        f2split(f2sub(f2(sc1[nt][2], sc1[nt][3]), mm), y2, y3);
+        const float p0 = fast_exp2(x0), p1 = fast_exp2(x1), p2 = fast_exp2(x2), p3 = fast_exp2(x3);
+        const float q0 = fast_exp2(y0), q1 = fast_exp2(y1), q2 = fast_exp2(y2), q3 = fast_exp2(y3);
+        const unsigned long long ls = f2add(f2add(f2(p0, p1), f2(p2, p3)), f2add(f2(q0, q1), f2(q2, q3)));
+        f2split(f2add(f2(l_run[nt][0], l_run[nt][1]), ls), l_run[nt][0], l_run[nt][1]);
         pb0[nt][0] = movmatrix_trans(pack_half2(p0, p1));
         pb0[nt][1] = movmatrix_trans(pack_half2(p2, p3));
         pb1[nt][0] = movmatrix_trans(pack_half2(q0, q1));
