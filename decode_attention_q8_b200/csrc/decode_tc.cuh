@@ -945,12 +945,11 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           sc[nt][3] = qs * (nB * sc[nt][3] + gB * sz[nt][3]);
         }
       } else {
+        const unsigned long long fa = f2(qs * nA, qs * nA), fb = f2(qs * nB, qs * nB);
 #pragma unroll
         for (int nt = 0; nt < NTH; ++nt) {
-          sc[nt][0] *= qs * nA;
-          sc[nt][1] *= qs * nA;
-          sc[nt][2] *= qs * nB;
-          sc[nt][3] *= qs * nB;
+          f2split(f2mul(f2(sc[nt][0], sc[nt][1]), fa), sc[nt][0], sc[nt][1]);
+          f2split(f2mul(f2(sc[nt][2], sc[nt][3]), fb), sc[nt][2], sc[nt][3]);
         }
       }
       return;
@@ -1380,19 +1379,14 @@ __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
           const float al0 = fast_exp2(m_run[nt][0] - mn0), al1 = fast_exp2(m_run[nt][1] - mn1);
           m_run[nt][0] = mn0;
           m_run[nt][1] = mn1;
-          l_run[nt][0] *= al0;
-          l_run[nt][1] *= al1;
+          const unsigned long long al = f2(al0, al1);
+          f2split(f2mul(f2(l_run[nt][0], l_run[nt][1]), al), l_run[nt][0], l_run[nt][1]);
 #pragma unroll
           for (int i = 0; i < NMT; ++i) {
-            acc[nt][i][0] *= al0;
-            acc[nt][i][1] *= al1;
-            acc[nt][i][2] *= al0;
-            acc[nt][i][3] *= al1;
+            f2split(f2mul(f2(acc[nt][i][0], acc[nt][i][1]), al), acc[nt][i][0], acc[nt][i][1]);
+            f2split(f2mul(f2(acc[nt][i][2], acc[nt][i][3]), al), acc[nt][i][2], acc[nt][i][3]);
           }
-          if (kVQ) {
-            off[nt][0] *= al0;
-            off[nt][1] *= al1;
-          }
+          if (kVQ) f2split(f2mul(f2(off[nt][0], off[nt][1]), al), off[nt][0], off[nt][1]);
         }
         // exponent arguments and the row sums two heads (2c, 2c+1) at a time
         const unsigned long long mm = f2(m_run[nt][0], m_run[nt][1]);
