@@ -62,7 +62,17 @@ __device__ __forceinline__ uint4 load_raw(const AppendParams& p, int64_t gtid, i
 // Packed binary32 pairs (low word: the first element), each lane rounded to
 // nearest like the scalar __fadd_rn / __fmul_rn.
 __device__ __forceinline__ unsigned long long pack_f32x2(float lo, float hi) {
-  return (unsigned long long)__float_as_uint(lo) | ((unsigned long long)__float_as_uint(hi) << 32);
+  unsigned long long d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void unpack_f32x2(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long sub_f32x2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 __device__ __forceinline__ unsigned long long add_f32x2(unsigned long long a, unsigned long long b) {
   unsigned long long d;
@@ -317,17 +327,21 @@ __device__ __forceinline__ void q8_0_block(const AppendParams& p, int64_t gblk, 
   const float rd = d != 0.0f ? __frcp_rn(d) : 0.0f;
   uint32_t code[8];
   bool near = false;
+  const unsigned long long rd2 = pack_f32x2(rd, rd), mg2 = pack_f32x2(kMagic, kMagic);
 #pragma unroll
   for (int w = 0; w < 8; ++w) {
-    uint32_t s4[4];
+    float s4[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float t = __fmul_rn(block_elem(raw, 4 * w + i), rd);
-      const float s = __fadd_rn(t, kMagic);
-      near |= fabsf(__fsub_rn(t, __fsub_rn(s, kMagic))) >= 0.49993896484375f;  // 0.5 - 2^-14
-      s4[i] = __float_as_uint(s);
+    for (int i = 0; i < 4; i += 2) {  // two elements per packed operation, the same roundings
+      const unsigned long long t2 = mul_f32x2(pack_f32x2(block_elem(raw, 4 * w + i), block_elem(raw, 4 * w + i + 1)), rd2);
+      const unsigned long long s2 = add_f32x2(t2, mg2);
+      float e0, e1;
+      unpack_f32x2(sub_f32x2(t2, sub_f32x2(s2, mg2)), e0, e1);
+      near |= fabsf(e0) >= 0.49993896484375f || fabsf(e1) >= 0.49993896484375f;  // 0.5 - 2^-14
+      unpack_f32x2(s2, s4[i], s4[i + 1]);
     }
-    code[w] = __byte_perm(__byte_perm(s4[0], s4[1], 0x0040), __byte_perm(s4[2], s4[3], 0x0040), 0x5410);
+    code[w] = __byte_perm(__byte_perm(__float_as_uint(s4[0]), __float_as_uint(s4[1]), 0x0040),
+                          __byte_perm(__float_as_uint(s4[2]), __float_as_uint(s4[3]), 0x0040), 0x5410);
   }
   if (near) {  // rare: some quotient is close to a tie
 #pragma unroll
@@ -553,32 +567,7 @@ __device__ __forceinline__ void append_turbo(const AppendParams& p, int64_t gtid
     float u[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) u[e] = 0.0f;
-    if constexpr (E % 2 == 0) {
-      if (pt != nullptr) {
-        // two outputs per packed binary32 pair operation (the same two roundings
-        // per term as the scalar loop below, lane by lane)
-        unsigned long long u2[E / 2];
-#pragma unroll
-        for (int k = 0; k < E / 2; ++k) u2[k] = 0ull;
-#pragma unroll 2
-        for (int jl = 0; jl < 32; ++jl) {
-#pragma unroll
-          for (int e2 = 0; e2 < E; ++e2) {
-            const float ej = __shfl_sync(0xffffffffu, res[e2], jl);
-            const unsigned long long* col =
-                reinterpret_cast<const unsigned long long*>(pt + (jl * E + e2) * D + lane * E);
-            const unsigned long long ej2 = pack_f32x2(ej, ej);
-#pragma unroll
-            for (int k = 0; k < E / 2; ++k) u2[k] = add_f32x2(u2[k], mul_f32x2(col[k], ej2));
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < E / 2; ++k) {
-          u[2 * k] = __uint_as_float((uint32_t)u2[k]);
-          u[2 * k + 1] = __uint_as_float((uint32_t)(u2[k] >> 32));
-        }
-      }
-    } else if (pt != nullptr) {
+    if (pt != nullptr) {
 #pragma unroll 2
       for (int jl = 0; jl < 32; ++jl) {
 #pragma unroll
