@@ -60,7 +60,10 @@ __device__ __forceinline__ uint4 load_raw(const AppendParams& p, int64_t gtid, i
 }
 
 // Packed binary32 pairs (low word: the first element), each lane rounded to
-// nearest like the scalar __fadd_rn / __fmul_rn.
+// nearest.  Used only where a stored bit does not hang on the last rounding
+// step: q8_0's tie test falls back to the exact divide near a tie.  (q4_0's
+// truncation, packed the same way, changed a nibble against the oracle, so it
+// keeps the scalar intrinsics.)
 __device__ __forceinline__ unsigned long long pack_f32x2(float lo, float hi) {
   unsigned long long d;
   asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
@@ -332,7 +335,7 @@ __device__ __forceinline__ void q8_0_block(const AppendParams& p, int64_t gblk, 
   for (int w = 0; w < 8; ++w) {
     float s4[4];
 #pragma unroll
-    for (int i = 0; i < 4; i += 2) {  // two elements per packed operation, the same roundings
+    for (int i = 0; i < 4; i += 2) {  // two elements per packed operation
       const unsigned long long t2 = mul_f32x2(pack_f32x2(block_elem(raw, 4 * w + i), block_elem(raw, 4 * w + i + 1)), rd2);
       const unsigned long long s2 = add_f32x2(t2, mg2);
       float e0, e1;
