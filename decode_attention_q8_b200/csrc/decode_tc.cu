@@ -112,30 +112,31 @@ bool decode_supported(int32_t k_type, int32_t v_type, int32_t G, int32_t D) {
 
 namespace {
 template <int KT>
-int ctas_k(int32_t v_type, int32_t D) {
+int ctas_k(int32_t v_type, int32_t D, int nth) {
   switch (v_type) {
-    case KVQ_F16: return tc::ctas_per_sm_for(KT, KVQ_F16, D);
-    case KVQ_Q8_0: return tc::ctas_per_sm_for(KT, KVQ_Q8_0, D);
-    case KVQ_Q4_0: return tc::ctas_per_sm_for(KT, KVQ_Q4_0, D);
-    case KVQ_Q5_0: return tc::ctas_per_sm_for(KT, KVQ_Q5_0, D);
-    case KVQ_TURBO2: return tc::ctas_per_sm_for(KT, KVQ_TURBO2, D);
-    case KVQ_TURBO3: return tc::ctas_per_sm_for(KT, KVQ_TURBO3, D);
-    case KVQ_TURBO4: return tc::ctas_per_sm_for(KT, KVQ_TURBO4, D);
+    case KVQ_F16: return tc::resident_ctas_for(KT, KVQ_F16, D, nth);
+    case KVQ_Q8_0: return tc::resident_ctas_for(KT, KVQ_Q8_0, D, nth);
+    case KVQ_Q4_0: return tc::resident_ctas_for(KT, KVQ_Q4_0, D, nth);
+    case KVQ_Q5_0: return tc::resident_ctas_for(KT, KVQ_Q5_0, D, nth);
+    case KVQ_TURBO2: return tc::resident_ctas_for(KT, KVQ_TURBO2, D, nth);
+    case KVQ_TURBO3: return tc::resident_ctas_for(KT, KVQ_TURBO3, D, nth);
+    case KVQ_TURBO4: return tc::resident_ctas_for(KT, KVQ_TURBO4, D, nth);
   }
   return 1;
 }
 }  // namespace
 
-int decode_ctas_per_sm(int32_t k_type, int32_t v_type, int32_t D) {
+int decode_ctas_per_sm(int32_t k_type, int32_t v_type, int32_t D, int32_t G) {
+  const int nth = G > 8 ? 2 : 1;  // query-head n-tiles of the instance
   switch (k_type) {
-    case KVQ_F16: return ctas_k<KVQ_F16>(v_type, D);
-    case KVQ_Q8_0: return ctas_k<KVQ_Q8_0>(v_type, D);
-    case KVQ_Q4_0: return ctas_k<KVQ_Q4_0>(v_type, D);
-    case KVQ_Q5_0: return ctas_k<KVQ_Q5_0>(v_type, D);
-    case KVQ_TURBO2: return ctas_k<KVQ_TURBO2>(v_type, D);
-    case KVQ_TURBO3: return ctas_k<KVQ_TURBO3>(v_type, D);
-    case KVQ_TURBO4: return ctas_k<KVQ_TURBO4>(v_type, D);
-    case KVQ_TURBO3_QJL: return ctas_k<KVQ_TURBO3_QJL>(v_type, D);
+    case KVQ_F16: return ctas_k<KVQ_F16>(v_type, D, nth);
+    case KVQ_Q8_0: return ctas_k<KVQ_Q8_0>(v_type, D, nth);
+    case KVQ_Q4_0: return ctas_k<KVQ_Q4_0>(v_type, D, nth);
+    case KVQ_Q5_0: return ctas_k<KVQ_Q5_0>(v_type, D, nth);
+    case KVQ_TURBO2: return ctas_k<KVQ_TURBO2>(v_type, D, nth);
+    case KVQ_TURBO3: return ctas_k<KVQ_TURBO3>(v_type, D, nth);
+    case KVQ_TURBO4: return ctas_k<KVQ_TURBO4>(v_type, D, nth);
+    case KVQ_TURBO3_QJL: return ctas_k<KVQ_TURBO3_QJL>(v_type, D, nth);
   }
   return 1;
 }

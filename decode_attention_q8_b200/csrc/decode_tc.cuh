@@ -141,6 +141,22 @@ __host__ __device__ constexpr int warps_for(int kt, int vt, int d) {
 __host__ __device__ constexpr int ctas_per_sm_for(int kt, int vt, int d) {
   return cta_smem(kt, vt, d, warps_for(kt, vt, d), 2) <= kSmemTwoCtas ? 2 : 1;
 }
+// Whether an instance is compiled for one resident CTA per SM (launch bounds
+// below): then it may use up to 255 registers a thread, and only as many CTAs
+// fit as 65536 registers allow -- one of 8 warps.
+__host__ __device__ constexpr bool one_cta_bound(int kt, int vt, int d, int nth) {
+  return d >= 256 || nth == 2 || ctas_per_sm_for(kt, vt, d) < 2;
+}
+// Resident CTAs per SM, by shared memory and by registers: the slots the host
+// sizes split counts and waiting combines for.
+__host__ __device__ constexpr int regs_ctas_for(int kt, int vt, int d) {
+  return 65536 / (warps_for(kt, vt, d) * 32 * 256) < 1 ? 1 : 65536 / (warps_for(kt, vt, d) * 32 * 256);
+}
+__host__ __device__ constexpr int resident_ctas_for(int kt, int vt, int d, int nth) {
+  return one_cta_bound(kt, vt, d, nth) && regs_ctas_for(kt, vt, d) < ctas_per_sm_for(kt, vt, d)
+             ? regs_ctas_for(kt, vt, d)
+             : ctas_per_sm_for(kt, vt, d);
+}
 __host__ __device__ constexpr int stages_for(int kt, int vt, int d) {
   return cta_smem(kt, vt, d, warps_for(kt, vt, d), 4) <= (ctas_per_sm_for(kt, vt, d) == 2 ? kSmemTwoCtas : kSmemOneCta)
              ? 4
@@ -405,7 +421,7 @@ struct TcArgs {
 // (a separate instantiation, so the contiguous kernel carries none of it).
 template <int KT, int VT, int NB, int NTH, bool PAGED>
 __global__ void __launch_bounds__(warps_for(KT, VT, NB * 32) * 32,
-                                  (NB >= 8 || NTH == 2 || ctas_per_sm_for(KT, VT, NB * 32) < 2) ? 1 : 2)
+                                  one_cta_bound(KT, VT, NB * 32, NTH) ? 1 : 2)
     decode_tc_kernel(const TcArgs args, const __grid_constant__ CUtensorMap tm_kc,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vc,
                      const __grid_constant__ CUtensorMap tm_vs) {

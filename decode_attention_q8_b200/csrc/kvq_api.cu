@@ -208,7 +208,7 @@ int64_t chunk_rows(int64_t ctx, int32_t S) { return round_up((ctx + S - 1) / S, 
 int32_t combining_ctas(const kvq_cache_desc* d, int32_t batch, int32_t S) {
   const int32_t G = d->n_q_heads / d->n_kv_heads;
   const int64_t groups = (int64_t)batch * d->n_kv_heads;
-  const int64_t slots = (int64_t)sm_count() * decode_ctas_per_sm(d->k_type, d->v_type, d->head_dim);
+  const int64_t slots = (int64_t)sm_count() * decode_ctas_per_sm(d->k_type, d->v_type, d->head_dim, G);
   if ((int64_t)G * S <= 200) return 1;
   int32_t k = (int32_t)std::min<int64_t>(G, (int64_t)G * S / 48);
   while (k > 1 && (int64_t)(k - 1) * groups * 2 > slots) --k;
@@ -219,7 +219,7 @@ int32_t combining_ctas(const kvq_cache_desc* d, int32_t batch, int32_t S) {
 // workspace for n_splits = 0).
 int32_t auto_splits_bound(const kvq_cache_desc* d, int32_t batch, int64_t ctx) {
   return choose_splits((int64_t)batch * d->n_kv_heads, ctx, sm_count(),
-                       decode_ctas_per_sm(d->k_type, d->v_type, d->head_dim));
+                       decode_ctas_per_sm(d->k_type, d->v_type, d->head_dim, d->n_q_heads / d->n_kv_heads));
 }
 
 // Explicit counts are used as given (trailing splits may be empty); the

@@ -159,7 +159,7 @@ cudaError_t launch_append(const AppendParams* k, int32_t k_type, const AppendPar
 cudaError_t launch_decode(int32_t k_type, int32_t v_type, const DecodeParams& p, cudaStream_t st);
 bool decode_supported(int32_t k_type, int32_t v_type, int32_t G, int32_t D);
 // Resident decode CTAs per SM (shared memory decides) that the split heuristic plans for.
-int decode_ctas_per_sm(int32_t k_type, int32_t v_type, int32_t D);
+int decode_ctas_per_sm(int32_t k_type, int32_t v_type, int32_t D, int32_t G);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t st);
 
 }  // namespace kvq
